@@ -1,0 +1,177 @@
+/*
+ * kvq.h -- C ABI of a B200 (sm_100a) library for decode attention over a transformed,
+ * percentile-clipped, affine-quantized 2/4-bit KV cache, and for the quantize-append
+ * step that fills that cache.
+ *
+ * The method (WUSH-KV, with AATC and NOVA-KV as related transform-coding work):
+ *  - "WUSH-KV: KV Cache Quantization with Data-Adaptive Transforms" (paperlayer
+ *    summary), section 1 and section 4.2: a dense d x d key transform per KV head is
+ *    applied after RoPE to every new key, and each query is compensated with T_k^{-T}
+ *    so that query-key products are preserved; a per-KV-head value transform is folded
+ *    into the projection weights on a real model (applied explicitly here), so the
+ *    attention output stays in the value-transform domain.
+ *  - same page, section 5.3 (downstream setup) and the abstract: OSCAR-style
+ *    percentile-clipped affine quantization of the transformed cache at 2 bits.
+ *  - same page, section 4.1: grouped-query attention; several query heads read one
+ *    KV head. Query head hq reads KV head hq / (Hq / Hkv).
+ *  - "Spend Bits Where Queries Look" (NOVA-KV project page), "Three requirements",
+ *    items 2 and 3: the cache is read at every decode step, and every token occupies
+ *    the same number of bits.
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers owned by the caller (allocated, e.g., by
+ *    PyTorch). The library allocates no memory and keeps no state between calls; it
+ *    is safe to call from several host threads on different streams.
+ *  - Work is enqueued on `stream` (NULL = the legacy default stream) and runs
+ *    asynchronously; pointers must stay valid until it completes.
+ *  - Argument errors are detected on the host before anything is launched and
+ *    return a kvq_status other than KVQ_OK. A failed launch returns KVQ_ERR_CUDA.
+ *    kvq_last_error() gives a one-line description (thread-local).
+ *  - Problems that depend on device data are never fatal: the kernels clamp or skip
+ *    and OR a bit into *dev_err (a device int32, nullable): see KVQ_DEVERR_*.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                        /* the CUDA runtime's cudaStream_t target */
+typedef struct CUstream_st *kvq_stream_t;  /* pass a cudaStream_t here */
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,   /* null pointer, inconsistent sizes or parameters */
+    KVQ_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels implement */
+    KVQ_ERR_CAPACITY = 3,      /* host-known length exceeds the cache capacity */
+    KVQ_ERR_WORKSPACE = 4,     /* workspace missing, too small or misaligned */
+    KVQ_ERR_CUDA = 5           /* a CUDA launch or query failed */
+} kvq_status;
+
+typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
+
+/* Bits in *dev_err (device int32, OR-ed, never cleared by the library). */
+#define KVQ_DEVERR_SEQLEN_CLAMPED 0x1   /* seqlens[b] < 0 or > max_seqlen: clamped */
+#define KVQ_DEVERR_POS_RANGE      0x2   /* pos[b] < 0 or pos[b] + n > T_cap: sequence skipped */
+#define KVQ_DEVERR_NONFINITE      0x4   /* a group had a non-finite clip range: codes 0 */
+#define KVQ_DEVERR_WAIT_TIMEOUT   0x8   /* a bounded pipeline wait gave up: output invalid */
+
+/*
+ * Quantizer parameters (WUSH-KV summary, section 5.3; percentile clipping).
+ * For a group of `group` consecutive dims of one token, with kappa = floor(clip_alpha *
+ * (group - 1)) computed in double on the host:
+ *   lo = x_(kappa), hi = x_(group-1-kappa)          order statistics, 0-indexed ascending
+ *   s  = f32(f32(hi - lo) / (2^bits - 1))           IEEE float32 division
+ *   s_h = f16_rn(s), z_h = f16_rn(lo)               stored as the pair (s_h, z_h)
+ *   c  = clamp(rint(f32(f32(x - z_h) / s_h)), 0, 2^bits - 1), rint ties-to-even;
+ *        s_h == 0 gives c = 0 for the whole group.
+ * Dequantization is x^ = z_h + c * s_h.
+ * Supported: bits_k, bits_v in {2, 4}; group divides d and is a multiple of 32;
+ * 0 <= kappa <= 8 and 2*kappa < group.
+ */
+typedef struct {
+    int bits_k;
+    int bits_v;
+    int group;
+    float clip_alpha;
+} kvq_qparams;
+
+/*
+ * Quantized cache (fixed width per token). Four caller-owned device planes:
+ *  k_codes [B][Hkv][T_cap][d*bits_k/8] bytes: one row per token, element j at bit
+ *          bits_k*j of the row (little-endian bit stream).
+ *  v_codes [B][Hkv][T_cap/16][16*d*bits_v/8] bytes: 16-token tiles laid out for the
+ *          P.V contraction. Tile = 32 lane chunks of d*bits_v/16 bytes; chunk L holds
+ *          tokens {t, t+4, t+8, t+12} (t = L % 4) at dims {8n + L/4}; inside it,
+ *          32-bit little-endian words, word p*W + r (W = d*bits_v/128, p = 0, 1)
+ *          holding token t+4p in its low 16 bits and token t+4p+8 in its high 16
+ *          bits, dim 8*(E*r + s) + L/4 at bit offset bits_v*s of the half (E = 16/bits_v).
+ *          Each token owns whole bytes, so single-token appends need no read-modify-write.
+ *  k_sz, v_sz [B][Hkv][T_cap][d/group] pairs of float16 (s_h, z_h), s_h first (4 bytes).
+ * T_cap must be a multiple of 64; d must be 64 or 128. All planes 16-byte aligned.
+ * qp must equal the parameters passed to kvq_quantize_append.
+ */
+typedef struct {
+    int B;
+    int Hkv;
+    int T_cap;
+    int d;
+    kvq_qparams qp;
+    void *k_codes;
+    void *k_sz;
+    void *v_codes;
+    void *v_sz;
+} kvq_cache;
+
+/* Size in bytes of plane `which` (0 k_codes, 1 k_sz, 2 v_codes, 3 v_sz); 0 if invalid. */
+size_t kvq_cache_plane_bytes(const kvq_cache *cache, int which);
+
+/*
+ * Write path: transform, clip, quantize and append n new tokens per sequence.
+ * (WUSH-KV summary, section 4.2: key transform after RoPE, value transform; section 5.3:
+ * percentile-clipped affine quantizer; NOVA-KV page, item 3: fixed-width store.)
+ *   k_post_rope, v: [B][n][Hkv][d] in_dtype (float32 or bfloat16), post-RoPE keys and values.
+ *   T_k, T_v: [Hkv][d][d] float32 row-major, x~_i = sum_j T[i][j] x_j; NULL = identity.
+ *   qp: must equal cache->qp.  pos: device int32 [B], first position written per sequence.
+ *   n >= 0 tokens per sequence (n == 0 is a no-op). Token i of sequence b goes to position
+ *   pos[b] + i; a sequence whose range leaves [0, T_cap) is skipped and flagged in dev_err.
+ * The transformed values are computed in float32 (fused multiply-add); for identical
+ * transformed inputs the codes, scales and zero-points equal the float64 definition
+ * above bit for bit.
+ */
+kvq_status kvq_quantize_append(const void *k_post_rope, const void *v, kvq_dtype in_dtype,
+                               const float *T_k, const float *T_v, const kvq_qparams *qp,
+                               kvq_cache *cache, const int32_t *pos, int n, int32_t *dev_err,
+                               kvq_stream_t stream);
+
+/* Workspace bytes kvq_decode_attention needs for this cache shape, Hq query heads and
+ * sequences of at most max_seqlen tokens (0 if the arguments are invalid). */
+size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int Hq, int max_seqlen);
+
+/*
+ * Read path: one decode step of grouped-query attention over the quantized cache.
+ * (WUSH-KV summary, sections 1, 4.1, 4.2; NOVA-KV page, "Three requirements" item 2.)
+ *   q: [B][Hq][d] q_dtype (float32 or bfloat16), post-RoPE queries; Hq % Hkv == 0.
+ *   Tk_invT: [Hkv][d][d] float32 row-major, M = T_k^{-T}; q~ = M q (NULL = identity).
+ *   seqlens: device int32 [B], tokens attended per sequence (0..max_seqlen; positions
+ *            [0, seqlens[b]) must hold appended tokens). max_seqlen <= T_cap.
+ *   out: [B][Hq][d] out_dtype: softmax_t(q~ . k^_t / sqrt(d)) v^_t, in the value-transform
+ *        domain; 0 for an empty sequence.
+ *   workspace: device buffer of at least kvq_decode_workspace_bytes(...) bytes,
+ *              256-byte aligned, used as scratch (contents need not be initialised).
+ * Computed as a split-K flash decode: scores and P.V on tensor cores with float32
+ * accumulation, float32 online softmax, then a merge of the splits.
+ */
+kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const float *Tk_invT,
+                                const kvq_cache *cache, const int32_t *seqlens, int max_seqlen,
+                                void *out, kvq_dtype out_dtype, void *workspace,
+                                size_t ws_bytes, int32_t *dev_err, kvq_stream_t stream);
+
+/* Workspace bytes kvq_bf16_decode needs (0 if the arguments are invalid). */
+size_t kvq_bf16_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seqlen);
+
+/*
+ * Uncompressed comparator: the same decode attention over bfloat16 keys and values
+ * [B][Hkv][T_cap][d] (no transform, no quantization); q, out [B][Hq][d] bfloat16.
+ * d in {64, 128}; T_cap a multiple of 64. Same workspace and error conventions.
+ */
+kvq_status kvq_bf16_decode(const void *q, int Hq, const void *k, const void *v, int B, int Hkv,
+                           int T_cap, int d, const int32_t *seqlens, int max_seqlen, void *out,
+                           void *workspace, size_t ws_bytes, int32_t *dev_err,
+                           kvq_stream_t stream);
+
+/* Static description of a status code. */
+const char *kvq_status_string(kvq_status status);
+
+/* Detail of the last non-OK status returned on this host thread ("" if none). */
+const char *kvq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -201,10 +201,10 @@ void oracle_quantize_group(const float *x, int g, int bits, int kappa,
  *   bk*j of the row (byte floor(bk*j/8), bit bk*j mod 8, little-endian).
  * V codes plane, [B][Hkv][T_cap/16][16*d*bv/8] bytes: tiles of 16 tokens. A tile is
  *   32 lane chunks of 2*d*bv/32 bytes. Lane L = 4*gq + tq holds tokens
- *   {2tq, 2tq+1, 2tq+8, 2tq+9} x dims {8n + gq}. Inside a chunk, 32-bit little-endian
+ *   {tq, tq+4, tq+8, tq+12} x dims {8n + gq}. Inside a chunk, 32-bit little-endian
  *   words; with E = 16/bv codes per 16-bit half and W = d/(8E) words per token pair,
- *   word p*W + r (p = token/8) holds, in its low half, token 2tq+8p and, in its high
- *   half, token 2tq+1+8p; half slot s (bits bv*s) holds dim 8*(E*r + s) + gq.
+ *   word p*W + r holds, in its low half, token tq+4p and, in its high half, token
+ *   tq+4p+8; half slot s (bits bv*s) holds dim 8*(E*r + s) + gq.
  * Scale/zero planes, [B][Hkv][T_cap][d/group] x 2 float16: (s, z) pairs, s first.
  */
 size_t oracle_k_row_bytes(int d, int bits) { return (size_t)d * bits / 8; }
@@ -223,8 +223,7 @@ void oracle_v_code_pos(int d, int bits, int tok, int j, size_t *byte, int *bit)
     int W = d / (8 * E);
     int chunk = 2 * d * bits / 32;                    /* bytes per lane chunk */
     int n = j / 8, gq = j % 8;
-    int tm = tok % 8, p = tok / 8;
-    int tq = tm / 2, hi = tm % 2;
+    int tq = tok % 4, p = (tok / 4) % 2, hi = tok / 8;
     int lane = 4 * gq + tq;
     int r = n / E, s = n % E;
     int word = p * W + r;

@@ -52,7 +52,7 @@ def test_v_tile_hand_derived_positions():
     for d, bits, tok, dim, byte, bit in _rows("v_tile_positions.txt"):
         assert oracle.v_code_pos(int(d), int(bits), int(tok), int(dim)) == (int(byte), int(bit))
         n += 1
-    assert n == 13
+    assert n == 14
 
 
 def test_bits_per_element_matches_pages():
