@@ -562,12 +562,12 @@ int oracle_decode(const void *q, int q_dtype, int B, int Hq, int Hkv, int d, con
     for (int u = 0; u < npairs; ++u) {
         int b = sel ? sel[2 * u] : u / Hq, hq = sel ? sel[2 * u + 1] : u % Hq;
         int G = Hq / Hkv;
-        double qt[1024], m, l;
-        double *o = out + ((size_t)b * Hq + hq) * d;
+        double qt[1024], o[1024], m, l;
         query_transform(q, q_dtype, M, Hq, Hkv, d, b, hq, qt);
         attend_range(&c, qt, b, hq / G, 0, seqlens[b], &m, &l, o);
+        /* accumulate privately, store once: a pair listed twice in sel is still safe */
         for (int j = 0; j < d; ++j)
-            o[j] = l > 0 ? o[j] / l : 0.0;
+            out[((size_t)b * Hq + hq) * d + j] = l > 0 ? o[j] / l : 0.0;
     }
     return 0;
 }
@@ -631,8 +631,7 @@ int oracle_bf16_decode(const uint16_t *q, int B, int Hq, int Hkv, int d,
         int b = sel ? sel[2 * u] : u / Hq, hq = sel ? sel[2 * u + 1] : u % Hq;
         int h = hq / (Hq / Hkv), n = seqlens[b];
         double sm = 1.0 / sqrt((double)d);
-        double qv[1024];
-        double *o = out + ((size_t)b * Hq + hq) * d;
+        double qv[1024], o[1024];
         double *logit = (double *)malloc(sizeof(double) * (n > 0 ? n : 1));
         for (int j = 0; j < d; ++j)
             qv[j] = oracle_bf16_to_f64(q[((size_t)b * Hq + hq) * d + j]);
@@ -657,7 +656,7 @@ int oracle_bf16_decode(const uint16_t *q, int B, int Hq, int Hkv, int d,
                 o[j] += p * oracle_bf16_to_f64(vr[j]);
         }
         for (int j = 0; j < d; ++j)
-            o[j] = l > 0 ? o[j] / l : 0.0;
+            out[((size_t)b * Hq + hq) * d + j] = l > 0 ? o[j] / l : 0.0;
         free(logit);
     }
     return 0;

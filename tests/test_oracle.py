@@ -386,7 +386,7 @@ def test_sampled_heads_equal_full_decode():
     q = np.random.default_rng(2).standard_normal((2, 4, 128)).astype(np.float32)
     seql = np.array([64, 33], np.int32)
     full = oracle.decode(q, None, c, seql)
-    sel = np.array([[1, 3], [0, 2]], np.int32)
+    sel = np.array([[1, 3], [0, 2], [1, 3], [1, 3], [0, 2]], np.int32)   # duplicates allowed
     part = oracle.decode(q, None, c, seql, sel=sel)
     for b, h in sel:
         assert np.array_equal(part[b, h], full[b, h])
