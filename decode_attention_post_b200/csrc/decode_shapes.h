@@ -1,0 +1,50 @@
+// Launch-time shapes shared by the decode kernels and the host-side C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kvq {
+
+constexpr int kDecodeWarps = 4;     // warps per decode CTA
+constexpr int kDecodeStages = 3;    // bulk-copy ring depth per warp
+constexpr int kDecodeBlock = 64;    // tokens per ring stage
+
+struct DecodeParams {
+    const uint8_t *k_codes;
+    const uint32_t *k_sz;
+    const uint8_t *v_codes;
+    const uint32_t *v_sz;
+    const int32_t *seqlens;
+    int B, Hkv, Hq, T_cap, max_seqlen;
+    int nsplit;          // CTAs per (sequence, KV head) along the tokens
+    int split_tokens;    // tokens per split, a multiple of kDecodeBlock
+    const uint32_t *qfrag;
+    const float *qscale;
+    const float *qw;
+    float *part;
+    int *ticket;
+    void *out;
+    int out_bf16;
+    int32_t *dev_err;
+};
+
+struct DecodeLaunch {
+    DecodeParams p;
+    const void *q;
+    int q_bf16;
+    const float *M;
+    int d, G, bits_k, bits_v;
+    int qprep_bb;        // sequences per q-prologue CTA
+};
+
+// Byte offsets of the decode workspace sections (each 256-byte aligned).
+struct DecodeWorkspace {
+    size_t qfrag, qscale, qw, part, ticket, total;
+};
+
+size_t decode_qfrag_words(int d, int G);
+cudaError_t launch_decode(const DecodeLaunch &L, cudaStream_t st);
+
+}  // namespace kvq

@@ -1,0 +1,343 @@
+// Host side of the C ABI declared in include/kvq.h: argument validation, workspace
+// sizing, split selection and kernel dispatch. Nothing here allocates device memory.
+#include "kvq_common.cuh"
+#include "decode_shapes.h"
+
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+namespace kvq {
+
+cudaError_t append_fp32(const void *k, const void *v, int in_bf16, const float *Tk,
+                        const float *Tv, int B, int n, const kvq_cache *c, int kappa,
+                        const int32_t *pos, int32_t *dev_err, cudaStream_t st);
+cudaError_t launch_bf16_decode(const void *q, int Hq, const void *k, const void *v, int B,
+                               int Hkv, int T_cap, int d, const int32_t *seqlens, int max_seqlen,
+                               void *out, void *ws, int nsplit, int split_tokens,
+                               int32_t *dev_err, cudaStream_t st);
+
+static thread_local char g_last_error[512];
+
+void set_error(const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+}
+
+static bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+static int kappa_of(float alpha, int group)
+{
+    double k = floor((double)alpha * (double)(group - 1));
+    return k < 0 ? 0 : (int)k;
+}
+
+static kvq_status check_qparams(const kvq_qparams *qp, int d)
+{
+    if (!qp)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "qparams is NULL");
+    if ((qp->bits_k != 2 && qp->bits_k != 4) || (qp->bits_v != 2 && qp->bits_v != 4))
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "bits_k=%d bits_v=%d: only 2 and 4 are implemented",
+                 qp->bits_k, qp->bits_v);
+    if (qp->group <= 0 || d % qp->group || qp->group % 32)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "group=%d must divide d=%d and be a multiple of 32",
+                 qp->group, d);
+    if (!(qp->clip_alpha >= 0.f) || !(qp->clip_alpha < 0.5f))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "clip_alpha=%g must be in [0, 0.5)", (double)qp->clip_alpha);
+    const int kap = kappa_of(qp->clip_alpha, qp->group);
+    if (2 * kap >= qp->group)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "clip index %d leaves no range in a group of %d", kap,
+                 qp->group);
+    if (kap > 8)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "clip index %d > 8 is not implemented", kap);
+    return KVQ_OK;
+}
+
+static kvq_status check_cache(const kvq_cache *c)
+{
+    if (!c)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (c->B <= 0 || c->Hkv <= 0 || c->T_cap <= 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "cache B=%d Hkv=%d T_cap=%d must be positive", c->B, c->Hkv,
+                 c->T_cap);
+    if (c->T_cap % kCapAlign)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "T_cap=%d must be a multiple of %d", c->T_cap, kCapAlign);
+    if (c->d != 64 && c->d != 128)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "d=%d: only 64 and 128 are implemented", c->d);
+    kvq_status s = check_qparams(&c->qp, c->d);
+    if (s != KVQ_OK)
+        return s;
+    if (!c->k_codes || !c->k_sz || !c->v_codes || !c->v_sz)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "a cache plane pointer is NULL");
+    if (!aligned(c->k_codes, 16) || !aligned(c->k_sz, 16) || !aligned(c->v_codes, 16) ||
+        !aligned(c->v_sz, 16))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "cache planes must be 16-byte aligned");
+    return KVQ_OK;
+}
+
+static bool same_qp(const kvq_qparams *a, const kvq_qparams *b)
+{
+    return a->bits_k == b->bits_k && a->bits_v == b->bits_v && a->group == b->group &&
+           a->clip_alpha == b->clip_alpha;
+}
+
+static int num_sms()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return sms;
+}
+
+// Splits along the tokens so that about 4 waves of 3 resident CTAs per SM cover the
+// (sequence, KV head) pairs; each split is a whole number of 64-token blocks.
+// KVQ_DECODE_SPLITS overrides the count (tuning).
+static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens)
+{
+    const int blocks = max_seqlen > 0 ? (max_seqlen + kDecodeBlock - 1) / kDecodeBlock : 1;
+    const long pairs = (long)B * Hkv;
+    const long target = (long)num_sms() * 3 * 4;
+    long ns = (target + pairs - 1) / pairs;
+    if (const char *e = getenv("KVQ_DECODE_SPLITS"))
+        ns = atol(e);
+    if (ns < 1)
+        ns = 1;
+    if (ns > blocks)
+        ns = blocks;
+    const int bps = (int)((blocks + ns - 1) / ns);
+    *split_tokens = bps * kDecodeBlock;
+    return (blocks + bps - 1) / bps;
+}
+
+static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static DecodeWorkspace decode_layout(int B, int Hkv, int Hq, int d, int nsplit)
+{
+    const int G = Hq / Hkv;
+    DecodeWorkspace w;
+    size_t off = 0;
+    w.qfrag = off;
+    off += up256((size_t)B * Hkv * decode_qfrag_words(d, G) * 4);
+    w.qscale = off;
+    off += up256((size_t)B * Hkv * 4);
+    w.qw = off;
+    off += up256((size_t)B * Hq * 4);
+    w.part = off;
+    off += up256((size_t)B * Hkv * nsplit * G * (d + 2) * 4);
+    w.ticket = off;
+    off += up256((size_t)B * Hkv * 4);
+    w.total = off;
+    return w;
+}
+
+static kvq_status check_decode_shape(const kvq_cache *c, int Hq, int max_seqlen)
+{
+    kvq_status s = check_cache(c);
+    if (s != KVQ_OK)
+        return s;
+    if (Hq <= 0 || Hq % c->Hkv)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d", Hq, c->Hkv);
+    const int G = Hq / c->Hkv;
+    if (G != 4 && G != 8)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "query heads per KV head G=%d: 4 and 8 are implemented", G);
+    if (c->qp.group != c->d)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "decode implements group == d (got group=%d, d=%d)",
+                 c->qp.group, c->d);
+    if (max_seqlen < 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "max_seqlen=%d is negative", max_seqlen);
+    if (max_seqlen > c->T_cap)
+        KVQ_FAIL(KVQ_ERR_CAPACITY, "max_seqlen=%d exceeds T_cap=%d", max_seqlen, c->T_cap);
+    return KVQ_OK;
+}
+
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+const char *kvq_status_string(kvq_status s)
+{
+    switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "cache capacity exceeded";
+    case KVQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case KVQ_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char *kvq_last_error(void) { return g_last_error; }
+
+size_t kvq_cache_plane_bytes(const kvq_cache *c, int which)
+{
+    if (!c || c->B <= 0 || c->Hkv <= 0 || c->T_cap <= 0 || c->d <= 0 || c->qp.group <= 0 ||
+        c->d % c->qp.group)
+        return 0;
+    const size_t tok = (size_t)c->B * c->Hkv * c->T_cap;
+    switch (which) {
+    case 0: return tok * c->d * c->qp.bits_k / 8;
+    case 1: return tok * (c->d / c->qp.group) * 4;
+    case 2: return tok * c->d * c->qp.bits_v / 8;
+    case 3: return tok * (c->d / c->qp.group) * 4;
+    }
+    return 0;
+}
+
+kvq_status kvq_quantize_append(const void *k, const void *v, kvq_dtype in_dtype, const float *T_k,
+                               const float *T_v, const kvq_qparams *qp, kvq_cache *cache,
+                               const int32_t *pos, int n, int32_t *dev_err, kvq_stream_t stream)
+{
+    g_last_error[0] = 0;
+    kvq_status s = check_cache(cache);
+    if (s != KVQ_OK)
+        return s;
+    s = check_qparams(qp, cache->d);
+    if (s != KVQ_OK)
+        return s;
+    if (!same_qp(qp, &cache->qp))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "qparams differ from the cache's qparams");
+    if (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "in_dtype=%d is not KVQ_F32 or KVQ_BF16", (int)in_dtype);
+    if (n < 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "n=%d is negative", n);
+    if (n > cache->T_cap)
+        KVQ_FAIL(KVQ_ERR_CAPACITY, "n=%d exceeds T_cap=%d", n, cache->T_cap);
+    if (n == 0)
+        return KVQ_OK;
+    if (!k || !v || !pos)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "k, v and pos must not be NULL");
+    cudaError_t e = append_fp32(k, v, in_dtype == KVQ_BF16, T_k, T_v, cache->B, n, cache,
+                                kappa_of(qp->clip_alpha, qp->group), pos, dev_err,
+                                (cudaStream_t)stream);
+    if (e != cudaSuccess)
+        KVQ_FAIL(KVQ_ERR_CUDA, "append launch: %s", cudaGetErrorString(e));
+    return KVQ_OK;
+}
+
+size_t kvq_decode_workspace_bytes(const kvq_cache *c, int Hq, int max_seqlen)
+{
+    if (check_decode_shape(c, Hq, max_seqlen) != KVQ_OK)
+        return 0;
+    int split_tokens = 0;
+    const int ns = choose_splits(c->B, c->Hkv, max_seqlen, &split_tokens);
+    return decode_layout(c->B, c->Hkv, Hq, c->d, ns).total;
+}
+
+kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const float *Tk_invT,
+                                const kvq_cache *c, const int32_t *seqlens, int max_seqlen,
+                                void *out, kvq_dtype out_dtype, void *workspace, size_t ws_bytes,
+                                int32_t *dev_err, kvq_stream_t stream)
+{
+    g_last_error[0] = 0;
+    kvq_status s = check_decode_shape(c, Hq, max_seqlen);
+    if (s != KVQ_OK)
+        return s;
+    if (!q || !seqlens || !out)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "q, seqlens and out must not be NULL");
+    if ((q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) ||
+        (out_dtype != KVQ_F32 && out_dtype != KVQ_BF16))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "q_dtype/out_dtype must be KVQ_F32 or KVQ_BF16");
+    int split_tokens = 0;
+    const int ns = choose_splits(c->B, c->Hkv, max_seqlen, &split_tokens);
+    const DecodeWorkspace w = decode_layout(c->B, c->Hkv, Hq, c->d, ns);
+    if (!workspace || !aligned(workspace, 256))
+        KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
+    if (ws_bytes < w.total)
+        KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, w.total);
+    unsigned char *ws = (unsigned char *)workspace;
+    DecodeLaunch L;
+    L.p.k_codes = (const uint8_t *)c->k_codes;
+    L.p.k_sz = (const uint32_t *)c->k_sz;
+    L.p.v_codes = (const uint8_t *)c->v_codes;
+    L.p.v_sz = (const uint32_t *)c->v_sz;
+    L.p.seqlens = seqlens;
+    L.p.B = c->B;
+    L.p.Hkv = c->Hkv;
+    L.p.Hq = Hq;
+    L.p.T_cap = c->T_cap;
+    L.p.max_seqlen = max_seqlen;
+    L.p.nsplit = ns;
+    L.p.split_tokens = split_tokens;
+    L.p.qfrag = (const uint32_t *)(ws + w.qfrag);
+    L.p.qscale = (const float *)(ws + w.qscale);
+    L.p.qw = (const float *)(ws + w.qw);
+    L.p.part = (float *)(ws + w.part);
+    L.p.ticket = (int *)(ws + w.ticket);
+    L.p.out = out;
+    L.p.out_bf16 = out_dtype == KVQ_BF16;
+    L.p.dev_err = dev_err;
+    L.q = q;
+    L.q_bf16 = q_dtype == KVQ_BF16;
+    L.M = Tk_invT;
+    L.d = c->d;
+    L.G = Hq / c->Hkv;
+    L.bits_k = c->qp.bits_k;
+    L.bits_v = c->qp.bits_v;
+    L.qprep_bb = 2;
+    cudaError_t e = launch_decode(L, (cudaStream_t)stream);
+    if (e != cudaSuccess)
+        KVQ_FAIL(KVQ_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return KVQ_OK;
+}
+
+size_t kvq_bf16_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seqlen)
+{
+    if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv || (d != 64 && d != 128) || max_seqlen < 0)
+        return 0;
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8)
+        return 0;
+    int split_tokens = 0;
+    const int ns = choose_splits(B, Hkv, max_seqlen, &split_tokens);
+    return up256((size_t)B * Hkv * ns * G * (d + 2) * 4) + up256((size_t)B * Hkv * 4);
+}
+
+kvq_status kvq_bf16_decode(const void *q, int Hq, const void *k, const void *v, int B, int Hkv,
+                           int T_cap, int d, const int32_t *seqlens, int max_seqlen, void *out,
+                           void *workspace, size_t ws_bytes, int32_t *dev_err, kvq_stream_t stream)
+{
+    g_last_error[0] = 0;
+    if (!q || !k || !v || !seqlens || !out)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "q, k, v, seqlens and out must not be NULL");
+    if (B <= 0 || Hkv <= 0 || T_cap <= 0 || Hq <= 0 || Hq % Hkv)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "bad shape B=%d Hq=%d Hkv=%d T_cap=%d", B, Hq, Hkv, T_cap);
+    if (T_cap % kCapAlign)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "T_cap=%d must be a multiple of %d", T_cap, kCapAlign);
+    if (d != 64 && d != 128)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "d=%d: only 64 and 128 are implemented", d);
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "query heads per KV head G=%d: 4 and 8 are implemented", G);
+    if (max_seqlen < 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "max_seqlen=%d is negative", max_seqlen);
+    if (max_seqlen > T_cap)
+        KVQ_FAIL(KVQ_ERR_CAPACITY, "max_seqlen=%d exceeds T_cap=%d", max_seqlen, T_cap);
+    if (!aligned(k, 16) || !aligned(v, 16))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "k and v must be 16-byte aligned");
+    const size_t need = kvq_bf16_decode_workspace_bytes(B, Hq, Hkv, d, max_seqlen);
+    if (!workspace || !aligned(workspace, 256))
+        KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
+    if (ws_bytes < need)
+        KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
+    int split_tokens = 0;
+    const int ns = choose_splits(B, Hkv, max_seqlen, &split_tokens);
+    cudaError_t e = launch_bf16_decode(q, Hq, k, v, B, Hkv, T_cap, d, seqlens, max_seqlen, out,
+                                       workspace, ns, split_tokens, dev_err, (cudaStream_t)stream);
+    if (e != cudaSuccess)
+        KVQ_FAIL(KVQ_ERR_CUDA, "bf16 decode launch: %s", cudaGetErrorString(e));
+    return KVQ_OK;
+}
+
+}  // extern "C"

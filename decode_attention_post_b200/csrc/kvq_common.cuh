@@ -1,0 +1,52 @@
+// Shared device/host helpers of the kvq CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kTileTokens = 16;      // V codes are stored in 16-token tiles
+constexpr int kCapAlign = 64;        // T_cap granularity (whole decode blocks)
+
+// Bits of the device error word (see kvq.h).
+__device__ __forceinline__ void flag(int32_t *dev_err, int32_t bit)
+{
+    if (dev_err)
+        atomicOr(dev_err, bit);
+}
+
+__device__ __forceinline__ float load_in(const void *p, int bf16, size_t i)
+{
+    if (bf16)
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+    return reinterpret_cast<const float *>(p)[i];
+}
+
+// Byte offset, inside a 16-token V tile, of the 16-bit half that holds token `tok`
+// (0..15) at the dims {8*(E*r + s) + gq : s < E}. Lane chunk 4*gq + tq holds tokens
+// {tq, tq+4, tq+8, tq+12}; word p*W + r holds token tq+4p (low half) and tq+4p+8 (high).
+__host__ __device__ __forceinline__ int v_half_offset(int d, int bits, int tok, int gq, int r)
+{
+    const int E = 16 / bits;
+    const int W = d / (8 * E);
+    const int chunk = d * bits / 16;
+    const int tq = tok & 3, p = (tok >> 2) & 1, hi = tok >> 3;
+    const int lane = 4 * gq + tq;
+    return lane * chunk + (p * W + r) * 4 + 2 * hi;
+}
+
+// Host-side: thread-local last error text.
+void set_error(const char *fmt, ...);
+
+}  // namespace kvq
+
+#define KVQ_FAIL(code, ...)                 \
+    do {                                    \
+        ::kvq::set_error(__VA_ARGS__);      \
+        return code;                        \
+    } while (0)

@@ -1,0 +1,232 @@
+"""ctypes binding of include/kvq.h. Argument marshalling only.
+
+Every function takes torch tensors that already live on a CUDA device (the caller owns
+them), checks dtype/shape/contiguity, and calls the C entry point of the same name on
+the current CUDA stream (or the stream given). A non-OK status raises KvqError with the
+library's own message. If ``libkvq.so`` is missing the first call raises: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import dataclasses
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libkvq.so")
+_lib = None
+
+KVQ_F32, KVQ_BF16 = 0, 1
+KVQ_DEVERR_SEQLEN_CLAMPED = 0x1
+KVQ_DEVERR_POS_RANGE = 0x2
+KVQ_DEVERR_NONFINITE = 0x4
+KVQ_DEVERR_WAIT_TIMEOUT = 0x8
+
+_P, _I, _F, _S = C.c_void_p, C.c_int, C.c_float, C.c_size_t
+
+
+class _QParams(C.Structure):
+    _fields_ = [("bits_k", _I), ("bits_v", _I), ("group", _I), ("clip_alpha", _F)]
+
+
+class _Cache(C.Structure):
+    _fields_ = [("B", _I), ("Hkv", _I), ("T_cap", _I), ("d", _I), ("qp", _QParams),
+                ("k_codes", _P), ("k_sz", _P), ("v_codes", _P), ("v_sz", _P)]
+
+
+class KvqError(RuntimeError):
+    def __init__(self, status: int, func: str, detail: str):
+        self.status = status
+        super().__init__(f"{func}: status {status}: {detail}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libkvq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m decode_attention_post_b200.build`")
+    L = C.CDLL(_LIB_PATH)
+    L.kvq_status_string.restype = C.c_char_p
+    L.kvq_status_string.argtypes = [_I]
+    L.kvq_last_error.restype = C.c_char_p
+    L.kvq_cache_plane_bytes.restype = _S
+    L.kvq_cache_plane_bytes.argtypes = [C.POINTER(_Cache), _I]
+    L.kvq_quantize_append.restype = _I
+    L.kvq_quantize_append.argtypes = [_P, _P, _I, _P, _P, C.POINTER(_QParams), C.POINTER(_Cache),
+                                      _P, _I, _P, _P]
+    L.kvq_decode_workspace_bytes.restype = _S
+    L.kvq_decode_workspace_bytes.argtypes = [C.POINTER(_Cache), _I, _I]
+    L.kvq_decode_attention.restype = _I
+    L.kvq_decode_attention.argtypes = [_P, _I, _I, _P, C.POINTER(_Cache), _P, _I, _P, _I, _P, _S,
+                                       _P, _P]
+    L.kvq_bf16_decode_workspace_bytes.restype = _S
+    L.kvq_bf16_decode_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+    L.kvq_bf16_decode.restype = _I
+    L.kvq_bf16_decode.argtypes = [_P, _I, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _S, _P, _P]
+    _lib = L
+    return L
+
+
+def _check(status: int, func: str):
+    if status != 0:
+        L = load()
+        raise KvqError(status, func, L.kvq_last_error().decode() or
+                       L.kvq_status_string(status).decode())
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _dt(t) -> int:
+    if t.dtype == torch.float32:
+        return KVQ_F32
+    if t.dtype == torch.bfloat16:
+        return KVQ_BF16
+    raise TypeError(f"expected float32 or bfloat16, got {t.dtype}")
+
+
+def _cuda(name, t, dtype=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+@dataclasses.dataclass(frozen=True)
+class QParams:
+    bits_k: int = 2
+    bits_v: int = 2
+    group: int = 128
+    clip_alpha: float = 0.01
+
+    def _c(self):
+        return _QParams(self.bits_k, self.bits_v, self.group, self.clip_alpha)
+
+
+class KVCache:
+    """The four cache planes (caller-owned device memory) plus their shape.
+
+    ``KVCache.allocate`` asks the library for each plane's size and allocates it with
+    torch; ``KVCache(planes=...)`` wraps existing uint8 tensors.
+    """
+
+    def __init__(self, B, Hkv, T_cap, d, qp: QParams, planes):
+        self.B, self.Hkv, self.T_cap, self.d, self.qp = B, Hkv, T_cap, d, qp
+        self.k_codes, self.k_sz, self.v_codes, self.v_sz = planes
+        for name, t in zip(("k_codes", "k_sz", "v_codes", "v_sz"), planes):
+            _cuda(name, t, torch.uint8)
+        self._desc = _Cache(B, Hkv, T_cap, d, qp._c(), _ptr(self.k_codes), _ptr(self.k_sz),
+                            _ptr(self.v_codes), _ptr(self.v_sz))
+
+    @staticmethod
+    def plane_bytes(B, Hkv, T_cap, d, qp: QParams):
+        desc = _Cache(B, Hkv, T_cap, d, qp._c(), None, None, None, None)
+        return [int(load().kvq_cache_plane_bytes(C.byref(desc), w)) for w in range(4)]
+
+    @classmethod
+    def allocate(cls, B, Hkv, T_cap, d, qp: QParams, device="cuda", zero=True):
+        sizes = cls.plane_bytes(B, Hkv, T_cap, d, qp)
+        if min(sizes) <= 0:
+            raise ValueError("invalid cache shape")
+        make = torch.zeros if zero else torch.empty
+        planes = [make(n, dtype=torch.uint8, device=device) for n in sizes]
+        return cls(B, Hkv, T_cap, d, qp, planes)
+
+    def view_sequence(self, b: int) -> "KVCache":
+        """The same cache restricted to sequence b (a B = 1 view of its planes)."""
+        per = [p.numel() // self.B for p in (self.k_codes, self.k_sz, self.v_codes, self.v_sz)]
+        planes = [p[b * n:(b + 1) * n] for p, n in zip((self.k_codes, self.k_sz, self.v_codes,
+                                                         self.v_sz), per)]
+        return KVCache(1, self.Hkv, self.T_cap, self.d, self.qp, planes)
+
+    @property
+    def desc(self):
+        return self._desc
+
+    def nbytes(self):
+        return sum(p.numel() for p in (self.k_codes, self.k_sz, self.v_codes, self.v_sz))
+
+
+def cache_plane_bytes(cache: KVCache, which: int) -> int:
+    return int(load().kvq_cache_plane_bytes(C.byref(cache.desc), which))
+
+
+def quantize_append(k_post_rope, v, T_k, T_v, qp: QParams, cache: KVCache, pos, n=None,
+                    dev_err=None, stream=None):
+    """kvq_quantize_append: k, v [B][n][Hkv][d] float32/bfloat16; T_k, T_v [Hkv][d][d]
+    float32 or None; pos int32 [B] on the device."""
+    L = load()
+    _cuda("k_post_rope", k_post_rope)
+    _cuda("v", v, k_post_rope.dtype)
+    _cuda("T_k", T_k, torch.float32)
+    _cuda("T_v", T_v, torch.float32)
+    _cuda("pos", pos, torch.int32)
+    _cuda("dev_err", dev_err, torch.int32)
+    if n is None:
+        n = k_post_rope.shape[1]
+    qpc = qp._c()
+    _check(L.kvq_quantize_append(_ptr(k_post_rope), _ptr(v), _dt(k_post_rope), _ptr(T_k),
+                                 _ptr(T_v), C.byref(qpc), C.byref(cache.desc), _ptr(pos), int(n),
+                                 _ptr(dev_err), _stream(stream)), "kvq_quantize_append")
+
+
+def decode_workspace_bytes(cache: KVCache, Hq: int, max_seqlen: int) -> int:
+    return int(load().kvq_decode_workspace_bytes(C.byref(cache.desc), int(Hq), int(max_seqlen)))
+
+
+def decode_attention(q, Tk_invT, cache: KVCache, seqlens, max_seqlen: int, out, workspace,
+                     dev_err=None, stream=None):
+    """kvq_decode_attention: q [B][Hq][d] float32/bfloat16; Tk_invT [Hkv][d][d] float32 or
+    None; seqlens int32 [B]; out [B][Hq][d] float32/bfloat16; workspace uint8 tensor."""
+    L = load()
+    _cuda("q", q)
+    _cuda("Tk_invT", Tk_invT, torch.float32)
+    _cuda("seqlens", seqlens, torch.int32)
+    _cuda("out", out)
+    _cuda("workspace", workspace, torch.uint8)
+    _cuda("dev_err", dev_err, torch.int32)
+    Hq = q.shape[1]
+    _check(L.kvq_decode_attention(_ptr(q), _dt(q), int(Hq), _ptr(Tk_invT), C.byref(cache.desc),
+                                  _ptr(seqlens), int(max_seqlen), _ptr(out), _dt(out),
+                                  _ptr(workspace), workspace.numel(), _ptr(dev_err),
+                                  _stream(stream)), "kvq_decode_attention")
+
+
+def bf16_decode_workspace_bytes(B, Hq, Hkv, d, max_seqlen) -> int:
+    return int(load().kvq_bf16_decode_workspace_bytes(int(B), int(Hq), int(Hkv), int(d),
+                                                      int(max_seqlen)))
+
+
+def bf16_decode(q, k, v, seqlens, max_seqlen: int, out, workspace, dev_err=None, stream=None):
+    """kvq_bf16_decode: q, out [B][Hq][d] bf16; k, v [B][Hkv][T_cap][d] bf16."""
+    L = load()
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _cuda(name, t, torch.bfloat16)
+    _cuda("seqlens", seqlens, torch.int32)
+    _cuda("workspace", workspace, torch.uint8)
+    _cuda("dev_err", dev_err, torch.int32)
+    B, Hq, d = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    _check(L.kvq_bf16_decode(_ptr(q), int(Hq), _ptr(k), _ptr(v), int(B), int(Hkv), int(T_cap),
+                             int(d), _ptr(seqlens), int(max_seqlen), _ptr(out), _ptr(workspace),
+                             workspace.numel(), _ptr(dev_err), _stream(stream)), "kvq_bf16_decode")

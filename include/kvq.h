@@ -40,6 +40,12 @@
 extern "C" {
 #endif
 
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
 struct CUstream_st;                        /* the CUDA runtime's cudaStream_t target */
 typedef struct CUstream_st *kvq_stream_t;  /* pass a cudaStream_t here */
 
@@ -108,7 +114,7 @@ typedef struct {
 } kvq_cache;
 
 /* Size in bytes of plane `which` (0 k_codes, 1 k_sz, 2 v_codes, 3 v_sz); 0 if invalid. */
-size_t kvq_cache_plane_bytes(const kvq_cache *cache, int which);
+KVQ_API size_t kvq_cache_plane_bytes(const kvq_cache *cache, int which);
 
 /*
  * Write path: transform, clip, quantize and append n new tokens per sequence.
@@ -123,14 +129,14 @@ size_t kvq_cache_plane_bytes(const kvq_cache *cache, int which);
  * transformed inputs the codes, scales and zero-points equal the float64 definition
  * above bit for bit.
  */
-kvq_status kvq_quantize_append(const void *k_post_rope, const void *v, kvq_dtype in_dtype,
+KVQ_API kvq_status kvq_quantize_append(const void *k_post_rope, const void *v, kvq_dtype in_dtype,
                                const float *T_k, const float *T_v, const kvq_qparams *qp,
                                kvq_cache *cache, const int32_t *pos, int n, int32_t *dev_err,
                                kvq_stream_t stream);
 
 /* Workspace bytes kvq_decode_attention needs for this cache shape, Hq query heads and
  * sequences of at most max_seqlen tokens (0 if the arguments are invalid). */
-size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int Hq, int max_seqlen);
+KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int Hq, int max_seqlen);
 
 /*
  * Read path: one decode step of grouped-query attention over the quantized cache.
@@ -146,29 +152,29 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int Hq, int max_seqlen
  * Computed as a split-K flash decode: scores and P.V on tensor cores with float32
  * accumulation, float32 online softmax, then a merge of the splits.
  */
-kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const float *Tk_invT,
+KVQ_API kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const float *Tk_invT,
                                 const kvq_cache *cache, const int32_t *seqlens, int max_seqlen,
                                 void *out, kvq_dtype out_dtype, void *workspace,
                                 size_t ws_bytes, int32_t *dev_err, kvq_stream_t stream);
 
 /* Workspace bytes kvq_bf16_decode needs (0 if the arguments are invalid). */
-size_t kvq_bf16_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seqlen);
+KVQ_API size_t kvq_bf16_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seqlen);
 
 /*
  * Uncompressed comparator: the same decode attention over bfloat16 keys and values
  * [B][Hkv][T_cap][d] (no transform, no quantization); q, out [B][Hq][d] bfloat16.
  * d in {64, 128}; T_cap a multiple of 64. Same workspace and error conventions.
  */
-kvq_status kvq_bf16_decode(const void *q, int Hq, const void *k, const void *v, int B, int Hkv,
+KVQ_API kvq_status kvq_bf16_decode(const void *q, int Hq, const void *k, const void *v, int B, int Hkv,
                            int T_cap, int d, const int32_t *seqlens, int max_seqlen, void *out,
                            void *workspace, size_t ws_bytes, int32_t *dev_err,
                            kvq_stream_t stream);
 
 /* Static description of a status code. */
-const char *kvq_status_string(kvq_status status);
+KVQ_API const char *kvq_status_string(kvq_status status);
 
 /* Detail of the last non-OK status returned on this host thread ("" if none). */
-const char *kvq_last_error(void);
+KVQ_API const char *kvq_last_error(void);
 
 #ifdef __cplusplus
 }

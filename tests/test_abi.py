@@ -1,0 +1,146 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every entry
+point include/kvq.h declares, sizes planes as the layout says, and rejects bad arguments
+before launching anything."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import decode_attention_post_b200 as kvq
+from decode_attention_post_b200 import kvq as K
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_function():
+    L = kvq.load()
+    names = _header_functions()
+    assert {"kvq_quantize_append", "kvq_decode_attention", "kvq_bf16_decode"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    L = kvq.load()
+    for s in range(6):
+        assert L.kvq_status_string(s)
+    assert L.kvq_status_string(99) == b"unknown status"
+
+
+def _desc(B=2, Hkv=2, T_cap=128, d=128, bits_k=2, bits_v=2, group=128, alpha=0.01,
+          ptr=0x1000):
+    qp = K._QParams(bits_k, bits_v, group, alpha)
+    return K._Cache(B, Hkv, T_cap, d, qp, ptr, ptr, ptr, ptr), qp
+
+
+def test_plane_bytes_follow_layout():
+    L = kvq.load()
+    desc, _ = _desc(B=3, Hkv=2, T_cap=192, d=128, bits_k=4, bits_v=2)
+    tok = 3 * 2 * 192
+    want = [tok * 64, tok * 4, tok * 32, tok * 4]
+    assert [L.kvq_cache_plane_bytes(C.byref(desc), w) for w in range(4)] == want
+    assert L.kvq_cache_plane_bytes(C.byref(desc), 7) == 0
+    # 2-bit, group 128: 2.25 bits per element including the float16 (s, z)
+    desc, _ = _desc(bits_k=2)
+    kb = L.kvq_cache_plane_bytes(C.byref(desc), 0) + L.kvq_cache_plane_bytes(C.byref(desc), 1)
+    assert kb * 8 / (2 * 2 * 128 * 128) == 2.25
+
+
+def _append(desc, qp, n=4, dtype=0, k=0x2000, pos=0x3000):
+    L = kvq.load()
+    return L.kvq_quantize_append(k, k, dtype, None, None, C.byref(qp), C.byref(desc), pos, n,
+                                 None, None)
+
+
+@pytest.mark.parametrize("mut,status", [
+    (dict(bits_k=3), 2), (dict(bits_v=8), 2), (dict(group=48), 1), (dict(group=256), 1),
+    (dict(d=96, group=32), 2), (dict(T_cap=100), 1), (dict(B=0), 1), (dict(alpha=0.6), 1),
+    (dict(alpha=0.2), 2),            # clip index 25 > 8
+    (dict(ptr=0x1004), 1),           # misaligned planes
+])
+def test_append_rejects_bad_cache(mut, status):
+    desc, qp = _desc(**mut)
+    assert _append(desc, qp) == status
+    assert kvq.load().kvq_last_error()
+
+
+def test_append_argument_errors():
+    L = kvq.load()
+    desc, qp = _desc()
+    other = K._QParams(2, 2, 128, 0.02)
+    assert L.kvq_quantize_append(0x2000, 0x2000, 0, None, None, C.byref(other), C.byref(desc),
+                                 0x3000, 4, None, None) == 1          # qp != cache qp
+    assert _append(desc, qp, n=-1) == 1
+    assert _append(desc, qp, n=129) == 3                              # > T_cap
+    assert _append(desc, qp, dtype=7) == 1
+    assert _append(desc, qp, k=0) == 1                                # NULL input
+    assert _append(desc, qp, n=0) == 0                                # no-op, nothing launched
+    assert L.kvq_quantize_append(0x2000, 0x2000, 0, None, None, C.byref(qp), None, 0x3000, 4,
+                                 None, None) == 1
+
+
+def _decode(desc, Hq=8, max_seqlen=64, ws=0x4000, ws_bytes=1 << 30, q=0x5000, out=0x6000,
+            qd=1, od=1):
+    L = kvq.load()
+    return L.kvq_decode_attention(q, qd, Hq, None, C.byref(desc), 0x7000, max_seqlen, out, od,
+                                  ws, ws_bytes, None, None)
+
+
+def test_decode_argument_errors():
+    desc, _ = _desc()
+    assert _decode(desc, Hq=7) == 1            # not a multiple of Hkv
+    assert _decode(desc, Hq=6) == 2            # G = 3 not implemented
+    assert _decode(desc, Hq=4) == 2            # G = 2 not implemented
+    assert _decode(desc, max_seqlen=129) == 3  # > T_cap
+    assert _decode(desc, max_seqlen=-1) == 1
+    assert _decode(desc, ws=0) == 4
+    assert _decode(desc, ws=0x4010) == 4       # not 256-byte aligned
+    assert _decode(desc, ws_bytes=16) == 4
+    assert _decode(desc, q=0) == 1
+    assert _decode(desc, qd=5) == 1
+    d2, _ = _desc(group=64)
+    assert _decode(d2) == 2                    # decode implements group == d
+
+
+def test_workspace_sizes_positive_and_monotone():
+    L = kvq.load()
+    desc, _ = _desc(B=4, Hkv=8, T_cap=16384)
+    a = L.kvq_decode_workspace_bytes(C.byref(desc), 32, 1024)
+    b = L.kvq_decode_workspace_bytes(C.byref(desc), 32, 16384)
+    assert 0 < a <= b
+    assert L.kvq_decode_workspace_bytes(C.byref(desc), 31, 1024) == 0
+    assert L.kvq_bf16_decode_workspace_bytes(4, 32, 8, 128, 16384) > 0
+    assert L.kvq_bf16_decode_workspace_bytes(4, 32, 8, 96, 16384) == 0
+
+
+def test_bf16_decode_argument_errors():
+    L = kvq.load()
+    args = dict(q=0x1000, Hq=32, k=0x2000, v=0x3000, B=2, Hkv=8, T_cap=128, d=128,
+                seqlens=0x4000, max_seqlen=64, out=0x5000, ws=0x6000, ws_bytes=1 << 30)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return L.kvq_bf16_decode(a["q"], a["Hq"], a["k"], a["v"], a["B"], a["Hkv"], a["T_cap"],
+                                 a["d"], a["seqlens"], a["max_seqlen"], a["out"], a["ws"],
+                                 a["ws_bytes"], None, None)
+    assert call(k=0) == 1
+    assert call(T_cap=100) == 1
+    assert call(d=80) == 2
+    assert call(Hq=16) == 2
+    assert call(max_seqlen=200) == 3
+    assert call(ws_bytes=8) == 4
+    assert call(k=0x2008) == 1
+
+
+def test_binding_requires_cuda_tensors():
+    import torch
+    qp = kvq.QParams()
+    with pytest.raises(TypeError):
+        kvq.KVCache(1, 1, 64, 128, qp, [torch.zeros(8, dtype=torch.uint8)] * 4)
