@@ -1,0 +1,513 @@
+#!/usr/bin/env python3
+"""Benchmark of the transformed-KV 2-bit decode hot path on B200.
+
+One step = one decode step of the serving loop on the Qwen3-8B-shaped high-concurrency
+workload (batch 64, 32 query / 8 KV heads, head_dim 128, ragged contexts uniform in
+[12288, 16384], 2-bit keys and values, group 128, bf16 queries and output):
+    kvq_quantize_append  the newest token of every sequence (transform, clip, quantize,
+                         pack) at position seqlen_b - 1
+    kvq_decode_attention over positions [0, seqlen_b) of every sequence
+All inputs are seeded synthetic stand-ins (tests/synth.py) for Qwen3-8B activations.
+The cache (~530 MB) is larger than the 126 MB L2, so no flush is needed between steps.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the
+data path); timing is the max over ranks. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tests import synth  # noqa: E402  (seeded input generators only)
+
+METRIC = "2-bit KV decode attention: achieved HBM GB/s and % of B200 peak; append tok/s"
+CONFIG_IDX = 2
+APPEND_CONFIG_IDX = 4
+
+
+def step_bytes(cfg, seqlens):
+    """Algorithmic bytes of one step.
+
+    decode: sum_b seqlen_b * Hkv * (d*bk/8 + 4*d/g + d*bv/8 + 4*d/g) + q + out
+    append: new k, v (bf16) + their codes and (s, z) + T_k, T_v once
+    """
+    ng = cfg.d // cfg.group
+    per_tok = cfg.Hkv * (cfg.d * cfg.bits_k // 8 + 4 * ng + cfg.d * cfg.bits_v // 8 + 4 * ng)
+    qo = 2 * cfg.B * cfg.Hq * cfg.d * 2
+    decode = int(np.sum(seqlens)) * per_tok + qo
+    append = cfg.B * cfg.Hkv * (2 * cfg.d * 2) + cfg.B * per_tok + 2 * cfg.Hkv * cfg.d * cfg.d * 4
+    return decode, append
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows
+                                    if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ----------------------------------------------------------------------------- GPU workload
+
+class Workload:
+    """Config-2 cache built by the library's own quantize-append, plus step inputs."""
+
+    def __init__(self, cfg, rank, device, with_bf16=True):
+        import torch
+        import decode_attention_post_b200 as kvq
+        self.cfg, self.dev = cfg, device
+        self.qp = kvq.QParams(cfg.bits_k, cfg.bits_v, cfg.group, cfg.clip_alpha)
+        self.cache = kvq.KVCache.allocate(cfg.B, cfg.Hkv, cfg.T_cap, cfg.d, self.qp, device=device)
+        self.seqlens = synth.seqlens(cfg)
+        Tk, Tv, Tit = synth.transforms(cfg)
+        g = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.Tk, self.Tv, self.Tit = g(Tk), g(Tv), g(Tit)
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device).to(torch.bfloat16)
+        self.kb = self.vb = None
+        if with_bf16:
+            self.kb = torch.zeros((cfg.B, cfg.Hkv, cfg.T_cap, cfg.d), dtype=torch.bfloat16,
+                                  device=device)
+            self.vb = torch.zeros_like(self.kb)
+        knew = np.empty((cfg.B, 1, cfg.Hkv, cfg.d), np.float32)
+        vnew = np.empty_like(knew)
+        zero = torch.zeros(1, dtype=torch.int32, device=device)
+        for b in range(cfg.B):
+            n = int(self.seqlens[b])
+            src = b + rank * cfg.B                       # each rank its own sequences
+            k = synth.keys(cfg, src, 0, n)
+            v = synth.values(cfg, src, 0, n)
+            kd, vd = bf(k), bf(v)                        # [n][Hkv][d] bf16
+            view = self.cache.view_sequence(b)
+            kvq.quantize_append(kd[None], vd[None], self.Tk, self.Tv, self.qp, view, zero)
+            if with_bf16:
+                self.kb[b, :, :n] = kd.transpose(0, 1)
+                self.vb[b, :, :n] = vd.transpose(0, 1)
+            knew[b, 0] = k[n - 1]
+            vnew[b, 0] = v[n - 1]
+        self.knew, self.vnew = bf(knew), bf(vnew)
+        self.q = bf(synth.queries(cfg))
+        self.pos = g(self.seqlens - 1)
+        self.seq_d = g(self.seqlens)
+        self.max_seqlen = cfg.T_cap
+        self.out = torch.empty((cfg.B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=device)
+        self.ws = torch.empty(kvq.decode_workspace_bytes(self.cache, cfg.Hq, self.max_seqlen),
+                              dtype=torch.uint8, device=device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        torch.cuda.synchronize()
+
+    def append(self):
+        import decode_attention_post_b200 as kvq
+        kvq.quantize_append(self.knew, self.vnew, self.Tk, self.Tv, self.qp, self.cache, self.pos,
+                            n=1, dev_err=self.err)
+
+    def decode(self):
+        import decode_attention_post_b200 as kvq
+        kvq.decode_attention(self.q, self.Tit, self.cache, self.seq_d, self.max_seqlen, self.out,
+                             self.ws, dev_err=self.err)
+
+    def step(self):
+        self.append()
+        self.decode()
+
+
+def time_events(fn, iters, stream, per_graph=1):
+    """Mean device time of one fn() call: fn is captured `per_graph` times into a CUDA
+    graph, each replay is bracketed by CUDA events on the launching stream, so host
+    launch overhead does not leak into the measurement."""
+    import torch
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(per_graph):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for a, b in evs:
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) / per_graph for a, b in evs]
+    del g
+    return times
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import decode_attention_post_b200 as kvq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device(device))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    cfg = synth.CONFIGS[CONFIG_IDX]
+    w = Workload(cfg, rank, device, with_bf16=not args.no_extras)
+    stream = torch.cuda.current_stream()
+    dec_bytes, app_bytes = step_bytes(cfg, w.seqlens)
+
+    # ---- warm-up, then capture one step in a CUDA graph (3 kernels per replay)
+    for _ in range(max(args.warmup, 3)):
+        w.step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        w.step()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps, barrier + synchronize on both sides
+    K = args.steps
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(K):
+            graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    clocks = sampler.summary()
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    ms_step = ms_total / K
+    value = world * (dec_bytes + app_bytes) / (ms_step * 1e-3) / 1e9
+
+    # ---- the dominant kernel (the decode call: q prologue + split-K decode) timed alone
+    dec_ms = statistics.mean(time_events(w.decode, min(K, 500), stream))
+    app_ms = statistics.mean(time_events(w.append, min(K, 200), stream, per_graph=20))
+    dec_ms = max_over_ranks(dec_ms)
+    peak, peak_kind = peaks()
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    dev_err = int(w.err.item())
+
+    # ---- end to end through the public API with pinned host buffers
+    q_h = w.q.cpu().pin_memory()
+    k_h, v_h = w.knew.cpu().pin_memory(), w.vnew.cpu().pin_memory()
+    s_h, p_h = w.seq_d.cpu().pin_memory(), w.pos.cpu().pin_memory()
+    out_h = torch.empty_like(w.out, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, s_h, p_h))
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        w.q.copy_(q_h, non_blocking=True)
+        w.knew.copy_(k_h, non_blocking=True)
+        w.vnew.copy_(v_h, non_blocking=True)
+        w.seq_d.copy_(s_h, non_blocking=True)
+        w.pos.copy_(p_h, non_blocking=True)
+        w.step()
+        out_h.copy_(w.out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    Ke = min(K, 500)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / Ke
+    e2e_value = world * (dec_bytes + app_bytes) / (e2e_ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "2-bit codes -> f16 mma, f32 accumulate/softmax", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
+                   "T_cap": cfg.T_cap, "seqlens": f"U[{cfg.seq_lo},{cfg.seq_hi}]",
+                   "sum_seqlens": int(np.sum(w.seqlens)), "bits_k": cfg.bits_k,
+                   "bits_v": cfg.bits_v, "group": cfg.group, "clip_alpha": cfg.clip_alpha,
+                   "q_out_dtype": "bf16", "step": "append 1 token/seq + decode",
+                   "l2": "inputs larger than L2 (decode reads ~%.0f MB per step)" % (dec_bytes / 1e6),
+                   "parallelism": f"dp{world} (independent batches)", "cuda_graph": True},
+        "roofline": {"bound": "hbm", "kernel": "kvq_decode_attention (qprep + decode_kernel)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "frac_of_nominal_8000": round(achieved / 8000.0, 4),
+                     "bytes_per_launch": dec_bytes, "ms_per_launch": round(dec_ms, 5),
+                     "traffic": None},
+        "append_decode_time": {"append_ms": round(app_ms, 5), "decode_ms": round(dec_ms, 5),
+                               "append_tok_per_s": round(cfg.B / (app_ms * 1e-3), 1)},
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * K,
+        "dev_err": dev_err,
+        "clocks": clocks,
+    }
+
+    if not args.no_extras:
+        line["bf16_comparator"] = bf16_comparator(w, cfg, K, stream, dec_ms)
+        del w
+        torch.cuda.empty_cache()
+        line["chunk_append"] = chunk_append(device, stream)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bf16_comparator(w, cfg, K, stream, dec_ms):
+    import torch
+    import decode_attention_post_b200 as kvq
+    out = torch.empty_like(w.out)
+    ws = torch.empty(kvq.bf16_decode_workspace_bytes(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.T_cap),
+                     dtype=torch.uint8, device=w.dev)
+    fn = lambda: kvq.bf16_decode(w.q, w.kb, w.vb, w.seq_d, cfg.T_cap, out, ws, dev_err=w.err)
+    ms = statistics.mean(time_events(fn, min(K, 200), stream))
+    nbytes = int(np.sum(w.seqlens)) * cfg.Hkv * cfg.d * 2 * 2 + 2 * cfg.B * cfg.Hq * cfg.d * 2
+    return {"ms_per_launch": round(ms, 5), "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "bytes_per_launch": nbytes, "speedup_of_2bit_decode": round(ms / dec_ms, 2)}
+
+
+def chunk_append(device, stream):
+    """32768-token chunk append of the GPT-OSS-20B-like shape (batch 8, 8 KV heads, d 64)."""
+    import torch
+    import decode_attention_post_b200 as kvq
+    cfg = synth.CONFIGS[APPEND_CONFIG_IDX]
+    n = cfg.append_n
+    qp = kvq.QParams(cfg.bits_k, cfg.bits_v, cfg.group, cfg.clip_alpha)
+    cache = kvq.KVCache.allocate(cfg.B, cfg.Hkv, cfg.T_cap, cfg.d, qp, device=device)
+    Tk, Tv, _ = synth.transforms(cfg)
+    k, v = synth.kv_batch(cfg, 0, n)
+    bf = lambda a: torch.from_numpy(a).to(device).to(torch.bfloat16)
+    kd, vd = bf(k), bf(v)
+    del k, v
+    Tk, Tv = torch.from_numpy(Tk).to(device), torch.from_numpy(Tv).to(device)
+    pos = torch.zeros(cfg.B, dtype=torch.int32, device=device)
+    fn = lambda: kvq.quantize_append(kd, vd, Tk, Tv, qp, cache, pos)
+    ms = statistics.mean(time_events(fn, 10, stream))
+    ng = cfg.d // cfg.group
+    tokheads = cfg.B * n * cfg.Hkv
+    nbytes = tokheads * (2 * cfg.d * 2 + cfg.d * (cfg.bits_k + cfg.bits_v) // 8 + 8 * ng) + \
+        2 * cfg.Hkv * cfg.d * cfg.d * 4
+    flops = tokheads * 4 * cfg.d * cfg.d
+    return {"workload": cfg.name, "ms": round(ms, 4),
+            "tok_per_s": round(cfg.B * n / (ms * 1e-3), 1),
+            "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "TFLOP_s": round(flops / (ms * 1e-3) / 1e12, 2), "bytes": nbytes}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+
+class OracleSample:
+    """A bounded sample of the config-2 step for the float64 CPU oracle: the first
+    `nseq` sequences, all heads, the cache built by the oracle itself."""
+
+    def __init__(self, cfg, nseq):
+        import oracle
+        self.oracle = oracle
+        self.cfg = cfg.with_(B=nseq)
+        self.seqlens = synth.seqlens(cfg)[:nseq]
+        Tk, Tv, self.Tit = synth.transforms(cfg)
+        self.Tk, self.Tv = Tk, Tv
+        self.cache = oracle.Cache.for_config(self.cfg)
+        knew = np.empty((nseq, 1, cfg.Hkv, cfg.d), np.uint16)
+        vnew = np.empty_like(knew)
+        for b in range(nseq):
+            n = int(self.seqlens[b])
+            k = synth.as_dtype(synth.keys(cfg, b, 0, n), "bf16")
+            v = synth.as_dtype(synth.values(cfg, b, 0, n), "bf16")
+            one = oracle.Cache(1, cfg.Hkv, cfg.T_cap, cfg.d, cfg.bits_k, cfg.bits_v, cfg.group)
+            oracle.quantize_append(k[None], v[None], Tk, Tv, cfg.bits_k, cfg.bits_v, cfg.group,
+                                   cfg.clip_alpha, one, [0])
+            for dst, src in zip(self.cache.planes(), one.planes()):
+                m = src.size
+                dst[b * m:(b + 1) * m] = src
+            knew[b, 0], vnew[b, 0] = k[n - 1], v[n - 1]
+        self.knew, self.vnew = knew, vnew
+        self.q = synth.as_dtype(synth.queries(cfg), "bf16")[:nseq].copy()
+
+    def step(self, sel=None):
+        c = self.cfg
+        self.oracle.quantize_append(self.knew, self.vnew, self.Tk, self.Tv, c.bits_k, c.bits_v,
+                                    c.group, c.clip_alpha, self.cache, self.seqlens - 1)
+        return self.oracle.decode(self.q, self.Tit, self.cache, self.seqlens, sel=sel)
+
+    def bytes(self, heads=None):
+        """Algorithmic bytes of the sample; decode bytes scale with the query heads run."""
+        d, a = step_bytes(self.cfg, self.seqlens)
+        frac = 1.0 if heads is None else heads / self.cfg.Hq
+        return d * frac + a
+
+
+def cpu_baseline(cfg, budget_s=12.0):
+    import oracle
+    s = OracleSample(cfg, 1)
+    t = time.perf_counter()
+    s.step()
+    one = time.perf_counter() - t
+    reps = max(1, int(budget_s / max(one, 1e-3)))
+    t = time.perf_counter()
+    for _ in range(reps):
+        s.step()
+    el = (time.perf_counter() - t) / reps
+    return {"value": round(s.bytes() / el / 1e9, 4), "unit": "GB/s",
+            "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"1 of {cfg.B} sequences (seqlen {int(s.seqlens[0])}), all {cfg.Hq} "
+                      f"query heads: append 1 token + decode, {reps} reps, "
+                      f"{el:.3f} s per step"}
+
+
+def run_reference(args):
+    """The float64 oracle as the reference arm, timed on the host cores. Each step is a
+    bounded sample of the config-2 step (the newest token of one sequence appended, then
+    the decode of that sequence for as many query heads as keep K steps within ~2 minutes)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    cfg = synth.CONFIGS[CONFIG_IDX]
+    s = OracleSample(cfg, 1)
+    t = time.perf_counter()
+    s.step()
+    full = time.perf_counter() - t
+    K = args.steps
+    heads = int(min(cfg.Hq, max(1, round(cfg.Hq * 120.0 / (max(K, 1) * full)))))
+    sel = np.array([[0, h] for h in range(heads)], np.int32)
+    for _ in range(max(args.warmup, 3)):
+        s.step(sel)
+    t = time.perf_counter()
+    for _ in range(K):
+        s.step(sel)
+    el = (time.perf_counter() - t) / K
+    value = s.bytes(heads) / el / 1e9
+    cores = oracle.get_threads()
+    sample = (f"sequence 0 of {cfg.B} (seqlen {int(s.seqlens[0])}): append 1 token (all KV "
+              f"heads) + decode of {heads} of {cfg.Hq} query heads per step")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(el * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv,
+                       "d": cfg.d, "T_cap": cfg.T_cap, "bits_k": cfg.bits_k,
+                       "bits_v": cfg.bits_v, "sample": sample},
+            "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("kvq", "reference"), default="kvq")
+    ap.add_argument("--no-extras", action="store_true", help="skip bf16 comparator and chunk append")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()
