@@ -18,6 +18,7 @@ from .kvq import (  # noqa: F401
     bf16_decode_workspace_bytes,
     cache_plane_bytes,
     decode_attention,
+    decode_attention_noalloc,
     decode_workspace_bytes,
     library_path,
     load,

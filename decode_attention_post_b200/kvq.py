@@ -68,6 +68,9 @@ def load():
     L.kvq_decode_attention.restype = _I
     L.kvq_decode_attention.argtypes = [_P, _I, _I, _P, C.POINTER(_Cache), _P, _I, _P, _I, _P, _S,
                                        _P, _P]
+    L.kvq_decode_attention_noalloc.restype = _I
+    L.kvq_decode_attention_noalloc.argtypes = [_P, _I, _I, _P, C.POINTER(_Cache), _P, _I, _P,
+                                               _I, _P, _P]
     L.kvq_bf16_decode_workspace_bytes.restype = _S
     L.kvq_bf16_decode_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
     L.kvq_bf16_decode.restype = _I
@@ -210,6 +213,26 @@ def decode_attention(q, Tk_invT, cache: KVCache, seqlens, max_seqlen: int, out, 
                                   _ptr(seqlens), int(max_seqlen), _ptr(out), _dt(out),
                                   _ptr(workspace), workspace.numel(), _ptr(dev_err),
                                   _stream(stream)), "kvq_decode_attention")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def decode_attention_noalloc(q, Tk_invT, cache: KVCache, seqlens, max_seqlen: int, out,
+                             dev_err=None, stream=None):
+    """kvq_decode_attention_noalloc: as decode_attention, with the library's fixed
+    device scratch array instead of a caller workspace (for callers that cannot
+    allocate device memory; calls must not overlap on the GPU)."""
+    L = load()
+    _cuda("q", q)
+    _cuda("Tk_invT", Tk_invT, torch.float32)
+    _cuda("seqlens", seqlens, torch.int32)
+    _cuda("out", out)
+    _cuda("dev_err", dev_err, torch.int32)
+    _check(L.kvq_decode_attention_noalloc(_ptr(q), _dt(q), int(q.shape[1]), _ptr(Tk_invT),
+                                          C.byref(cache.desc), _ptr(seqlens), int(max_seqlen),
+                                          _ptr(out), _dt(out), _ptr(dev_err), _stream(stream)),
+           "kvq_decode_attention_noalloc")
 
 
 def bf16_decode_workspace_bytes(B, Hq, Hkv, d, max_seqlen) -> int:

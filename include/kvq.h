@@ -170,6 +170,30 @@ KVQ_API kvq_status kvq_bf16_decode(const void *q, int Hq, const void *k, const v
                            void *workspace, size_t ws_bytes, int32_t *dev_err,
                            kvq_stream_t stream);
 
+/*
+ * Allocation-free decode (no counterpart in the paper; an addition for callers that
+ * cannot allocate device memory). Same arguments and result as kvq_decode_attention
+ * minus the workspace: an inference engine that has reserved nearly all device memory
+ * for its own KV pool, or a latency-critical serving loop that forbids cudaMalloc
+ * (it synchronises the device), can call this instead. The scratch lives in a fixed
+ * array that the library declares in device memory:
+ *  - every GPU that loads the library holds KVQ_NOALLOC_SCRATCH_BYTES for it until exit;
+ *  - if kvq_decode_workspace_bytes(cache, Hq, max_seqlen) exceeds that size the call
+ *    returns KVQ_ERR_WORKSPACE without launching;
+ *  - all calls on a device share the array and it keeps the last call's contents (each
+ *    call re-initialises what must start at zero); calls whose kernels overlap on the
+ *    GPU (e.g. on unordered streams) race on it and must be avoided;
+ *  - the first call on each device looks up the array's address (once per device, that
+ *    device current); make that first call before any stream capture.
+ * No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define KVQ_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+KVQ_API kvq_status kvq_decode_attention_noalloc(const void *q, kvq_dtype q_dtype, int Hq,
+                                                const float *Tk_invT, const kvq_cache *cache,
+                                                const int32_t *seqlens, int max_seqlen,
+                                                void *out, kvq_dtype out_dtype,
+                                                int32_t *dev_err, kvq_stream_t stream);
+
 /* Static description of a status code. */
 KVQ_API const char *kvq_status_string(kvq_status status);
 
