@@ -24,11 +24,12 @@ namespace {
 
 constexpr int kAppendThreads = 256;
 constexpr int kAppendWarps = kAppendThreads / 32;
-constexpr int kTokPerWarp = 4;
-constexpr int kTokPerTile = kAppendWarps * kTokPerWarp;   // 32
 
-template <int D>
+// TPW tokens per warp: 4 for bulk appends (register tiling amortises the T reads),
+// 1 for small ones (decode-time appends), so that more warps share the work.
+template <int D, int TPW>
 struct AppendSmem {
+    static constexpr int kTokPerTile = kAppendWarps * TPW;
     float Tt[D * (D + 1)];          // Tt[j*(D+1) + i] = T[i][j]
     float X[kTokPerTile][D];
     uint8_t codes[kAppendWarps][D];
@@ -71,7 +72,7 @@ __device__ __forceinline__ float order_stat(const float (&vals)[NV], int kappa, 
     return m;
 }
 
-template <int D>
+template <int D, int TPW>
 __global__ void __launch_bounds__(kAppendThreads)
 append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in, int in_bf16,
                    const float *__restrict__ Tk, const float *__restrict__ Tv, int B, int n,
@@ -81,7 +82,10 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
                    const int32_t *__restrict__ pos, int32_t *dev_err)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    AppendSmem<D> &sm = *reinterpret_cast<AppendSmem<D> *>(smem_raw);
+    using Smem = AppendSmem<D, TPW>;
+    constexpr int kTokPerWarp = TPW;
+    constexpr int kTokPerTile = Smem::kTokPerTile;
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
 
     const int h = blockIdx.y;
     const int which = blockIdx.z;               // 0 = keys, 1 = values
@@ -96,22 +100,34 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
     const int qmax = (1 << bits) - 1;
 
     if (T) {
-        const float *Th = T + (size_t)h * D * D;
-        for (int idx = threadIdx.x; idx < D * D; idx += kAppendThreads) {
-            int i = idx / D, j = idx % D;
-            sm.Tt[j * (D + 1) + i] = Th[idx];
+        // 16 independent float4 loads in flight per thread, then transposed stores
+        const float4 *Th4 = reinterpret_cast<const float4 *>(T + (size_t)h * D * D);
+        constexpr int N4 = D * D / 4 / kAppendThreads;
+#pragma unroll 16
+        for (int it = 0; it < N4; ++it) {
+            const int idx4 = threadIdx.x + kAppendThreads * it;
+            const float4 v4 = Th4[idx4];
+            const int i = (4 * idx4) / D, j = (4 * idx4) % D;
+            sm.Tt[(j + 0) * (D + 1) + i] = v4.x;
+            sm.Tt[(j + 1) * (D + 1) + i] = v4.y;
+            sm.Tt[(j + 2) * (D + 1) + i] = v4.z;
+            sm.Tt[(j + 3) * (D + 1) + i] = v4.w;
         }
     }
 
     for (long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         const long u0 = tile * kTokPerTile;
         __syncthreads();                        // previous tile's readers are done
-        for (int idx = threadIdx.x; idx < kTokPerTile * D; idx += kAppendThreads) {
-            int tk = idx / D, j = idx % D;
-            long u = u0 + tk;
+#pragma unroll
+        for (int it = 0; it < (kTokPerTile * D + kAppendThreads - 1) / kAppendThreads; ++it) {
+            const int idx = threadIdx.x + kAppendThreads * it;
+            if (idx >= kTokPerTile * D)
+                break;
+            const int tk = idx / D, j = idx % D;
+            const long u = u0 + tk;
             float x = 0.f;
             if (u < total) {
-                long b = u / n, i = u % n;
+                const long b = u / n, i = u % n;
                 x = load_in(in, in_bf16, (((size_t)b * n + i) * Hkv + h) * D + j);
             }
             sm.X[tk][j] = x;
@@ -232,21 +248,26 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
     }
 }
 
-template <int D>
+template <int D, int TPW>
 cudaError_t launch_append_fp32(const void *k, const void *v, int in_bf16, const float *Tk,
                                const float *Tv, int B, int n, const kvq_cache *c, int kappa,
                                const int32_t *pos, int32_t *dev_err, cudaStream_t st)
 {
-    const size_t smem = sizeof(AppendSmem<D>);
-    cudaError_t e = cudaFuncSetAttribute(append_fp32_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess)
-        return e;
+    using Smem = AppendSmem<D, TPW>;
+    const size_t smem = sizeof(Smem);
+    static int attr_set = 0;                // once per process (before any graph capture)
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(append_fp32_kernel<D, TPW>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        attr_set = 1;
+    }
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long total = (long)B * n;
-    const long tiles = (total + kTokPerTile - 1) / kTokPerTile;
+    const long tiles = (total + Smem::kTokPerTile - 1) / Smem::kTokPerTile;
     long want = (2L * sms + 2L * c->Hkv - 1) / (2L * c->Hkv);   // ~2 CTAs per SM overall
     if (want < 1)
         want = 1;
@@ -255,7 +276,7 @@ cudaError_t launch_append_fp32(const void *k, const void *v, int in_bf16, const 
     if (tiles > want * 8)
         gx = (tiles + 7) / 8 < 65535 ? (tiles + 7) / 8 : 65535;
     dim3 grid((unsigned)gx, (unsigned)c->Hkv, 2);
-    append_fp32_kernel<D><<<grid, kAppendThreads, smem, st>>>(
+    append_fp32_kernel<D, TPW><<<grid, kAppendThreads, smem, st>>>(
         k, v, in_bf16, Tk, Tv, B, n, c->Hkv, c->T_cap, c->qp.bits_k, c->qp.bits_v, c->qp.group,
         kappa, (uint8_t *)c->k_codes, (uint32_t *)c->k_sz, (uint8_t *)c->v_codes,
         (uint32_t *)c->v_sz, pos, dev_err);
@@ -268,9 +289,12 @@ cudaError_t append_fp32(const void *k, const void *v, int in_bf16, const float *
                         const float *Tv, int B, int n, const kvq_cache *c, int kappa,
                         const int32_t *pos, int32_t *dev_err, cudaStream_t st)
 {
+    const bool small = (long)B * n <= 2048;
     if (c->d == 64)
-        return launch_append_fp32<64>(k, v, in_bf16, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
-    return launch_append_fp32<128>(k, v, in_bf16, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
+        return small ? launch_append_fp32<64, 1>(k, v, in_bf16, Tk, Tv, B, n, c, kappa, pos, dev_err, st)
+                     : launch_append_fp32<64, 4>(k, v, in_bf16, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
+    return small ? launch_append_fp32<128, 1>(k, v, in_bf16, Tk, Tv, B, n, c, kappa, pos, dev_err, st)
+                 : launch_append_fp32<128, 4>(k, v, in_bf16, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
 }
 
 }  // namespace kvq

@@ -347,10 +347,14 @@ cudaError_t launch_t(const void *q, int Hq, const void *k, const void *v, int B,
     cudaError_t e = cudaMemsetAsync(ticket, 0, (size_t)B * Hkv * 4, st);
     if (e != cudaSuccess)
         return e;
-    e = cudaFuncSetAttribute(bf16_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM);
-    if (e != cudaSuccess)
-        return e;
+    static int attr_set = 0;
+    if (!attr_set) {
+        e = cudaFuncSetAttribute(bf16_decode_kernel<D, G>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess)
+            return e;
+        attr_set = 1;
+    }
     dim3 grid(nsplit, Hkv, B);
     bf16_decode_kernel<D, G><<<grid, kBWarps * 32, C::SMEM, st>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, B, Hq, Hkv,

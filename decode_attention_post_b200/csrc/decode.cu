@@ -30,6 +30,7 @@
 #include "decode_shapes.h"
 
 #include <math.h>
+#include <type_traits>
 
 namespace kvq {
 
@@ -124,7 +125,8 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u)
 // One CTA per (KV head, chunk of `bb` sequences). Computes q~ = M q in float32, then
 //   eq  = power-of-two exponent bringing max|q~| * 2^(BK*(CPB-1)) to about 2^14,
 //   frag[nt][ks][lane][2] = float16 hi/lo pieces of q~ * 2^eq * 2^(BK*(CPB-1-k)) laid
-//                           out as the B operand of the Q.K product,
+//                           out as the B operand of the Q.K product; n-tile nt holds
+//                           heads 4nt..4nt+3, column 2h' = hi and 2h'+1 = lo of head 4nt+h',
 //   cs  = log2(e) / sqrt(d) / F with F = 2^(eq + BK*(CPB-1) - 24) the product scale,
 //   w_h = log2(e) / sqrt(d) * sum_j q~_hj,
 // and zeroes the split-merge ticket of the (sequence, KV head).
@@ -149,31 +151,58 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
         red[tid] = 0.f;
 
     if (M) {
-        const float *Mh = M + (size_t)h * D * D;
-        for (int idx = tid; idx < D * D; idx += 256) {
-            int i = idx / D, j = idx % D;
-            Mt[j * (D + 1) + i] = Mh[idx];
+        const float4 *Mh4 = reinterpret_cast<const float4 *>(M + (size_t)h * D * D);
+        constexpr int N4 = D * D / 4 / 256;
+#pragma unroll 16
+        for (int it = 0; it < N4; ++it) {
+            const int idx4 = tid + 256 * it;
+            const float4 v4 = Mh4[idx4];
+            const int i = (4 * idx4) / D, j = (4 * idx4) % D;
+            Mt[(j + 0) * (D + 1) + i] = v4.x;
+            Mt[(j + 1) * (D + 1) + i] = v4.y;
+            Mt[(j + 2) * (D + 1) + i] = v4.z;
+            Mt[(j + 3) * (D + 1) + i] = v4.w;
         }
     }
-    for (int idx = tid; idx < nb * G * D; idx += 256) {
-        int v = idx / D, j = idx % D;
-        int bi = v / G, gg = v % G;
-        qs[idx] = load_in(q, q_bf16, ((size_t)(b0 + bi) * Hq + h * G + gg) * D + j);
+    // queries stored transposed, qs[j][v] (v = sequence-in-chunk * G + head), so that one
+    // 16-byte load feeds four vectors
+    const int NV = nb * G;
+    for (int idx = tid; idx < NV * D; idx += 256) {
+        const int v = idx / D, j = idx % D;
+        const int bi = v / G, gg = v % G;
+        qs[j * (bb * G) + v] = load_in(q, q_bf16, ((size_t)(b0 + bi) * Hq + h * G + gg) * D + j);
     }
     __syncthreads();
-    for (int idx = tid; idx < nb * G * D; idx += 256) {
-        int v = idx / D, i = idx % D;
-        float acc;
-        if (M) {
-            acc = 0.f;
-            const float *qv = qs + v * D;
+    // thread -> (output dim i, group of 4 vectors); register-tiled over the 4 vectors
+    {
+        const int VG = bb * G / 4;                          // vector groups of 4
+        for (int task = tid; task < D * VG; task += 256) {
+            const int i = task % D, vg = task / D;
+            if (4 * vg >= NV)
+                continue;
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            if (M) {
 #pragma unroll 8
-            for (int j = 0; j < D; ++j)
-                acc = fmaf(Mt[j * (D + 1) + i], qv[j], acc);
-        } else {
-            acc = qs[idx];
+                for (int j = 0; j < D; ++j) {
+                    const float m = Mt[j * (D + 1) + i];
+                    const float4 x = *reinterpret_cast<const float4 *>(qs + j * (bb * G) + 4 * vg);
+                    a0 = fmaf(m, x.x, a0);
+                    a1 = fmaf(m, x.y, a1);
+                    a2 = fmaf(m, x.z, a2);
+                    a3 = fmaf(m, x.w, a3);
+                }
+            } else {
+                const float4 x = *reinterpret_cast<const float4 *>(qs + i * (bb * G) + 4 * vg);
+                a0 = x.x;
+                a1 = x.y;
+                a2 = x.z;
+                a3 = x.w;
+            }
+            qt[(4 * vg + 0) * D + i] = a0;
+            qt[(4 * vg + 1) * D + i] = a1;
+            qt[(4 * vg + 2) * D + i] = a2;
+            qt[(4 * vg + 3) * D + i] = a3;
         }
-        qt[idx] = acc;
     }
     __syncthreads();
     // per sequence: max |q~| over its G heads; per head: sum of q~
@@ -215,7 +244,7 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
             const int rho = idx & 1, ln = (idx >> 1) & 31, ks = (idx >> 6) % KSTEPS;
             const int nt = (idx >> 6) / KSTEPS;
             const int g = ln >> 2, t = ln & 3;
-            const int col = 8 * nt + g, head = col % G, piece = col / G;
+            const int head = 4 * nt + g / 2, piece = g & 1;     // columns (hi, lo) per head
             const int e = 2 * ks + rho;
             const int w = WPT * t + e / (2 * CPB), beta = (e / CPB) & 1, k = e % CPB;
             const int dlo = (4 * w + beta) * CPB + k, dhi = (4 * w + 2 + beta) * CPB + k;
@@ -237,7 +266,7 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
 // ---------------------------------------------------------------- main decode
 
 template <int D, int G, int BK, int BV>
-__global__ void __launch_bounds__(kDecodeWarps * 32, 3) decode_kernel(DecodeParams P)
+__global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_kernel(DecodeParams P)
 {
     using C = Cfg<D, G, BK, BV>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -320,165 +349,137 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3) decode_kernel(DecodePara
                 qB[nt][ks][1] = v.y;
             }
     }
-    const int hp = (2 * t) % G;                 // this thread's head pair (hp, hp+1)
+    // Thread (g, t) owns head 4nt + t of every n-tile nt (columns 2t = hi, 2t+1 = lo) and
+    // tokens g, g+8 of every 16-token sub-tile.
     const float cs = P.qscale[pair];
-    const float wq0 = P.qw[(size_t)b * P.Hq + h * G + hp];
-    const float wq1 = P.qw[(size_t)b * P.Hq + h * G + hp + 1];
+    float wq[C::NT];
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt)
+        wq[nt] = P.qw[(size_t)b * P.Hq + h * G + 4 * nt + t];
 
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f}, lz_run[2] = {0.f, 0.f};
+    float m_run[C::NT], l_run[C::NT], lz_run[C::NT];
     float O[C::MT][C::NT][4];
 #pragma unroll
-    for (int m = 0; m < C::MT; ++m)
+    for (int nt = 0; nt < C::NT; ++nt) {
+        m_run[nt] = -INFINITY;
+        l_run[nt] = 0.f;
+        lz_run[nt] = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < C::NT; ++nt)
+        for (int m = 0; m < C::MT; ++m)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 O[m][nt][i] = 0.f;
-
-    constexpr int TPT = (G == 4) ? 1 : 2;       // tokens per thread per 16-token sub-tile
+    }
     bool timed_out = false;
 
-    for (int jj = 0; jj < my_nblk; ++jj) {
-        const int s = jj % kDecodeStages;
-        if (!mbar_wait_bounded(&bars[s], (jj / kDecodeStages) & 1)) {
-            timed_out = true;
-            // wait (bounded) for this warp's copies still in flight, then stop
-            for (int k2 = jj + 1; k2 < jj + kDecodeStages && k2 < my_nblk; ++k2)
-                mbar_wait_bounded(&bars[k2 % kDecodeStages], (k2 / kDecodeStages) & 1);
-            break;
-        }
-        const unsigned char *st = wring + s * C::STAGE;
+    // One 64-token block. FULL: every token is below t_end (no per-token masking).
+    auto block = [&](const unsigned char *st, int tok0, auto full_tag) {
+        constexpr bool FULL = decltype(full_tag)::value;
         const uint32_t *kszw = reinterpret_cast<const uint32_t *>(st + C::KC_BYTES);
         const uint32_t *vszw =
             reinterpret_cast<const uint32_t *>(st + C::KC_BYTES + C::SZ_BYTES + C::VC_BYTES);
-        const int tok0 = t_begin + (warp + jj * kDecodeWarps) * kDecodeBlock;
 
-        // ---- scores S^T for 4 sub-tiles of 16 tokens
+        // ---- scores S^T for 4 sub-tiles: independent chains interleaved per k-step
         float S[4][C::NT][4];
+        uint32_t kw[4][2][C::WPT];
 #pragma unroll
         for (int stt = 0; stt < 4; ++stt) {
             const unsigned char *kt = st + stt * 16 * C::ROWK + t * 4 * C::WPT;
-            uint32_t kw0[C::WPT], kw1[C::WPT];
-            lds_words<C::WPT>(kw0, kt + g * C::ROWK);
-            lds_words<C::WPT>(kw1, kt + (g + 8) * C::ROWK);
+            lds_words<C::WPT>(kw[stt][0], kt + g * C::ROWK);
+            lds_words<C::WPT>(kw[stt][1], kt + (g + 8) * C::ROWK);
 #pragma unroll
             for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     S[stt][nt][i] = 0.f;
+        }
 #pragma unroll
-            for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                const uint32_t a0 = ext_k<BK, C::CPBK>(kw0, 2 * ks);
-                const uint32_t a1 = ext_k<BK, C::CPBK>(kw1, 2 * ks);
-                const uint32_t a2 = ext_k<BK, C::CPBK>(kw0, 2 * ks + 1);
-                const uint32_t a3 = ext_k<BK, C::CPBK>(kw1, 2 * ks + 1);
+        for (int ks = 0; ks < C::KSTEPS; ++ks) {
+#pragma unroll
+            for (int stt = 0; stt < 4; ++stt) {
+                const uint32_t a0 = ext_k<BK, C::CPBK>(kw[stt][0], 2 * ks);
+                const uint32_t a1 = ext_k<BK, C::CPBK>(kw[stt][1], 2 * ks);
+                const uint32_t a2 = ext_k<BK, C::CPBK>(kw[stt][0], 2 * ks + 1);
+                const uint32_t a3 = ext_k<BK, C::CPBK>(kw[stt][1], 2 * ks + 1);
 #pragma unroll
                 for (int nt = 0; nt < C::NT; ++nt)
                     mma_f16(S[stt][nt], a0, a1, a2, a3, qB[nt][ks][0], qB[nt][ks][1]);
             }
         }
 
-        // ---- combine hi/lo pieces; logits (log2 units); block max per head
-        float L2[4][TPT][2];
-        int tokl[4][TPT];
+        // ---- logits (log2 units): hi + lo columns, then the per-token affine terms
+        float L2[4][2][C::NT];
+        float bm[C::NT];
 #pragma unroll
-        for (int stt = 0; stt < 4; ++stt) {
-            float v[TPT][2];
-            if constexpr (G == 4) {
-                const bool lo_side = t >= 2;
-                const float s0 = lo_side ? S[stt][0][0] : S[stt][0][2];
-                const float s1 = lo_side ? S[stt][0][1] : S[stt][0][3];
-                const float r0 = __shfl_xor_sync(0xffffffffu, s0, 2);
-                const float r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
-                v[0][0] = (lo_side ? S[stt][0][2] : S[stt][0][0]) + r0;
-                v[0][1] = (lo_side ? S[stt][0][3] : S[stt][0][1]) + r1;
-                tokl[stt][0] = 16 * stt + g + (lo_side ? 8 : 0);
-            } else {
-#pragma unroll
-                for (int tk = 0; tk < 2; ++tk) {
-                    v[tk][0] = S[stt][0][2 * tk] + S[stt][1][2 * tk];
-                    v[tk][1] = S[stt][0][2 * tk + 1] + S[stt][1][2 * tk + 1];
-                    tokl[stt][tk] = 16 * stt + g + 8 * tk;
-                }
-            }
-#pragma unroll
-            for (int tk = 0; tk < TPT; ++tk) {
-                const int tl = tokl[stt][tk];
-                const bool valid = tok0 + tl < t_end;
-                const float2 sz = half2_bits_to_float2(kszw[tl]);
-                const float a = sz.x * cs;
-                L2[stt][tk][0] = valid ? fmaf(a, v[tk][0], sz.y * wq0) : -INFINITY;
-                L2[stt][tk][1] = valid ? fmaf(a, v[tk][1], sz.y * wq1) : -INFINITY;
-            }
-        }
-        float bm[2] = {-INFINITY, -INFINITY};
+        for (int nt = 0; nt < C::NT; ++nt)
+            bm[nt] = -INFINITY;
 #pragma unroll
         for (int stt = 0; stt < 4; ++stt)
 #pragma unroll
-            for (int tk = 0; tk < TPT; ++tk) {
-                bm[0] = fmaxf(bm[0], L2[stt][tk][0]);
-                bm[1] = fmaxf(bm[1], L2[stt][tk][1]);
+            for (int tk = 0; tk < 2; ++tk) {
+                const int tl = 16 * stt + g + 8 * tk;
+                const float2 sz = half2_bits_to_float2(kszw[tl]);
+                const float a = sz.x * cs;
+                const bool valid = FULL || (tok0 + tl < t_end);
+#pragma unroll
+                for (int nt = 0; nt < C::NT; ++nt) {
+                    const float v = S[stt][nt][2 * tk] + S[stt][nt][2 * tk + 1];
+                    float l2 = fmaf(a, v, sz.y * wq[nt]);
+                    if constexpr (!FULL)
+                        l2 = valid ? l2 : -INFINITY;
+                    L2[stt][tk][nt] = l2;
+                    bm[nt] = fmaxf(bm[nt], l2);
+                }
             }
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            if constexpr (G == 4)
-                bm[hh] = fmaxf(bm[hh], __shfl_xor_sync(0xffffffffu, bm[hh], 2));
-            bm[hh] = fmaxf(bm[hh], __shfl_xor_sync(0xffffffffu, bm[hh], 4));
-            bm[hh] = fmaxf(bm[hh], __shfl_xor_sync(0xffffffffu, bm[hh], 8));
-            bm[hh] = fmaxf(bm[hh], __shfl_xor_sync(0xffffffffu, bm[hh], 16));
-            if (bm[hh] > m_run[hh] + kLazy) {
-                const float alpha = ex2(m_run[hh] - bm[hh]);
-                l_run[hh] *= alpha;
-                lz_run[hh] *= alpha;
+        for (int nt = 0; nt < C::NT; ++nt) {
+            bm[nt] = fmaxf(bm[nt], __shfl_xor_sync(0xffffffffu, bm[nt], 4));
+            bm[nt] = fmaxf(bm[nt], __shfl_xor_sync(0xffffffffu, bm[nt], 8));
+            bm[nt] = fmaxf(bm[nt], __shfl_xor_sync(0xffffffffu, bm[nt], 16));
+            if (bm[nt] > m_run[nt] + kLazy) {
+                const float alpha = ex2(m_run[nt] - bm[nt]);
+                l_run[nt] *= alpha;
+                lz_run[nt] *= alpha;
 #pragma unroll
                 for (int m = 0; m < C::MT; ++m)
 #pragma unroll
-                    for (int nt = 0; nt < C::NT; ++nt) {
-                        O[m][nt][hh] *= alpha;
-                        O[m][nt][2 + hh] *= alpha;
-                    }
-                m_run[hh] = bm[hh];
+                    for (int i = 0; i < 4; ++i)
+                        O[m][nt][i] *= alpha;
+                m_run[nt] = bm[nt];
             }
         }
 
-        // ---- probabilities, value-scale products P' = p * s^v split into f16 hi/lo,
-        //      written transposed (column = head piece, slot pairs (j, j+8))
+        // ---- P' = p * s^v as float16 hi/lo, written transposed: column 8nt + 2t (hi) and
+        //      8nt + 2t + 1 (lo), slots (2g, 2g+1) = tokens (g, g+8) of the sub-tile
 #pragma unroll
         for (int stt = 0; stt < 4; ++stt) {
-            __half ph[TPT][2][2];               // [token][head][hi/lo]
-#pragma unroll
-            for (int tk = 0; tk < TPT; ++tk) {
-                const int tl = tokl[stt][tk];
-                const bool valid = tok0 + tl < t_end;
-                const float2 vz = half2_bits_to_float2(vszw[tl]);
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const float p = ex2(L2[stt][tk][hh] - m_run[hh]);
-                    l_run[hh] += p;
-                    lz_run[hh] = valid ? fmaf(p, vz.y, lz_run[hh]) : lz_run[hh];
-                    const float pp = valid ? p * vz.x : 0.f;
-                    const __half hi = __float2half_rn(pp);
-                    const __half lo = __float2half_rn(pp - __half2float(hi));
-                    ph[tk][hh][0] = hi;
-                    ph[tk][hh][1] = lo;
-                }
+            const float2 vz0 = half2_bits_to_float2(vszw[16 * stt + g]);
+            const float2 vz1 = half2_bits_to_float2(vszw[16 * stt + g + 8]);
+            bool v0 = true, v1 = true;
+            if constexpr (!FULL) {
+                v0 = tok0 + 16 * stt + g < t_end;
+                v1 = tok0 + 16 * stt + g + 8 < t_end;
             }
-            if constexpr (G == 4) {
-                const int slot = 16 * stt + 2 * g + (t >= 2 ? 1 : 0);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    pbuf[(hp + hh) * C::PSTRIDE + slot] = ph[0][hh][0];
-                    pbuf[(G + hp + hh) * C::PSTRIDE + slot] = ph[0][hh][1];
+            for (int nt = 0; nt < C::NT; ++nt) {
+                const float p0 = ex2(L2[stt][0][nt] - m_run[nt]);
+                const float p1 = ex2(L2[stt][1][nt] - m_run[nt]);
+                l_run[nt] += p0 + p1;
+                float pp0 = p0 * vz0.x, pp1 = p1 * vz1.x;
+                float z0 = p0 * vz0.y, z1 = p1 * vz1.y;
+                if constexpr (!FULL) {
+                    pp0 = v0 ? pp0 : 0.f;
+                    pp1 = v1 ? pp1 : 0.f;
+                    z0 = v0 ? z0 : 0.f;
+                    z1 = v1 ? z1 : 0.f;
                 }
-            } else {
-                const int slot = 16 * stt + 2 * g;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int pc = 0; pc < 2; ++pc) {
-                        __half2 w2 = __halves2half2(ph[0][hh][pc], ph[1][hh][pc]);
-                        *reinterpret_cast<__half2 *>(&pbuf[(pc * G + hp + hh) * C::PSTRIDE + slot]) = w2;
-                    }
+                lz_run[nt] += z0 + z1;
+                const __half2 hi = __floats2half2_rn(pp0, pp1);
+                const float2 hif = __half22float2(hi);
+                const __half2 lo = __floats2half2_rn(pp0 - hif.x, pp1 - hif.y);
+                __half *col = pbuf + (8 * nt + 2 * t) * C::PSTRIDE + 16 * stt + 2 * g;
+                *reinterpret_cast<__half2 *>(col) = hi;
+                *reinterpret_cast<__half2 *>(col + C::PSTRIDE) = lo;
             }
         }
         __syncwarp();
@@ -507,6 +508,23 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3) decode_kernel(DecodePara
             }
         }
         __syncwarp();
+    };
+
+    for (int jj = 0; jj < my_nblk; ++jj) {
+        const int s = jj % kDecodeStages;
+        if (!mbar_wait_bounded(&bars[s], (jj / kDecodeStages) & 1)) {
+            timed_out = true;
+            // wait (bounded) for this warp's copies still in flight, then stop
+            for (int k2 = jj + 1; k2 < jj + kDecodeStages && k2 < my_nblk; ++k2)
+                mbar_wait_bounded(&bars[k2 % kDecodeStages], (k2 / kDecodeStages) & 1);
+            break;
+        }
+        const unsigned char *st = wring + s * C::STAGE;
+        const int tok0 = t_begin + (warp + jj * kDecodeWarps) * kDecodeBlock;
+        if (tok0 + kDecodeBlock <= t_end)
+            block(st, tok0, std::true_type{});
+        else
+            block(st, tok0, std::false_type{});
         if (lane == 0 && jj + kDecodeStages < my_nblk) {
             fence_proxy_async_smem();
             issue(jj + kDecodeStages, s);
@@ -515,28 +533,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3) decode_kernel(DecodePara
     if (timed_out && lane == 0)
         flag(P.dev_err, KVQ_DEVERR_WAIT_TIMEOUT);
 
-    // ---- per-warp reduction across threads sharing heads
+    // ---- per-warp reduction across the 8 lanes sharing a head (same t)
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        if constexpr (G == 4) {
-            l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], 2);
-            lz_run[hh] += __shfl_xor_sync(0xffffffffu, lz_run[hh], 2);
-        }
+    for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
-            l_run[hh] += __shfl_xor_sync(0xffffffffu, l_run[hh], off);
-            lz_run[hh] += __shfl_xor_sync(0xffffffffu, lz_run[hh], off);
-        }
-    }
-    float Osum[C::MT][4];
-#pragma unroll
-    for (int m = 0; m < C::MT; ++m)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if constexpr (G == 4)
-                Osum[m][i] = O[m][0][i] + __shfl_xor_sync(0xffffffffu, O[m][0][i], 2);
-            else
-                Osum[m][i] = O[m][0][i] + O[m][1][i];
+            l_run[nt] += __shfl_xor_sync(0xffffffffu, l_run[nt], off);
+            lz_run[nt] += __shfl_xor_sync(0xffffffffu, lz_run[nt], off);
         }
 
     __syncthreads();                             // all warps are done with the ring
@@ -545,24 +548,24 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3) decode_kernel(DecodePara
     float *mw = reinterpret_cast<float *>(ring);                 // [W][G]
     float *lw = mw + kDecodeWarps * G;                           // [W][G]
     float *ow = lw + kDecodeWarps * G;                           // [W][G][D]
-    const bool writer = (G == 4) ? (t < 2) : true;
-    if (writer) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int head = hp + hh;
-            if (g == 0) {
-                mw[warp * G + head] = m_run[hh];
-                lw[warp * G + head] = l_run[hh];
-            }
+    for (int nt = 0; nt < C::NT; ++nt) {
+        const int head = 4 * nt + t;
+        if (g == 0) {
+            mw[warp * G + head] = m_run[nt];
+            lw[warp * G + head] = l_run[nt];
+        }
 #pragma unroll
-            for (int m = 0; m < C::MT; ++m) {
-                // rows g (n = 2m) and g+8 (n = 2m+1); value-field factor 2^(BV*(n % CPB))
-                const int n0 = 2 * m, n1 = 2 * m + 1;
-                const float f0 = __int_as_float((127 + 24 - BV * (n0 % C::CPBV)) << 23);
-                const float f1 = __int_as_float((127 + 24 - BV * (n1 % C::CPBV)) << 23);
-                ow[(warp * G + head) * D + 8 * n0 + g] = fmaf(Osum[m][hh], f0, lz_run[hh]);
-                ow[(warp * G + head) * D + 8 * n1 + g] = fmaf(Osum[m][2 + hh], f1, lz_run[hh]);
-            }
+        for (int m = 0; m < C::MT; ++m) {
+            // rows g (n = 2m) and g+8 (n = 2m+1); value-field factor 2^(BV*(n % CPB));
+            // columns 2t (hi) and 2t+1 (lo) of the same head
+            const int n0 = 2 * m, n1 = 2 * m + 1;
+            const float f0 = __int_as_float((127 + 24 - BV * (n0 % C::CPBV)) << 23);
+            const float f1 = __int_as_float((127 + 24 - BV * (n1 % C::CPBV)) << 23);
+            ow[(warp * G + head) * D + 8 * n0 + g] =
+                fmaf(O[m][nt][0] + O[m][nt][1], f0, lz_run[nt]);
+            ow[(warp * G + head) * D + 8 * n1 + g] =
+                fmaf(O[m][nt][2] + O[m][nt][3], f1, lz_run[nt]);
         }
     }
     __syncthreads();
@@ -640,23 +643,32 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
     {
         const int bb = L.qprep_bb;
         size_t smem = (size_t)((L.M ? D * (D + 1) : 0) + 2 * bb * G * D + 2 * bb) * 4;
-        cudaError_t e = cudaFuncSetAttribute(qprep_kernel<D, G, BK>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess)
-            return e;
+        static int qprep_attr = 0;          // set once per process (before any graph capture)
+        if (smem > 48 * 1024 && !qprep_attr) {
+            cudaError_t e = cudaFuncSetAttribute(qprep_kernel<D, G, BK>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)((D * (D + 1) + 2 * 8 * G * D + 16) * 4));
+            if (e != cudaSuccess)
+                return e;
+            qprep_attr = 1;
+        }
         dim3 grid(L.p.Hkv, (L.p.B + bb - 1) / bb);
         qprep_kernel<D, G, BK><<<grid, 256, smem, st>>>(L.q, L.q_bf16, L.M, L.p.B, L.p.Hq,
                                                        L.p.Hkv, bb, const_cast<uint32_t *>(L.p.qfrag),
                                                        const_cast<float *>(L.p.qscale),
                                                        const_cast<float *>(L.p.qw), L.p.ticket);
-        e = cudaGetLastError();
+        cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
     }
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, BK, BV>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess)
-        return e;
+    static int decode_attr = 0;
+    if (!decode_attr) {
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, BK, BV>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess)
+            return e;
+        decode_attr = 1;
+    }
     dim3 grid(L.p.nsplit, L.p.Hkv, L.p.B);
     decode_kernel<D, G, BK, BV><<<grid, kDecodeWarps * 32, C::SMEM, st>>>(L.p);
     return cudaGetLastError();

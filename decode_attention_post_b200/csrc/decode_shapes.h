@@ -8,7 +8,8 @@
 namespace kvq {
 
 constexpr int kDecodeWarps = 4;     // warps per decode CTA
-constexpr int kDecodeStages = 3;    // bulk-copy ring depth per warp
+constexpr int kDecodeStages = 2;    // bulk-copy ring depth per warp
+constexpr int kDecodeMinBlocks = 4; // resident CTAs per SM the register budget targets
 constexpr int kDecodeBlock = 64;    // tokens per ring stage
 
 struct DecodeParams {

@@ -98,14 +98,14 @@ static int num_sms()
     return sms;
 }
 
-// Splits along the tokens so that about 4 waves of 3 resident CTAs per SM cover the
+// Splits along the tokens so that about 4 waves of the resident CTAs per SM cover the
 // (sequence, KV head) pairs; each split is a whole number of 64-token blocks.
 // KVQ_DECODE_SPLITS overrides the count (tuning).
 static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens)
 {
     const int blocks = max_seqlen > 0 ? (max_seqlen + kDecodeBlock - 1) / kDecodeBlock : 1;
     const long pairs = (long)B * Hkv;
-    const long target = (long)num_sms() * 3 * 4;
+    const long target = (long)num_sms() * kDecodeMinBlocks * 4;
     long ns = (target + pairs - 1) / pairs;
     if (const char *e = getenv("KVQ_DECODE_SPLITS"))
         ns = atol(e);
@@ -285,7 +285,7 @@ kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const 
     L.G = Hq / c->Hkv;
     L.bits_k = c->qp.bits_k;
     L.bits_v = c->qp.bits_v;
-    L.qprep_bb = 2;
+    L.qprep_bb = 4;
     cudaError_t e = launch_decode(L, (cudaStream_t)stream);
     if (e != cudaSuccess)
         KVQ_FAIL(KVQ_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
