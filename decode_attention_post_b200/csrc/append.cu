@@ -285,11 +285,23 @@ cudaError_t launch_append_fp32(const void *k, const void *v, int in_bf16, const 
 
 }  // namespace
 
-cudaError_t append_fp32(const void *k, const void *v, int in_bf16, const float *Tk,
-                        const float *Tv, int B, int n, const kvq_cache *c, int kappa,
-                        const int32_t *pos, int32_t *dev_err, cudaStream_t st)
+cudaError_t append_mma(const void *k, const void *v, const float *Tk, const float *Tv, int B,
+                       int n, const kvq_cache *c, int kappa, const int32_t *pos, int32_t *dev_err,
+                       cudaStream_t st);
+
+// Chunks of bfloat16 inputs with both transforms go to the tensor-core kernel; float32
+// inputs, identity transforms, small (decode-time) appends and unaligned inputs use the
+// float32 CUDA-core kernel.
+cudaError_t append_launch(const void *k, const void *v, int in_bf16, const float *Tk,
+                          const float *Tv, int B, int n, const kvq_cache *c, int kappa,
+                          const int32_t *pos, int32_t *dev_err, cudaStream_t st)
 {
-    const bool small = (long)B * n <= 2048;
+    const long tokens = (long)B * n;
+    const bool a16 = ((uintptr_t)k % 16 == 0) && ((uintptr_t)v % 16 == 0) &&
+                     ((uintptr_t)Tk % 16 == 0) && ((uintptr_t)Tv % 16 == 0);
+    if (in_bf16 && Tk && Tv && a16 && tokens >= 256)
+        return append_mma(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
+    const bool small = tokens <= 2048;
     if (c->d == 64)
         return small ? launch_append_fp32<64, 1>(k, v, in_bf16, Tk, Tv, B, n, c, kappa, pos, dev_err, st)
                      : launch_append_fp32<64, 4>(k, v, in_bf16, Tk, Tv, B, n, c, kappa, pos, dev_err, st);

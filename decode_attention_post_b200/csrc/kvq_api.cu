@@ -11,9 +11,9 @@
 
 namespace kvq {
 
-cudaError_t append_fp32(const void *k, const void *v, int in_bf16, const float *Tk,
-                        const float *Tv, int B, int n, const kvq_cache *c, int kappa,
-                        const int32_t *pos, int32_t *dev_err, cudaStream_t st);
+cudaError_t append_launch(const void *k, const void *v, int in_bf16, const float *Tk,
+                          const float *Tv, int B, int n, const kvq_cache *c, int kappa,
+                          const int32_t *pos, int32_t *dev_err, cudaStream_t st);
 cudaError_t launch_bf16_decode(const void *q, int Hq, const void *k, const void *v, int B,
                                int Hkv, int T_cap, int d, const int32_t *seqlens, int max_seqlen,
                                void *out, void *ws, int nsplit, int split_tokens,
@@ -218,7 +218,7 @@ kvq_status kvq_quantize_append(const void *k, const void *v, kvq_dtype in_dtype,
         return KVQ_OK;
     if (!k || !v || !pos)
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "k, v and pos must not be NULL");
-    cudaError_t e = append_fp32(k, v, in_dtype == KVQ_BF16, T_k, T_v, cache->B, n, cache,
+    cudaError_t e = append_launch(k, v, in_dtype == KVQ_BF16, T_k, T_v, cache->B, n, cache,
                                 kappa_of(qp->clip_alpha, qp->group), pos, dev_err,
                                 (cudaStream_t)stream);
     if (e != cudaSuccess)

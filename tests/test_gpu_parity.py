@@ -189,6 +189,50 @@ def test_append_with_transform_end_to_end(cfg, B, n, pos, dtype):
     assert frac <= 1e-3, frac
 
 
+MMA_APPEND_CASES = [
+    # (d, bits_k, bits_v, group, clip_alpha, B, n, pos): bf16 chunks of >= 256 tokens take
+    # the tensor-core transform path; kappa 0, 1 and the general kappa >= 2 path
+    (64, 2, 2, 64, 0.01, 3, 130, [0, 200, 64]),
+    (128, 2, 2, 128, 0.01, 2, 300, [0, 212]),
+    (128, 4, 2, 128, 0.005, 1, 512, [0]),
+    (128, 4, 4, 32, 0.1, 2, 140, [5, 300]),
+    (64, 2, 4, 64, 0.05, 2, 160, [96, 0]),
+]
+
+
+@pytest.mark.parametrize("d,bk,bv,group,alpha,B,n,pos", MMA_APPEND_CASES)
+def test_append_tensor_core_path_with_identity_matrix_bit_exact(d, bk, bv, group, alpha, B, n, pos):
+    """T = I passed as a matrix: bf16 inputs times the identity on tensor cores reproduce
+    the inputs exactly, so clipping, quantization and packing of the tensor-core path must
+    equal the oracle's (T = None) bit for bit."""
+    cfg = synth.Config(97, "mma", B=B, Hq=4 * 2, Hkv=2, d=d, T_cap=512, bits_k=bk, bits_v=bv,
+                       group=group, clip_alpha=alpha, in_dtype="bf16", q_dtype="bf16",
+                       out_dtype="bf16", seq_lo=1, seq_hi=1)
+    k, v = _inputs(cfg, B, n, "bf16")
+    eye = np.broadcast_to(np.eye(d, dtype=np.float32), (cfg.Hkv, d, d)).copy()
+    oc = oracle.Cache(B, cfg.Hkv, cfg.T_cap, d, bk, bv, group)
+    oracle.quantize_append(k, v, None, None, bk, bv, group, alpha, oc, pos)
+    gc, err = gpu_append(cfg, k, v, eye, eye, pos)
+    assert err == 0
+    for name, a, b in zip(("k_codes", "k_sz", "v_codes", "v_sz"), planes_to_host(gc), oc.planes()):
+        assert np.array_equal(a, b.view(np.uint8)), name
+
+
+@pytest.mark.parametrize("d,bk,bv,group,alpha,B,n,pos", MMA_APPEND_CASES[:3])
+def test_append_tensor_core_path_end_to_end(d, bk, bv, group, alpha, B, n, pos):
+    cfg = synth.Config(96, "mma", B=B, Hq=8, Hkv=2, d=d, T_cap=512, bits_k=bk, bits_v=bv,
+                       group=group, clip_alpha=alpha, in_dtype="bf16", q_dtype="bf16",
+                       out_dtype="bf16", seq_lo=1, seq_hi=1)
+    k, v = _inputs(cfg, B, n, "bf16")
+    Tk, Tv, _ = synth.transforms(cfg)
+    oc = oracle.Cache(B, cfg.Hkv, cfg.T_cap, d, bk, bv, group)
+    oracle.quantize_append(k, v, Tk, Tv, bk, bv, group, alpha, oc, pos)
+    gc, err = gpu_append(cfg, k, v, Tk, Tv, pos)
+    assert err == 0
+    frac = _compare_codes_end_to_end(gc, oc, cfg, B, pos, n)
+    assert frac <= 1e-3, frac
+
+
 def test_append_out_of_range_sequence_is_skipped_and_flagged():
     cfg = small(synth.CONFIGS[1], T_cap=64)
     k, v = _inputs(cfg, 2, 10, "f32")
