@@ -51,6 +51,28 @@ def step_bytes(cfg, seqlens):
     return decode, append
 
 
+def reduce_max(x: float, world: int, device="cpu") -> float:
+    """Max of a per-rank scalar over all ranks (the timing rule: slowest rank counts)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_gbs(bytes_per_rank: float, ms_per_step_max: float, world: int) -> float:
+    """Whole-job GB/s: every rank processes its own batch of the same size, so the job
+    moves world * bytes_per_rank per step in the slowest rank's step time."""
+    return world * bytes_per_rank / (ms_per_step_max * 1e-3) / 1e9
+
+
+def rank_sequence_offset(b: int, rank: int, B: int) -> int:
+    """Index of the synthetic sequence that rank `rank` uses as its sequence b."""
+    return b + rank * B
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -146,7 +168,7 @@ class Workload:
         zero = torch.zeros(1, dtype=torch.int32, device=device)
         for b in range(cfg.B):
             n = int(self.seqlens[b])
-            src = b + rank * cfg.B                       # each rank its own sequences
+            src = rank_sequence_offset(b, rank, cfg.B)   # each rank its own sequences
             k = synth.keys(cfg, src, 0, n)
             v = synth.values(cfg, src, 0, n)
             kd, vd = bf(k), bf(v)                        # [n][Hkv][d] bf16
@@ -229,11 +251,7 @@ def run_gpu(args):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, device)
 
     cfg = synth.CONFIGS[CONFIG_IDX]
     w = Workload(cfg, rank, device, with_bf16=not args.no_extras)
@@ -268,7 +286,7 @@ def run_gpu(args):
     clocks = sampler.summary()
     ms_total = max_over_ranks(t0.elapsed_time(t1))
     ms_step = ms_total / K
-    value = world * (dec_bytes + app_bytes) / (ms_step * 1e-3) / 1e9
+    value = weak_scaling_gbs(dec_bytes + app_bytes, ms_step, world)
 
     # ---- the dominant kernel (the decode call: q prologue + split-K decode) timed alone
     dec_ms = statistics.mean(time_events(w.decode, min(K, 500), stream))
@@ -309,7 +327,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / Ke
-    e2e_value = world * (dec_bytes + app_bytes) / (e2e_ms * 1e-3) / 1e9
+    e2e_value = weak_scaling_gbs(dec_bytes + app_bytes, e2e_ms, world)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,

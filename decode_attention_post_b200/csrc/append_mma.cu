@@ -31,7 +31,7 @@ struct MmaSmem {
     static constexpr int CS = D + 16;      // code bytes per staged token row
     __nv_bfloat16 Thi[D * TS];
     __nv_bfloat16 Tlo[D * TS];
-    __nv_bfloat16 X[kMmaWarps][16 * TS];
+    __nv_bfloat16 X[kMmaWarps][2][16 * TS];      // double-buffered input rows
     uint8_t codes[kMmaWarps][16 * CS];
 };
 
@@ -132,25 +132,41 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
     }
     __syncthreads();
 
-    __nv_bfloat16 *X = sm.X[warp];
     uint8_t *codes = sm.codes[warp];
-    for (long tile = (long)blockIdx.x * kMmaWarps + warp; tile < tiles;
-         tile += (long)gridDim.x * kMmaWarps) {
-        const long u0 = tile * 16;
-        // ---- stage the 16 input rows (bf16) of this KV head
-        constexpr int CH = D / 8;                     // 16-byte chunks per row
+    constexpr int CH = D / 8;                         // 16-byte chunks per input row
+    // cp.async the 16 input rows of `tile` into buffer `buf` (rows past the end zero-fill)
+    auto fetch = [&](long tile, int buf) {
+        __nv_bfloat16 *Xb = sm.X[warp][buf];
 #pragma unroll
         for (int c = lane; c < 16 * CH; c += 32) {
             const int r = c / CH, ch = c % CH;
-            const long u = u0 + r;
-            uint4 val = make_uint4(0, 0, 0, 0);
+            const long u = tile * 16 + r;
+            const __nv_bfloat16 *src = in;
+            uint32_t bytes = 0;
             if (u < total) {
                 const long b = u / n, i = u % n;
-                val = *reinterpret_cast<const uint4 *>(in + (((size_t)b * n + i) * Hkv + h) * D + 8 * ch);
+                src = in + (((size_t)b * n + i) * Hkv + h) * D + 8 * ch;
+                bytes = 16;
             }
-            *reinterpret_cast<uint4 *>(X + r * TS + 8 * ch) = val;
+            cp_async16(Xb + r * TS + 8 * ch, src, bytes);
+        }
+        cp_async_commit();
+    };
+    const long stride = (long)gridDim.x * kMmaWarps;
+    long tile = (long)blockIdx.x * kMmaWarps + warp;
+    int buf = 0;
+    if (tile < tiles)
+        fetch(tile, 0);
+    for (; tile < tiles; tile += stride, buf ^= 1) {
+        const long u0 = tile * 16;
+        if (tile + stride < tiles) {
+            fetch(tile + stride, buf ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
         __syncwarp();
+        const __nv_bfloat16 *X = sm.X[warp][buf];
 
         // ---- X~ = X . T^T on tensor cores
         float acc[NT][4];

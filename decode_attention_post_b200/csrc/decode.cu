@@ -38,6 +38,7 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 4.0f;     // rescale the running sums only when the max grows by > 2^4
+constexpr int kQprepSeqs = 2;     // sequences per q-prologue CTA
 
 template <int D, int G, int BK, int BV>
 struct Cfg {
@@ -122,7 +123,8 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u)
 
 // ---------------------------------------------------------------- q prologue
 
-// One CTA per (KV head, chunk of `bb` sequences). Computes q~ = M q in float32, then
+// One CTA per (KV head, chunk of `bb` sequences), D threads: thread i owns output dim i
+// and streams row i of M with 16-byte loads. Computes q~ = M q in float32, then
 //   eq  = power-of-two exponent bringing max|q~| * 2^(BK*(CPB-1)) to about 2^14,
 //   frag[nt][ks][lane][2] = float16 hi/lo pieces of q~ * 2^eq * 2^(BK*(CPB-1-k)) laid
 //                           out as the B operand of the Q.K product; n-tile nt holds
@@ -131,87 +133,68 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u)
 //   w_h = log2(e) / sqrt(d) * sum_j q~_hj,
 // and zeroes the split-merge ticket of the (sequence, KV head).
 template <int D, int G, int BK>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(D)
 qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M, int B, int Hq,
              int Hkv, int bb, uint32_t *__restrict__ qfrag, float *__restrict__ qscale,
              float *__restrict__ qw, int *__restrict__ ticket)
 {
     constexpr int CPB = 8 / BK, KSTEPS = D / 16, NT = (2 * G) / 8, WPT = D * BK / 128;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    float *Mt = reinterpret_cast<float *>(smem_raw);                 // [D][D+1] or unused
-    float *qs = Mt + (M ? D * (D + 1) : 0);                            // [bb*G][D]
-    float *qt = qs + bb * G * D;                                       // [bb*G][D]
-    float *red = qt + bb * G * D;                                      // [bb][2]
+    constexpr int NVMAX = kQprepSeqs * G;
+    __shared__ __align__(16) float qs[NVMAX * D];     // input vectors
+    __shared__ __align__(16) float qt[NVMAX * D];     // transformed vectors
+    __shared__ float red[kQprepSeqs];
 
     const int h = blockIdx.x;
     const int b0 = blockIdx.y * bb;
     const int nb = min(bb, B - b0);
-    const int tid = threadIdx.x;
-    if (tid < bb)
-        red[tid] = 0.f;
-
-    if (M) {
-        const float4 *Mh4 = reinterpret_cast<const float4 *>(M + (size_t)h * D * D);
-        constexpr int N4 = D * D / 4 / 256;
-#pragma unroll 16
-        for (int it = 0; it < N4; ++it) {
-            const int idx4 = tid + 256 * it;
-            const float4 v4 = Mh4[idx4];
-            const int i = (4 * idx4) / D, j = (4 * idx4) % D;
-            Mt[(j + 0) * (D + 1) + i] = v4.x;
-            Mt[(j + 1) * (D + 1) + i] = v4.y;
-            Mt[(j + 2) * (D + 1) + i] = v4.z;
-            Mt[(j + 3) * (D + 1) + i] = v4.w;
-        }
-    }
-    // queries stored transposed, qs[j][v] (v = sequence-in-chunk * G + head), so that one
-    // 16-byte load feeds four vectors
     const int NV = nb * G;
-    for (int idx = tid; idx < NV * D; idx += 256) {
+    const int tid = threadIdx.x;
+    if (tid < kQprepSeqs)
+        red[tid] = 0.f;
+    for (int idx = tid; idx < NV * D; idx += D) {
         const int v = idx / D, j = idx % D;
         const int bi = v / G, gg = v % G;
-        qs[j * (bb * G) + v] = load_in(q, q_bf16, ((size_t)(b0 + bi) * Hq + h * G + gg) * D + j);
+        qs[idx] = load_in(q, q_bf16, ((size_t)(b0 + bi) * Hq + h * G + gg) * D + j);
     }
     __syncthreads();
-    // thread -> (output dim i, group of 4 vectors); register-tiled over the 4 vectors
     {
-        const int VG = bb * G / 4;                          // vector groups of 4
-        for (int task = tid; task < D * VG; task += 256) {
-            const int i = task % D, vg = task / D;
-            if (4 * vg >= NV)
-                continue;
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            if (M) {
-#pragma unroll 8
-                for (int j = 0; j < D; ++j) {
-                    const float m = Mt[j * (D + 1) + i];
-                    const float4 x = *reinterpret_cast<const float4 *>(qs + j * (bb * G) + 4 * vg);
-                    a0 = fmaf(m, x.x, a0);
-                    a1 = fmaf(m, x.y, a1);
-                    a2 = fmaf(m, x.z, a2);
-                    a3 = fmaf(m, x.w, a3);
+        const int i = tid;
+        float acc[NVMAX];
+#pragma unroll
+        for (int v = 0; v < NVMAX; ++v)
+            acc[v] = 0.f;
+        if (M) {
+            const float4 *Mrow = reinterpret_cast<const float4 *>(M + ((size_t)h * D + i) * D);
+#pragma unroll 4
+            for (int c = 0; c < D / 4; ++c) {
+                const float4 m = __ldg(Mrow + c);
+#pragma unroll
+                for (int v = 0; v < NVMAX; ++v) {
+                    if (v < NV) {
+                        const float4 x = reinterpret_cast<const float4 *>(qs + v * D)[c];
+                        acc[v] = fmaf(m.x, x.x, fmaf(m.y, x.y, fmaf(m.z, x.z, fmaf(m.w, x.w, acc[v]))));
+                    }
                 }
-            } else {
-                const float4 x = *reinterpret_cast<const float4 *>(qs + i * (bb * G) + 4 * vg);
-                a0 = x.x;
-                a1 = x.y;
-                a2 = x.z;
-                a3 = x.w;
             }
-            qt[(4 * vg + 0) * D + i] = a0;
-            qt[(4 * vg + 1) * D + i] = a1;
-            qt[(4 * vg + 2) * D + i] = a2;
-            qt[(4 * vg + 3) * D + i] = a3;
+        } else {
+#pragma unroll
+            for (int v = 0; v < NVMAX; ++v)
+                if (v < NV)
+                    acc[v] = qs[v * D + i];
         }
+#pragma unroll
+        for (int v = 0; v < NVMAX; ++v)
+            if (v < NV)
+                qt[v * D + i] = acc[v];
     }
     __syncthreads();
     // per sequence: max |q~| over its G heads; per head: sum of q~
     const int warp = tid >> 5, lane = tid & 31;
     const float sm = rsqrtf((float)D);
-    for (int v = warp; v < nb * G; v += 8) {
+    for (int v = warp; v < NV; v += D / 32) {
         float s = 0.f, a = 0.f;
         for (int j = lane; j < D; j += 32) {
-            float x = qt[v * D + j];
+            const float x = qt[v * D + j];
             s += x;
             a = fmaxf(a, fabsf(x));
         }
@@ -221,7 +204,7 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
             a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
         }
         if (lane == 0) {
-            int bi = v / G, gg = v % G;
+            const int bi = v / G, gg = v % G;
             qw[(size_t)(b0 + bi) * Hq + h * G + gg] = kLog2e * sm * s;
             atomicMax(reinterpret_cast<int *>(&red[bi]), __float_as_int(a));   // a >= 0
         }
@@ -240,7 +223,7 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
             ticket[pair] = 0;
         }
         uint32_t *fr = qfrag + pair * (size_t)(NT * KSTEPS * 64);
-        for (int idx = tid; idx < NT * KSTEPS * 64; idx += 256) {
+        for (int idx = tid; idx < NT * KSTEPS * 64; idx += D) {
             const int rho = idx & 1, ln = (idx >> 1) & 31, ks = (idx >> 6) % KSTEPS;
             const int nt = (idx >> 6) / KSTEPS;
             const int g = ln >> 2, t = ln & 3;
@@ -321,20 +304,41 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_ke
     }
     __syncwarp();
 
+    // Block jj of this warp into stage s: lane 0 announces the stage's bytes, then lanes
+    // 0..3 each issue one bulk copy (K codes, K scale/zero, V codes, V scale/zero).
+    // Called by the whole warp.
     auto issue = [&](int jj, int s) {
         const int tok0 = t_begin + (warp + jj * kDecodeWarps) * kDecodeBlock;
         unsigned char *st = wring + s * C::STAGE;
-        mbar_arrive_expect_tx(&bars[s], C::STAGE);
-        bulk_g2s(st, kc + (size_t)tok0 * C::ROWK, C::KC_BYTES, &bars[s]);
-        bulk_g2s(st + C::KC_BYTES, ksz + (size_t)tok0 * 4, C::SZ_BYTES, &bars[s]);
-        bulk_g2s(st + C::KC_BYTES + C::SZ_BYTES, vc + (size_t)tok0 * (D * BV / 8), C::VC_BYTES,
-                 &bars[s]);
-        bulk_g2s(st + C::KC_BYTES + C::SZ_BYTES + C::VC_BYTES, vsz + (size_t)tok0 * 4,
-                 C::SZ_BYTES, &bars[s]);
+        if (lane == 0)
+            mbar_arrive_expect_tx(&bars[s], C::STAGE);
+        __syncwarp();
+        if (lane < 4) {
+            const void *src;
+            unsigned char *dst;
+            uint32_t bytes;
+            if (lane == 0) {
+                src = kc + (size_t)tok0 * C::ROWK;
+                dst = st;
+                bytes = C::KC_BYTES;
+            } else if (lane == 1) {
+                src = ksz + (size_t)tok0 * 4;
+                dst = st + C::KC_BYTES;
+                bytes = C::SZ_BYTES;
+            } else if (lane == 2) {
+                src = vc + (size_t)tok0 * (D * BV / 8);
+                dst = st + C::KC_BYTES + C::SZ_BYTES;
+                bytes = C::VC_BYTES;
+            } else {
+                src = vsz + (size_t)tok0 * 4;
+                dst = st + C::KC_BYTES + C::SZ_BYTES + C::VC_BYTES;
+                bytes = C::SZ_BYTES;
+            }
+            bulk_g2s(dst, src, bytes, &bars[s]);
+        }
     };
-    if (lane == 0)
-        for (int jj = 0; jj < kDecodeStages && jj < my_nblk; ++jj)
-            issue(jj, jj);
+    for (int jj = 0; jj < kDecodeStages && jj < my_nblk; ++jj)
+        issue(jj, jj);
 
     // q~ operand fragments and per-head constants
     uint32_t qB[C::NT][C::KSTEPS][2];
@@ -525,10 +529,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_ke
             block(st, tok0, std::true_type{});
         else
             block(st, tok0, std::false_type{});
-        if (lane == 0 && jj + kDecodeStages < my_nblk) {
-            fence_proxy_async_smem();
+        // every lane has consumed the stage (its values are in registers) before the
+        // warp-synchronous refill below
+        if (jj + kDecodeStages < my_nblk)
             issue(jj + kDecodeStages, s);
-        }
     }
     if (timed_out && lane == 0)
         flag(P.dev_err, KVQ_DEVERR_WAIT_TIMEOUT);
@@ -641,22 +645,11 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
     using C = Cfg<D, G, BK, BV>;
     // q prologue
     {
-        const int bb = L.qprep_bb;
-        size_t smem = (size_t)((L.M ? D * (D + 1) : 0) + 2 * bb * G * D + 2 * bb) * 4;
-        static int qprep_attr = 0;          // set once per process (before any graph capture)
-        if (smem > 48 * 1024 && !qprep_attr) {
-            cudaError_t e = cudaFuncSetAttribute(qprep_kernel<D, G, BK>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)((D * (D + 1) + 2 * 8 * G * D + 16) * 4));
-            if (e != cudaSuccess)
-                return e;
-            qprep_attr = 1;
-        }
-        dim3 grid(L.p.Hkv, (L.p.B + bb - 1) / bb);
-        qprep_kernel<D, G, BK><<<grid, 256, smem, st>>>(L.q, L.q_bf16, L.M, L.p.B, L.p.Hq,
-                                                       L.p.Hkv, bb, const_cast<uint32_t *>(L.p.qfrag),
-                                                       const_cast<float *>(L.p.qscale),
-                                                       const_cast<float *>(L.p.qw), L.p.ticket);
+        dim3 grid(L.p.Hkv, (L.p.B + kQprepSeqs - 1) / kQprepSeqs);
+        qprep_kernel<D, G, BK><<<grid, D, 0, st>>>(L.q, L.q_bf16, L.M, L.p.B, L.p.Hq, L.p.Hkv,
+                                                  kQprepSeqs, const_cast<uint32_t *>(L.p.qfrag),
+                                                  const_cast<float *>(L.p.qscale),
+                                                  const_cast<float *>(L.p.qw), L.p.ticket);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;

@@ -37,7 +37,6 @@ struct DecodeLaunch {
     int q_bf16;
     const float *M;
     int d, G, bits_k, bits_v;
-    int qprep_bb;        // sequences per q-prologue CTA
 };
 
 // Byte offsets of the decode workspace sections (each 256-byte aligned).

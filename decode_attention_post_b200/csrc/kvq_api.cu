@@ -285,7 +285,6 @@ kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const 
     L.G = Hq / c->Hkv;
     L.bits_k = c->qp.bits_k;
     L.bits_v = c->qp.bits_v;
-    L.qprep_bb = 4;
     cudaError_t e = launch_decode(L, (cudaStream_t)stream);
     if (e != cudaSuccess)
         KVQ_FAIL(KVQ_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
