@@ -7,10 +7,11 @@
 // Two kernels per call:
 //  qprep   q~ = T_k^{-T} q for every query head (float32), and from it the tensor-core
 //          operand fragments, the logit scale and sum(q~) per head.
-//  decode  split-K flash decode. CTA = (split, KV head, sequence), 4 warps. Each warp
-//          streams 64-token blocks (K codes, K scale/zero, V codes, V scale/zero) with
-//          cp.async.bulk into a private 3-stage shared-memory ring (mbarrier completion,
-//          bounded waits), and per block:
+//  decode  split-K flash decode. CTA = (KV head, sequence, split), 4 warps; launched as a
+//          programmatic dependent of qprep, it requests its first cache blocks before
+//          waiting for qprep. Each warp streams 64-token blocks (K codes, K scale/zero,
+//          V codes, V scale/zero) with cp.async.bulk into a private 2-stage shared-memory
+//          ring (mbarrier completion, bounded waits), and per block:
 //            S^T[16 tok x (hi,lo)*G] = Kcodes[16 tok x d] . q~'[d x 2G]   (mma f16, f32 acc)
 //            logit = log2(e)/sqrt(d) * (s_t * q~.c_t + z_t * sum q~)       (affine dequant
 //                    folded per token: x^ = z + c s)
@@ -65,7 +66,13 @@ struct Cfg {
     static constexpr int MERGE = kDecodeWarps * G * (D + 2) * 4;
     static constexpr int SMEM = (RING > MERGE ? RING : MERGE) + kDecodeWarps * PBUF +
                                 kDecodeWarps * kDecodeStages * 8 + 16;
+    // resident CTAs per SM the register budget targets: kDecodeMinBlocks, or fewer when
+    // shared memory (227 KB per SM, 1 KB reserved per CTA) holds fewer
+    static constexpr int SMEM_FIT = (227 * 1024) / (SMEM + 1024);
+    static constexpr int MINB = SMEM_FIT < kDecodeMinBlocks ? SMEM_FIT : kDecodeMinBlocks;
+    static_assert(MINB >= 1, "decode CTA does not fit in shared memory");
     static_assert(STAGE % 16 == 0, "stage alignment");
+    static_assert(MERGE % 16 == 0, "merge area alignment");
     static_assert(NT >= 1 && (2 * G) % 8 == 0, "G must be a multiple of 4");
 };
 
@@ -123,75 +130,123 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u)
 
 // ---------------------------------------------------------------- q prologue
 
-// One CTA per (KV head, chunk of `bb` sequences), D threads: thread i owns output dim i
-// and streams row i of M with 16-byte loads. Computes q~ = M q in float32, then
+// One CTA per (KV head, chunk of `bb` sequences), kQprepThreads threads. M_h is staged in
+// shared memory with one cp.async round trip (row stride D+4 floats: the float4 reads of
+// row i by 8 consecutive threads fall in distinct banks), the q vectors as qs[j][v].
+// Thread (i, part) accumulates output dim i of every vector over one of JP slices of j;
+// the slices are summed in shared memory. From q~ = M q (float32) it derives
 //   eq  = power-of-two exponent bringing max|q~| * 2^(BK*(CPB-1)) to about 2^14,
 //   frag[nt][ks][lane][2] = float16 hi/lo pieces of q~ * 2^eq * 2^(BK*(CPB-1-k)) laid
 //                           out as the B operand of the Q.K product; n-tile nt holds
 //                           heads 4nt..4nt+3, column 2h' = hi and 2h'+1 = lo of head 4nt+h',
 //   cs  = log2(e) / sqrt(d) / F with F = 2^(eq + BK*(CPB-1) - 24) the product scale,
 //   w_h = log2(e) / sqrt(d) * sum_j q~_hj,
-// and zeroes the split-merge ticket of the (sequence, KV head).
+// zeroes the split-merge ticket of each (sequence, KV head), and writes the zero output
+// of every empty sequence. It lets the dependent decode launch start at once: the decode
+// kernel requests its first cache blocks, then waits for this grid.
+constexpr int kQprepThreads = 256;
+
+template <int D, int G>
+struct QprepSmem {
+    static constexpr int NVMAX = kQprepSeqs * G;
+    static constexpr int JP = kQprepThreads / D;     // slices of the j range
+    static constexpr int MSTRIDE = D + 4;
+    static constexpr int BYTES = (D * MSTRIDE + D * NVMAX + JP * NVMAX * D + kQprepSeqs) * 4;
+};
+
 template <int D, int G, int BK>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kQprepThreads)
 qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M, int B, int Hq,
-             int Hkv, int bb, uint32_t *__restrict__ qfrag, float *__restrict__ qscale,
+             int Hkv, int bb, const int32_t *__restrict__ seqlens, int max_seqlen, void *out,
+             int out_bf16, uint32_t *__restrict__ qfrag, float *__restrict__ qscale,
              float *__restrict__ qw, int *__restrict__ ticket)
 {
     constexpr int CPB = 8 / BK, KSTEPS = D / 16, NT = (2 * G) / 8, WPT = D * BK / 128;
-    constexpr int NVMAX = kQprepSeqs * G;
-    __shared__ __align__(16) float qs[NVMAX * D];     // input vectors
-    __shared__ __align__(16) float qt[NVMAX * D];     // transformed vectors
-    __shared__ float red[kQprepSeqs];
+    using S = QprepSmem<D, G>;
+    constexpr int NVMAX = S::NVMAX, JP = S::JP, JL = D / JP;
+    extern __shared__ __align__(16) float qsm[];
+    float *Ms = qsm;                              // [D][D+4]
+    float *qs = Ms + D * S::MSTRIDE;              // [D][NVMAX]
+    float *pt = qs + D * NVMAX;                   // [JP][NVMAX][D]; slice 0 ends up as q~
+    float *red = pt + JP * NVMAX * D;             // [kQprepSeqs]
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int h = blockIdx.x;
     const int b0 = blockIdx.y * bb;
     const int nb = min(bb, B - b0);
     const int NV = nb * G;
     const int tid = threadIdx.x;
+    if (M) {
+        const float *Mh = M + (size_t)h * D * D;
+#pragma unroll
+        for (int k = 0; k < D * D / 4 / kQprepThreads; ++k) {
+            const int f = tid + k * kQprepThreads, r = f / (D / 4), c = 4 * (f % (D / 4));
+            cp_async16(Ms + r * S::MSTRIDE + c, Mh + (size_t)r * D + c, 16);
+        }
+        cp_async_commit();
+    }
     if (tid < kQprepSeqs)
         red[tid] = 0.f;
-    for (int idx = tid; idx < NV * D; idx += D) {
+    for (int idx = tid; idx < NVMAX * D; idx += kQprepThreads) {
         const int v = idx / D, j = idx % D;
         const int bi = v / G, gg = v % G;
-        qs[idx] = load_in(q, q_bf16, ((size_t)(b0 + bi) * Hq + h * G + gg) * D + j);
+        qs[j * NVMAX + v] =
+            v < NV ? load_in(q, q_bf16, ((size_t)(b0 + bi) * Hq + h * G + gg) * D + j) : 0.f;
     }
+    cp_async_wait<0>();
     __syncthreads();
     {
-        const int i = tid;
+        const int i = tid % D, jp = tid / D;          // jp is warp-uniform (D >= 64)
         float acc[NVMAX];
 #pragma unroll
         for (int v = 0; v < NVMAX; ++v)
             acc[v] = 0.f;
         if (M) {
-            const float4 *Mrow = reinterpret_cast<const float4 *>(M + ((size_t)h * D + i) * D);
-#pragma unroll 4
-            for (int c = 0; c < D / 4; ++c) {
-                const float4 m = __ldg(Mrow + c);
+            const float4 *Mrow = reinterpret_cast<const float4 *>(Ms + i * S::MSTRIDE + jp * JL);
+#pragma unroll 2
+            for (int j4 = 0; j4 < JL / 4; ++j4) {
+                const float4 m = Mrow[j4];
+                const float mj[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
-                for (int v = 0; v < NVMAX; ++v) {
-                    if (v < NV) {
-                        const float4 x = reinterpret_cast<const float4 *>(qs + v * D)[c];
-                        acc[v] = fmaf(m.x, x.x, fmaf(m.y, x.y, fmaf(m.z, x.z, fmaf(m.w, x.w, acc[v]))));
+                for (int jj = 0; jj < 4; ++jj) {
+                    const float4 *x =
+                        reinterpret_cast<const float4 *>(qs + (jp * JL + 4 * j4 + jj) * NVMAX);
+#pragma unroll
+                    for (int v4 = 0; v4 < NVMAX / 4; ++v4) {
+                        const float4 xv = x[v4];
+                        acc[4 * v4] = fmaf(mj[jj], xv.x, acc[4 * v4]);
+                        acc[4 * v4 + 1] = fmaf(mj[jj], xv.y, acc[4 * v4 + 1]);
+                        acc[4 * v4 + 2] = fmaf(mj[jj], xv.z, acc[4 * v4 + 2]);
+                        acc[4 * v4 + 3] = fmaf(mj[jj], xv.w, acc[4 * v4 + 3]);
                     }
                 }
             }
-        } else {
+        } else if (jp == 0) {
 #pragma unroll
             for (int v = 0; v < NVMAX; ++v)
-                if (v < NV)
-                    acc[v] = qs[v * D + i];
+                acc[v] = qs[i * NVMAX + v];
         }
 #pragma unroll
         for (int v = 0; v < NVMAX; ++v)
-            if (v < NV)
-                qt[v * D + i] = acc[v];
+            pt[(jp * NVMAX + v) * D + i] = acc[v];
     }
     __syncthreads();
+    if (JP > 1) {
+        for (int idx = tid; idx < NV * D; idx += kQprepThreads) {
+            float x = pt[idx];
+#pragma unroll
+            for (int jp = 1; jp < JP; ++jp)
+                x += pt[jp * NVMAX * D + idx];
+            pt[idx] = x;
+        }
+        __syncthreads();
+    }
+    const float *qt = pt;                         // [NVMAX][D]
     // per sequence: max |q~| over its G heads; per head: sum of q~
     const int warp = tid >> 5, lane = tid & 31;
     const float sm = rsqrtf((float)D);
-    for (int v = warp; v < NV; v += D / 32) {
+    for (int v = warp; v < NV; v += kQprepThreads / 32) {
         float s = 0.f, a = 0.f;
         for (int j = lane; j < D; j += 32) {
             const float x = qt[v * D + j];
@@ -223,7 +278,7 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
             ticket[pair] = 0;
         }
         uint32_t *fr = qfrag + pair * (size_t)(NT * KSTEPS * 64);
-        for (int idx = tid; idx < NT * KSTEPS * 64; idx += D) {
+        for (int idx = tid; idx < NT * KSTEPS * 64; idx += kQprepThreads) {
             const int rho = idx & 1, ln = (idx >> 1) & 31, ks = (idx >> 6) % KSTEPS;
             const int nt = (idx >> 6) / KSTEPS;
             const int g = ln >> 2, t = ln & 3;
@@ -243,13 +298,24 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
             }
             fr[idx] = packed;
         }
+        // an empty sequence (after clamping to [0, max_seqlen]) attends to nothing: zeros
+        const int sl = seqlens[b0 + bi];
+        if (sl <= 0 || max_seqlen == 0) {
+            for (int idx = tid; idx < G * D; idx += kQprepThreads) {
+                const size_t o = ((size_t)(b0 + bi) * Hq + h * G) * D + idx;
+                if (out_bf16)
+                    reinterpret_cast<__nv_bfloat16 *>(out)[o] = __float2bfloat16_rn(0.f);
+                else
+                    reinterpret_cast<float *>(out)[o] = 0.f;
+            }
+        }
     }
 }
 
 // ---------------------------------------------------------------- main decode
 
 template <int D, int G, int BK, int BV>
-__global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_kernel(DecodeParams P)
+__global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) decode_kernel(DecodeParams P)
 {
     using C = Cfg<D, G, BK, BV>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -259,7 +325,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_ke
                                                       kDecodeWarps * C::PBUF);
     int *flag_smem = reinterpret_cast<int *>(bars_all + kDecodeWarps * kDecodeStages);
 
-    const int sigma = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const size_t pair = (size_t)b * P.Hkv + h;
@@ -271,18 +337,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_ke
         seqlen = seqlen < 0 ? 0 : P.max_seqlen;
     }
     const int t_begin = sigma * P.split_tokens;
-    if (t_begin >= seqlen) {
-        if (sigma == 0) {                       // empty sequence: the output is 0
-            for (int idx = threadIdx.x; idx < G * D; idx += kDecodeWarps * 32) {
-                const size_t o = ((size_t)b * P.Hq + h * G + idx / D) * D + idx % D;
-                if (P.out_bf16)
-                    reinterpret_cast<__nv_bfloat16 *>(P.out)[o] = __float2bfloat16_rn(0.f);
-                else
-                    reinterpret_cast<float *>(P.out)[o] = 0.f;
-            }
-        }
-        return;
-    }
+    if (t_begin >= seqlen)
+        return;                                 // nothing here (the prologue zeroes empty ones)
     const int t_end = min(t_begin + P.split_tokens, seqlen);
     const int nsplit_b = (seqlen + P.split_tokens - 1) / P.split_tokens;
     const int nblk = (t_end - t_begin + kDecodeBlock - 1) / kDecodeBlock;
@@ -311,7 +367,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_ke
         const int tok0 = t_begin + (warp + jj * kDecodeWarps) * kDecodeBlock;
         unsigned char *st = wring + s * C::STAGE;
         if (lane == 0)
-            mbar_arrive_expect_tx(&bars[s], C::STAGE);
+            mbar_arrive_expect_tx_relaxed(&bars[s], C::STAGE);
         __syncwarp();
         if (lane < 4) {
             const void *src;
@@ -339,6 +395,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_ke
     };
     for (int jj = 0; jj < kDecodeStages && jj < my_nblk; ++jj)
         issue(jj, jj);
+    // everything below reads what the q prologue writes
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // q~ operand fragments and per-head constants
     uint32_t qB[C::NT][C::KSTEPS][2];
@@ -609,14 +667,20 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_ke
     }
     if (nsplit_b == 1)
         return;
-    __threadfence();
+    // ---- the last split of the pair to finish merges all splits. The barrier orders
+    //      every thread's partial stores before thread 0's device-scope fence and ticket;
+    //      the merging CTA's thread 0 fences after its ticket and the barrier orders that
+    //      before every thread's loads.
     __syncthreads();
-    if (threadIdx.x == 0)
-        *flag_smem = (atomicAdd(&P.ticket[pair], 1) == nsplit_b - 1);
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int last = (atomicAdd(&P.ticket[pair], 1) == nsplit_b - 1);
+        __threadfence();
+        *flag_smem = last;
+    }
     __syncthreads();
     if (!*flag_smem)
         return;
-    __threadfence();
     const float *pall = P.part + pair * P.nsplit * (size_t)(G * (D + 2));
     for (int idx = threadIdx.x; idx < G * D; idx += kDecodeWarps * 32) {
         const int head = idx / D, dim = idx % D;
@@ -639,32 +703,59 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks) decode_ke
     }
 }
 
+// cudaFuncSetAttribute applies to the current device: remember it per device.
+template <typename F>
+cudaError_t ensure_dynamic_smem(F *func, int bytes, unsigned long long &done_mask)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done_mask & bit)
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        done_mask |= bit;
+    return e;
+}
+
 template <int D, int G, int BK, int BV>
 cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
 {
     using C = Cfg<D, G, BK, BV>;
+    using QS = QprepSmem<D, G>;
+    static unsigned long long qprep_attr = 0, decode_attr = 0;
+    cudaError_t e = ensure_dynamic_smem(qprep_kernel<D, G, BK>, QS::BYTES, qprep_attr);
+    if (e != cudaSuccess)
+        return e;
+    e = ensure_dynamic_smem(decode_kernel<D, G, BK, BV>, C::SMEM, decode_attr);
+    if (e != cudaSuccess)
+        return e;
     // q prologue
     {
         dim3 grid(L.p.Hkv, (L.p.B + kQprepSeqs - 1) / kQprepSeqs);
-        qprep_kernel<D, G, BK><<<grid, D, 0, st>>>(L.q, L.q_bf16, L.M, L.p.B, L.p.Hq, L.p.Hkv,
-                                                  kQprepSeqs, const_cast<uint32_t *>(L.p.qfrag),
-                                                  const_cast<float *>(L.p.qscale),
-                                                  const_cast<float *>(L.p.qw), L.p.ticket);
-        cudaError_t e = cudaGetLastError();
+        qprep_kernel<D, G, BK><<<grid, kQprepThreads, QS::BYTES, st>>>(
+            L.q, L.q_bf16, L.M, L.p.B, L.p.Hq, L.p.Hkv, kQprepSeqs, L.p.seqlens, L.p.max_seqlen,
+            L.p.out, L.p.out_bf16, const_cast<uint32_t *>(L.p.qfrag),
+            const_cast<float *>(L.p.qscale), const_cast<float *>(L.p.qw), L.p.ticket);
+        e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
     }
-    static int decode_attr = 0;
-    if (!decode_attr) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, BK, BV>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess)
-            return e;
-        decode_attr = 1;
-    }
-    dim3 grid(L.p.nsplit, L.p.Hkv, L.p.B);
-    decode_kernel<D, G, BK, BV><<<grid, kDecodeWarps * 32, C::SMEM, st>>>(L.p);
-    return cudaGetLastError();
+    // decode: CTA (KV head, sequence, split), splits slowest so that the short last
+    // splits of the sequences run last; a programmatic dependent of the prologue
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(L.p.Hkv, L.p.B, L.p.nsplit);
+    cfg.blockDim = dim3(kDecodeWarps * 32);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<D, G, BK, BV>, L.p);
 }
 
 }  // namespace

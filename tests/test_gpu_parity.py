@@ -310,6 +310,22 @@ def test_decode_split_invariance(splits, monkeypatch):
     assert_close(out.cpu().numpy(), want, where=f"splits={splits}")
 
 
+@pytest.mark.parametrize("splits", ["1", "3", "100"])
+def test_decode_many_short_sequences(splits, monkeypatch):
+    # short, empty and capacity-length sequences side by side, each split count
+    cfg = small(synth.CONFIGS[1], T_cap=256)
+    seql = [5, 0, 64, 200, 0, 0, 1, 130, 256, 65]
+    oc, M = oracle_built_cache(cfg, len(seql), 256)
+    gc = upload_cache(oc, cfg)
+    q = synth.as_dtype(synth.queries(cfg.with_(B=len(seql))), cfg.q_dtype)
+    want = oracle.decode(q, M, oc, np.array(seql, np.int32))
+    monkeypatch.setenv("KVQ_DECODE_SPLITS", splits)
+    out, err = gpu_decode(cfg, q, M, gc, seql, max_seqlen=256)
+    assert err == 0
+    assert not out[1].any() and not out[4].any() and not out[5].any()
+    assert_close(out.cpu().numpy(), want, where=f"splits={splits}")
+
+
 def test_decode_edge_lengths():
     cfg = small(synth.CONFIGS[1], T_cap=320)
     seql = [0, 1, 63, 64, 65, 128, 319, 320]
