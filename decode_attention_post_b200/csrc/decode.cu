@@ -59,17 +59,17 @@ struct Cfg {
     static constexpr int SZ_BYTES = kDecodeBlock * 4;
     static constexpr int VC_BYTES = kDecodeBlock * D * BV / 8;
     static constexpr int STAGE = KC_BYTES + SZ_BYTES + VC_BYTES + SZ_BYTES;
-    static constexpr int PSTRIDE = kDecodeBlock + 8; // halves per P'^T column (padded)
-    static constexpr int PBUF = COLS * PSTRIDE * 2;  // bytes per warp
     static constexpr int QFRAG = NT * KSTEPS * 32 * 2;
     static constexpr int RING = kDecodeWarps * kDecodeStages * STAGE;
     static constexpr int MERGE = kDecodeWarps * G * (D + 2) * 4;
-    static constexpr int SMEM = (RING > MERGE ? RING : MERGE) + kDecodeWarps * PBUF +
-                                kDecodeWarps * kDecodeStages * 8 + 16;
+    static constexpr int SMEM = (RING > MERGE ? RING : MERGE) + kDecodeWarps * kDecodeStages * 8 + 16;
     // resident CTAs per SM the register budget targets: kDecodeMinBlocks, or fewer when
     // shared memory (227 KB per SM, 1 KB reserved per CTA) holds fewer
     static constexpr int SMEM_FIT = (227 * 1024) / (SMEM + 1024);
-    static constexpr int MINB = SMEM_FIT < kDecodeMinBlocks ? SMEM_FIT : kDecodeMinBlocks;
+    // d = 128 with G = 8 keeps 64 output accumulators and 32 query-fragment registers per
+    // thread: it needs the register budget of 3 CTAs per SM
+    static constexpr int REG_FIT = (D == 128 && G == 8) ? 3 : kDecodeMinBlocks;
+    static constexpr int MINB = SMEM_FIT < REG_FIT ? SMEM_FIT : REG_FIT;
     static_assert(MINB >= 1, "decode CTA does not fit in shared memory");
     static_assert(STAGE % 16 == 0, "stage alignment");
     static_assert(MERGE % 16 == 0, "merge area alignment");
@@ -320,14 +320,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     using C = Cfg<D, G, BK, BV>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *ring = smem_raw;
-    __half *pbuf_all = reinterpret_cast<__half *>(smem_raw + (C::RING > C::MERGE ? C::RING : C::MERGE));
-    uint64_t *bars_all = reinterpret_cast<uint64_t *>(reinterpret_cast<unsigned char *>(pbuf_all) +
-                                                      kDecodeWarps * C::PBUF);
+    uint64_t *bars_all =
+        reinterpret_cast<uint64_t *>(smem_raw + (C::RING > C::MERGE ? C::RING : C::MERGE));
     int *flag_smem = reinterpret_cast<int *>(bars_all + kDecodeWarps * kDecodeStages);
 
     const int h = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
+    // Tokens of a 16-token sub-tile held in accumulator rows g and g+8: row 2i holds token
+    // i and row 2i+1 token i+8 (i < 4), row 8+2i token i+4 and row 9+2i token i+12. After
+    // the 8x8 transposes the value product then sees key slot 2t = token t, 2t+1 = t+8,
+    // 2t+8 = t+4, 2t+9 = t+12 -- the token order of the value-code tiles.
+    const int ta = (g >> 1) + 8 * (g & 1), tb = ta + 4;
     const size_t pair = (size_t)b * P.Hkv + h;
 
     int seqlen = P.seqlens[b];
@@ -345,7 +349,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     const int my_nblk = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
 
     unsigned char *wring = ring + warp * kDecodeStages * C::STAGE;
-    __half *pbuf = pbuf_all + warp * (C::PBUF / 2);
     uint64_t *bars = bars_all + warp * kDecodeStages;
 
     const uint8_t *kc = P.k_codes + pair * (size_t)P.T_cap * C::ROWK;
@@ -441,14 +444,15 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
         const uint32_t *vszw =
             reinterpret_cast<const uint32_t *>(st + C::KC_BYTES + C::SZ_BYTES + C::VC_BYTES);
 
-        // ---- scores S^T for 4 sub-tiles: independent chains interleaved per k-step
+        // ---- scores S^T for 4 sub-tiles: independent chains interleaved per k-step.
+        //      Accumulator rows g and g+8 hold tokens ta and tb of the sub-tile (see below).
         float S[4][C::NT][4];
         uint32_t kw[4][2][C::WPT];
 #pragma unroll
         for (int stt = 0; stt < 4; ++stt) {
             const unsigned char *kt = st + stt * 16 * C::ROWK + t * 4 * C::WPT;
-            lds_words<C::WPT>(kw[stt][0], kt + g * C::ROWK);
-            lds_words<C::WPT>(kw[stt][1], kt + (g + 8) * C::ROWK);
+            lds_words<C::WPT>(kw[stt][0], kt + ta * C::ROWK);
+            lds_words<C::WPT>(kw[stt][1], kt + tb * C::ROWK);
 #pragma unroll
             for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
         for (int stt = 0; stt < 4; ++stt)
 #pragma unroll
             for (int tk = 0; tk < 2; ++tk) {
-                const int tl = 16 * stt + g + 8 * tk;
+                const int tl = 16 * stt + (tk ? tb : ta);
                 const float2 sz = half2_bits_to_float2(kszw[tl]);
                 const float a = sz.x * cs;
                 const bool valid = FULL || (tok0 + tl < t_end);
@@ -511,16 +515,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
             }
         }
 
-        // ---- P' = p * s^v as float16 hi/lo, written transposed: column 8nt + 2t (hi) and
-        //      8nt + 2t + 1 (lo), slots (2g, 2g+1) = tokens (g, g+8) of the sub-tile
+        // ---- P' = p * s^v as float16 (hi, lo) pairs in the accumulator layout (row = token,
+        //      columns 2t, 2t+1 = hi, lo of head 4nt+t); one 8x8 transpose per row half turns
+        //      them into the B operand of the value product
+        uint32_t pb[4][C::NT][2];
 #pragma unroll
         for (int stt = 0; stt < 4; ++stt) {
-            const float2 vz0 = half2_bits_to_float2(vszw[16 * stt + g]);
-            const float2 vz1 = half2_bits_to_float2(vszw[16 * stt + g + 8]);
+            const float2 vz0 = half2_bits_to_float2(vszw[16 * stt + ta]);
+            const float2 vz1 = half2_bits_to_float2(vszw[16 * stt + tb]);
             bool v0 = true, v1 = true;
             if constexpr (!FULL) {
-                v0 = tok0 + 16 * stt + g < t_end;
-                v1 = tok0 + 16 * stt + g + 8 < t_end;
+                v0 = tok0 + 16 * stt + ta < t_end;
+                v1 = tok0 + 16 * stt + tb < t_end;
             }
 #pragma unroll
             for (int nt = 0; nt < C::NT; ++nt) {
@@ -539,25 +545,17 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
                 const __half2 hi = __floats2half2_rn(pp0, pp1);
                 const float2 hif = __half22float2(hi);
                 const __half2 lo = __floats2half2_rn(pp0 - hif.x, pp1 - hif.y);
-                __half *col = pbuf + (8 * nt + 2 * t) * C::PSTRIDE + 16 * stt + 2 * g;
-                *reinterpret_cast<__half2 *>(col) = hi;
-                *reinterpret_cast<__half2 *>(col + C::PSTRIDE) = lo;
+                const __half2 ra = __lows2half2(hi, lo), rb = __highs2half2(hi, lo);
+                pb[stt][nt][0] = movmatrix_trans(*reinterpret_cast<const uint32_t *>(&ra));
+                pb[stt][nt][1] = movmatrix_trans(*reinterpret_cast<const uint32_t *>(&rb));
             }
         }
-        __syncwarp();
 
         // ---- O^T += Vcodes^T . P'^T
 #pragma unroll
         for (int stt = 0; stt < 4; ++stt) {
             uint32_t vw[2 * C::WV];
             lds_words<2 * C::WV>(vw, st + C::KC_BYTES + C::SZ_BYTES + stt * C::VTILE + lane * C::VCH);
-            uint32_t pb[C::NT][2];
-#pragma unroll
-            for (int nt = 0; nt < C::NT; ++nt) {
-                const __half *pc = pbuf + (8 * nt + g) * C::PSTRIDE + 16 * stt + 2 * t;
-                pb[nt][0] = *reinterpret_cast<const uint32_t *>(pc);
-                pb[nt][1] = *reinterpret_cast<const uint32_t *>(pc + 8);
-            }
 #pragma unroll
             for (int m = 0; m < C::MT; ++m) {
                 const uint32_t a0 = ext_v<BV, C::CPBV, C::EV, C::WV>(vw, 0, 2 * m);
@@ -566,7 +564,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
                 const uint32_t a3 = ext_v<BV, C::CPBV, C::EV, C::WV>(vw, 1, 2 * m + 1);
 #pragma unroll
                 for (int nt = 0; nt < C::NT; ++nt)
-                    mma_f16(O[m][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                    mma_f16(O[m][nt], a0, a1, a2, a3, pb[stt][nt][0], pb[stt][nt][1]);
             }
         }
         __syncwarp();

@@ -139,6 +139,15 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void *
                  : "r"(smem_addr(p)));
 }
 
+// Transpose of an 8x8 matrix of 16-bit elements held one .b32 (row lane/4, columns
+// 2(lane%4), 2(lane%4)+1) per lane, returned in the same layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a)
+{
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+
 // 16-byte asynchronous copy global -> shared (L2 only); src_bytes < 16 zero-fills the rest.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes)
 {
