@@ -15,7 +15,9 @@
 //   c = clamp(rint(f32(x - z)/s)) computed as (x - z) * rcp_rn(s), which differs from the
 //   IEEE quotient by under 2 ulp; a value within 2^-20 of a rounding tie is recomputed
 //   with IEEE division, so the codes are those of the definition bit for bit.
-//   Codes go through shared memory and are stored as whole K-row words / V-tile halves.
+//   Codes are packed in registers: a K-row word from the quad's 4 lanes (two xor
+//   shuffles), a V-tile half from one lane (it holds every column of that half), and
+//   stored whole.
 #include "kvq_common.cuh"
 #include "kvq_ptx.cuh"
 
@@ -28,11 +30,9 @@ constexpr int kMmaWarps = 4;
 template <int D>
 struct MmaSmem {
     static constexpr int TS = D + 8;       // bf16 per staged row
-    static constexpr int CS = D + 16;      // code bytes per staged token row
     __nv_bfloat16 Thi[D * TS];
     __nv_bfloat16 Tlo[D * TS];
     __nv_bfloat16 X[kMmaWarps][2][16 * TS];      // double-buffered input rows
-    uint8_t codes[kMmaWarps][16 * CS];
 };
 
 __device__ __forceinline__ void quad_minmax(float &mn, float &mx)
@@ -87,6 +87,50 @@ __device__ __forceinline__ float quad_order_stat(const float (&vals)[NV], int ka
     return m;
 }
 
+// K row: little-endian bit stream, column j at bit BITS*j. A 32-bit word holds 32/BITS
+// columns, i.e. 2 (2-bit) or 1 (4-bit) n-tiles of 8 columns; lane t of the quad holds
+// columns 8nt + 2t + {0, 1} of every n-tile, so the quad's 4 lanes together hold a word:
+// partial words are OR-ed over the quad and lane t stores words t, t+4, ...
+template <int D, int BITS, int NV>
+__device__ __forceinline__ void store_k_row(const uint32_t (&cq)[NV], uint32_t *dst, int t, bool ok)
+{
+    constexpr int WORDS = D * BITS / 32, TPW = 4 / BITS;
+#pragma unroll
+    for (int w = 0; w < WORDS; ++w) {
+        uint32_t part = 0;
+#pragma unroll
+        for (int q = 0; q < TPW; ++q) {
+            const int nt = w * TPW + q;
+            part |= cq[2 * nt] << (BITS * (8 * q + 2 * t));
+            part |= cq[2 * nt + 1] << (BITS * (8 * q + 2 * t + 1));
+        }
+        part |= __shfl_xor_sync(0xffffffffu, part, 1);
+        part |= __shfl_xor_sync(0xffffffffu, part, 2);
+        if (ok && (w & 3) == t)
+            dst[w] = part;
+    }
+}
+
+// V tile halves of one token: half (gq, rr) holds dims 8(E rr + s) + gq at bits BITS*s,
+// E = 16/BITS. Lane t holds gq = 2t and 2t+1 of every n-tile, so both are local.
+template <int D, int BITS, int NV>
+__device__ __forceinline__ void store_v_halves(const uint32_t (&cq)[NV], unsigned char *tile_base,
+                                               int tok, int t)
+{
+    constexpr int E = 16 / BITS, W = D * BITS / 128;
+#pragma unroll
+    for (int odd = 0; odd < 2; ++odd)
+#pragma unroll
+        for (int rr = 0; rr < W; ++rr) {
+            uint32_t val = 0;
+#pragma unroll
+            for (int s2 = 0; s2 < E; ++s2)
+                val |= cq[2 * (E * rr + s2) + odd] << (BITS * s2);
+            *reinterpret_cast<uint16_t *>(tile_base + v_half_offset(D, BITS, tok, 2 * t + odd, rr)) =
+                (uint16_t)val;
+        }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kMmaWarps * 32)
 append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *__restrict__ v_in,
@@ -97,7 +141,7 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                   const int32_t *__restrict__ pos, int32_t *dev_err)
 {
     using Sm = MmaSmem<D>;
-    constexpr int TS = Sm::TS, CS = Sm::CS, NT = D / 8, NV = 2 * NT;
+    constexpr int TS = Sm::TS, NT = D / 8, NV = 2 * NT;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     Sm &sm = *reinterpret_cast<Sm *>(smem_raw);
 
@@ -132,7 +176,6 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
     }
     __syncthreads();
 
-    uint8_t *codes = sm.codes[warp];
     constexpr int CH = D / 8;                         // 16-byte chunks per input row
     // cp.async the 16 input rows of `tile` into buffer `buf` (rows past the end zero-fill)
     auto fetch = [&](long tile, int buf) {
@@ -193,15 +236,29 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
             }
         }
 
-        // ---- per token (rows g and g+8): clip range, scale/zero, codes
+        // ---- sequence and position of the tile's first token (one division per tile)
+        int b0, i0;
+        if (total <= 0x7fffffffL) {
+            const unsigned uu = (unsigned)u0, nn = (unsigned)n;
+            b0 = (int)(uu / nn);
+            i0 = (int)(uu - (unsigned)b0 * nn);
+        } else {
+            b0 = (int)(u0 / n);
+            i0 = (int)(u0 - (long)b0 * n);
+        }
+
+        // ---- per token (rows g and g+8): clip range, scale/zero, codes, packed stores
 #pragma unroll
         for (int tk = 0; tk < 2; ++tk) {
-            const long u = u0 + g + 8 * tk;
+            const int r = g + 8 * tk;
+            const long u = u0 + r;
             bool ok = u < total;
-            int b = 0, i = 0, p0 = 0;
+            int b = b0, i = i0 + r, p0 = 0;
+            while (i >= n) {                          // the tile may run into later sequences
+                i -= n;
+                ++b;
+            }
             if (ok) {
-                b = (int)(u / n);
-                i = (int)(u % n);
                 p0 = pos[b];
                 if (p0 < 0 || (long)p0 + n > T_cap) {
                     if (i == 0 && t == 0)
@@ -216,6 +273,7 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                 x[2 * nt] = acc[nt][2 * tk];
                 x[2 * nt + 1] = acc[nt][2 * tk + 1];
             }
+            uint32_t cq[NV];                          // codes of this lane's columns
             for (int gr = 0; gr < ng; ++gr) {
                 const int c0 = gr * group, c1 = c0 + group;    // columns of this group
                 float lo, hi;
@@ -279,7 +337,7 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                 if (ok && !finite && t == 0)
                     flag(dev_err, KVQ_DEVERR_NONFINITE);
                 const bool zero = !finite || sf == 0.f;
-                const float r = zero ? 0.f : __frcp_rn(sf);
+                const float rc = zero ? 0.f : __frcp_rn(sf);
 #pragma unroll
                 for (int e = 0; e < NV; ++e) {
                     const int col = 8 * (e >> 1) + 2 * t + (e & 1);
@@ -288,7 +346,7 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                     int c = 0;
                     if (!zero) {
                         const float dlt = __fsub_rn(x[e], zf);
-                        float y = __fmul_rn(dlt, r);
+                        float y = __fmul_rn(dlt, rc);
                         float k = rintf(y);
                         // within 2^-20 relative of a tie: take the IEEE quotient
                         if (fabsf(y - k) >= 0.5f - 9.5367431640625e-07f * fmaxf(fabsf(y), 1.f)) {
@@ -297,7 +355,7 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                         }
                         c = (int)fminf(fmaxf(k, 0.f), (float)qmax);
                     }
-                    codes[(g + 8 * tk) * CS + col] = (uint8_t)c;
+                    cq[e] = (uint32_t)c;
                 }
                 if (ok && t == 0) {
                     const size_t row = ((size_t)b * Hkv + h) * T_cap + p0 + i;
@@ -306,49 +364,24 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                     (which ? v_sz : k_sz)[row * ng + gr] = pair;
                 }
             }
-        }
-        __syncwarp();
 
-        // ---- whole-word (K rows) / whole-half (V tiles) stores
-        if (!which) {
-            constexpr int WORDS = D * 2 / 32;              // per row at 2 bits; 4-bit doubles
-            const int words = D * bits / 32, cpw = 32 / bits;
-            for (int task = lane; task < 16 * words; task += 32) {
-                const int r = task / words, w = task % words;
-                const long u = u0 + r;
-                if (u >= total)
-                    continue;
-                const int b = (int)(u / n), i = (int)(u % n), p0 = pos[b];
-                if (p0 < 0 || (long)p0 + n > T_cap)
-                    continue;
-                uint32_t word = 0;
-                for (int e = 0; e < cpw; ++e)
-                    word |= (uint32_t)codes[r * CS + w * cpw + e] << (bits * e);
-                const size_t row = ((size_t)b * Hkv + h) * T_cap + p0 + i;
-                reinterpret_cast<uint32_t *>(k_codes + row * (D * bits / 8))[w] = word;
-            }
-            (void)WORDS;
-        } else {
-            const int E = 16 / bits, halves = D / E;
-            for (int task = lane; task < 16 * halves; task += 32) {
-                const int r = task / halves, hv = task % halves;
-                const long u = u0 + r;
-                if (u >= total)
-                    continue;
-                const int b = (int)(u / n), i = (int)(u % n), p0 = pos[b];
-                if (p0 < 0 || (long)p0 + n > T_cap)
-                    continue;
-                const int gq = hv & 7, rr = hv >> 3;
-                uint32_t val = 0;
-                for (int s2 = 0; s2 < E; ++s2)
-                    val |= (uint32_t)codes[r * CS + 8 * (E * rr + s2) + gq] << (bits * s2);
+            // ---- packed stores, built in registers
+            const size_t row = ((size_t)b * Hkv + h) * T_cap + p0 + i;
+            if (!which) {
+                uint32_t *dst = reinterpret_cast<uint32_t *>(k_codes + row * (D * bits / 8));
+                if (bits == 2)
+                    store_k_row<D, 2>(cq, dst, t, ok);
+                else
+                    store_k_row<D, 4>(cq, dst, t, ok);
+            } else if (ok) {
                 const int tpos = p0 + i;
-                const size_t tile_base =
-                    (((size_t)b * Hkv + h) * (T_cap / kTileTokens) + tpos / kTileTokens) *
-                    (kTileTokens * D * bits / 8);
-                *reinterpret_cast<uint16_t *>(v_codes + tile_base +
-                                              v_half_offset(D, bits, tpos % kTileTokens, gq, rr)) =
-                    (uint16_t)val;
+                unsigned char *tile_base =
+                    v_codes + (((size_t)b * Hkv + h) * (T_cap / kTileTokens) + tpos / kTileTokens) *
+                                  (kTileTokens * D * bits / 8);
+                if (bits == 2)
+                    store_v_halves<D, 2>(cq, tile_base, tpos % kTileTokens, t);
+                else
+                    store_v_halves<D, 4>(cq, tile_base, tpos % kTileTokens, t);
             }
         }
         __syncwarp();
