@@ -34,6 +34,10 @@ from tests import synth  # noqa: E402  (seeded input generators only)
 
 METRIC = "2-bit KV decode attention: achieved HBM GB/s and % of B200 peak; append tok/s"
 CONFIG_IDX = 2
+# dram__bytes_read.sum + dram__bytes_write.sum of one decode_kernel launch on this workload
+# (ncu --set full --clock-control none, profiles directory); None once the kernel changes.
+DECODE_TRAFFIC_BYTES = 549_279_744
+DECODE_TRAFFIC_KERNEL = "decode_kernel<128,4,2,2>"
 APPEND_CONFIG_IDX = 4
 
 
@@ -346,7 +350,7 @@ def run_gpu(args):
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_nominal_8000": round(achieved / 8000.0, 4),
                      "bytes_per_launch": dec_bytes, "ms_per_launch": round(dec_ms, 5),
-                     "traffic": None},
+                     "traffic": DECODE_TRAFFIC_BYTES, "traffic_kernel": DECODE_TRAFFIC_KERNEL},
         "append_decode_time": {"append_ms": round(app_ms, 5), "decode_ms": round(dec_ms, 5),
                                "append_tok_per_s": round(cfg.B / (app_ms * 1e-3), 1)},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
