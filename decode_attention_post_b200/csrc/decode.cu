@@ -6,26 +6,29 @@
 //
 // Two kernels per call:
 //  qprep   q~ = T_k^{-T} q for every query head (float32), and from it the tensor-core
-//          operand fragments, the logit scale and sum(q~) per head.
+//          operand fragments (q~ as 16-bit fixed point, two int8 pieces), the logit
+//          scale and sum(q~) per head.
 //  decode  split-K flash decode. CTA = (KV head, sequence, split), 4 warps; launched as a
 //          programmatic dependent of qprep, it requests its first cache blocks before
 //          waiting for qprep. Each warp streams 64-token blocks (K codes, K scale/zero,
 //          V codes, V scale/zero) with cp.async.bulk into a private 2-stage shared-memory
 //          ring (mbarrier completion, bounded waits), and per block:
-//            S^T[16 tok x (hi,lo)*G] = Kcodes[16 tok x d] . q~'[d x 2G]   (mma f16, f32 acc)
+//            S^T[16 tok x (hi,lo)*G] = Kcodes[16 tok x d] . q_int[d x 2G]  (mma int8,
+//                    int32 accumulate: exact)
 //            logit = log2(e)/sqrt(d) * (s_t * q~.c_t + z_t * sum q~)       (affine dequant
 //                    folded per token: x^ = z + c s)
 //            online softmax in float32 (lazy rescale), P' = p * s^v_t split f16 hi/lo
-//            O^T[d x (hi,lo)*G] += Vcodes^T[d x 16 tok] . P'^T[16 tok x 2G]
+//            O^T[d x (hi,lo)*G] += Vcodes^T[d x 16 tok] . P'^T[16 tok x 2G]  (mma f16)
 //          and sum_t p_t z^v_t for the value zero-points.
 //          Warps merge in shared memory; splits merge in the last CTA to finish a
 //          (sequence, KV head) (atomic ticket, no spin-wait).
 //
-// Codes reach the tensor cores without a float conversion: a 2-bit (4-bit) code field
-// masked in place inside a 32-bit word is the float16 subnormal c * 2^(bits*k) * 2^-24,
-// where k is its field position inside the byte. The per-position factor 2^(bits*k) is
-// compensated in the q~ operand (keys) or per output dim (values), so every product
-// carries the same power-of-two scale. Tensor cores take float16 subnormals exactly.
+// Codes reach the tensor cores without unpacking. Keys: masking field position k of
+// every byte of a 32-bit word leaves four uint8 operands c * 2^(bits*k); one int8 MMA per
+// field position, with the int32 accumulator multiplied by 2^bits between positions,
+// sums every code with the same weight. Values: a 2-bit (4-bit) field masked in place is
+// the float16 subnormal c * 2^(bits*k) * 2^-24; the per-position factor is compensated
+// per output dim. Tensor cores take float16 subnormals exactly.
 #include "kvq_common.cuh"
 #include "kvq_ptx.cuh"
 #include "decode_shapes.h"
@@ -43,7 +46,8 @@ constexpr int kQprepSeqs = 2;     // sequences per q-prologue CTA
 
 template <int D, int G, int BK, int BV>
 struct Cfg {
-    static constexpr int KSTEPS = D / 16;            // k-steps of the Q.K contraction
+    static constexpr int KCH = D * BK / 256 > 0 ? D * BK / 256 : 1;  // int8 k-chunks per field
+    static constexpr int KS = (8 / BK) * KCH;        // int8 k-steps of the Q.K contraction
     static constexpr int MT = D / 16;                // m-tiles (output dims) of P.V
     static constexpr int NT = (2 * G) / 8;           // n-tiles of (hi, lo) x G columns
     static constexpr int COLS = 2 * G;
@@ -59,7 +63,7 @@ struct Cfg {
     static constexpr int SZ_BYTES = kDecodeBlock * 4;
     static constexpr int VC_BYTES = kDecodeBlock * D * BV / 8;
     static constexpr int STAGE = KC_BYTES + SZ_BYTES + VC_BYTES + SZ_BYTES;
-    static constexpr int QFRAG = NT * KSTEPS * 32 * 2;
+    static constexpr int QFRAG = NT * KS * 32 * 2;
     static constexpr int RING = kDecodeWarps * kDecodeStages * STAGE;
     static constexpr int MERGE = kDecodeWarps * G * (D + 2) * 4;
     static constexpr int SMEM = (RING > MERGE ? RING : MERGE) + kDecodeWarps * kDecodeStages * 8 + 16;
@@ -77,19 +81,6 @@ struct Cfg {
 };
 
 // ---------------------------------------------------------------- operand extraction
-
-// Key operand: extraction e (0 .. d/8-1) of this thread's WPT words of one token.
-// Word e / (2 CPB), byte-half beta = (e / CPB) % 2, field k = e % CPB. The float16
-// pair holds dims (4w+beta)*CPB + k (low) and (4w+2+beta)*CPB + k (high), w the
-// token-row word index, each scaled by 2^(BK*k) * 2^-24.
-template <int BK, int CPB>
-__device__ __forceinline__ uint32_t ext_k(const uint32_t *kw, int e)
-{
-    constexpr uint32_t M = ((1u << BK) - 1u) * 0x00010001u;
-    const int wl = e / (2 * CPB), beta = (e / CPB) & 1, k = e % CPB;
-    const uint32_t w = beta ? (kw[wl] >> 8) : kw[wl];
-    return w & (M << (BK * k));
-}
 
 // Value operand: the float16 pair (token t+4p, token t+4p+8) of output dim 8n + g.
 template <int BV, int CPB, int EV, int WV>
@@ -135,11 +126,12 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t u)
 // row i by 8 consecutive threads fall in distinct banks), the q vectors as qs[j][v].
 // Thread (i, part) accumulates output dim i of every vector over one of JP slices of j;
 // the slices are summed in shared memory. From q~ = M q (float32) it derives
-//   eq  = power-of-two exponent bringing max|q~| * 2^(BK*(CPB-1)) to about 2^14,
-//   frag[nt][ks][lane][2] = float16 hi/lo pieces of q~ * 2^eq * 2^(BK*(CPB-1-k)) laid
-//                           out as the B operand of the Q.K product; n-tile nt holds
-//                           heads 4nt..4nt+3, column 2h' = hi and 2h'+1 = lo of head 4nt+h',
-//   cs  = log2(e) / sqrt(d) / F with F = 2^(eq + BK*(CPB-1) - 24) the product scale,
+//   eq  = per head, the power-of-two exponent that brings max|q~| to 2^14..32512,
+//   q_int = rint(q~ 2^eq) = 256 hi + lo (int8 hi, lo),
+//   frag[nt][ks][lane][2] = int8 hi/lo pieces of q_int laid out as the B operand of the
+//                           int8 Q.K product (k-step = field position x k-chunk); n-tile
+//                           nt holds heads 4nt..4nt+3, column 2h' = hi and 2h'+1 = lo,
+//   cs  = log2(e) / sqrt(d) / (2^(BK*(CPB-1)) 2^eq), per head,
 //   w_h = log2(e) / sqrt(d) * sum_j q~_hj,
 // zeroes the split-merge ticket of each (sequence, KV head), and writes the zero output
 // of every empty sequence. It lets the dependent decode launch start at once: the decode
@@ -151,7 +143,7 @@ struct QprepSmem {
     static constexpr int NVMAX = kQprepSeqs * G;
     static constexpr int JP = kQprepThreads / D;     // slices of the j range
     static constexpr int MSTRIDE = D + 4;
-    static constexpr int BYTES = (D * MSTRIDE + D * NVMAX + JP * NVMAX * D + kQprepSeqs) * 4;
+    static constexpr int BYTES = (D * MSTRIDE + D * NVMAX + JP * NVMAX * D + NVMAX) * 4;
 };
 
 template <int D, int G, int BK>
@@ -161,14 +153,15 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
              int out_bf16, uint32_t *__restrict__ qfrag, float *__restrict__ qscale,
              float *__restrict__ qw, int *__restrict__ ticket)
 {
-    constexpr int CPB = 8 / BK, KSTEPS = D / 16, NT = (2 * G) / 8, WPT = D * BK / 128;
+    constexpr int CPB = 8 / BK, NT = (2 * G) / 8, WPT = D * BK / 128;
+    constexpr int KCH = WPT >= 2 ? WPT / 2 : 1, KS = CPB * KCH;
     using S = QprepSmem<D, G>;
     constexpr int NVMAX = S::NVMAX, JP = S::JP, JL = D / JP;
     extern __shared__ __align__(16) float qsm[];
     float *Ms = qsm;                              // [D][D+4]
     float *qs = Ms + D * S::MSTRIDE;              // [D][NVMAX]
     float *pt = qs + D * NVMAX;                   // [JP][NVMAX][D]; slice 0 ends up as q~
-    float *red = pt + JP * NVMAX * D;             // [kQprepSeqs]
+    int *eqv = reinterpret_cast<int *>(pt + JP * NVMAX * D);   // [NVMAX] per-head exponent
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
@@ -186,8 +179,6 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
         }
         cp_async_commit();
     }
-    if (tid < kQprepSeqs)
-        red[tid] = 0.f;
     for (int idx = tid; idx < NVMAX * D; idx += kQprepThreads) {
         const int v = idx / D, j = idx % D;
         const int bi = v / G, gg = v % G;
@@ -260,41 +251,42 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
         }
         if (lane == 0) {
             const int bi = v / G, gg = v % G;
-            qw[(size_t)(b0 + bi) * Hq + h * G + gg] = kLog2e * sm * s;
-            atomicMax(reinterpret_cast<int *>(&red[bi]), __float_as_int(a));   // a >= 0
+            const size_t hq = (size_t)(b0 + bi) * Hq + h * G + gg;
+            qw[hq] = kLog2e * sm * s;
+            // q_int = rint(q~ 2^eq) with max |q_int| <= 127 * 256, so that q_int = 256 hi + lo
+            // with int8 hi and lo: 2^15 when the mantissa of max|q~| allows it, else 2^14
+            int ex = 0;
+            const float m = a > 0.f ? frexpf(a, &ex) : 0.f;   // a = m 2^ex, m in [0.5, 1)
+            const int eq = a > 0.f ? (m <= 0.9921875f ? 15 - ex : 14 - ex) : 0;
+            eqv[v] = eq;
+            // S = 2^(BK*(CPB-1)) * sum_j c_j q_int_j; cs = log2e * sm / (2^(BK*(CPB-1)) 2^eq)
+            qscale[hq] = kLog2e * sm * ldexpf(1.f, -eq - BK * (CPB - 1));
         }
     }
     __syncthreads();
     for (int bi = 0; bi < nb; ++bi) {
         const size_t pair = (size_t)(b0 + bi) * Hkv + h;
-        const float amax = red[bi];
-        int ex = 0;
-        if (amax > 0.f)
-            frexpf(amax, &ex);                         // amax <= 2^ex
-        const int eq = amax > 0.f ? 14 - BK * (CPB - 1) - ex : 0;
-        if (tid == 0) {
-            // F = 2^(eq + BK*(CPB-1) - 24); cs = log2e * sm / F
-            qscale[pair] = kLog2e * sm * ldexpf(1.f, 24 - eq - BK * (CPB - 1));
+        if (tid == 0)
             ticket[pair] = 0;
-        }
-        uint32_t *fr = qfrag + pair * (size_t)(NT * KSTEPS * 64);
-        for (int idx = tid; idx < NT * KSTEPS * 64; idx += kQprepThreads) {
-            const int rho = idx & 1, ln = (idx >> 1) & 31, ks = (idx >> 6) % KSTEPS;
-            const int nt = (idx >> 6) / KSTEPS;
+        uint32_t *fr = qfrag + pair * (size_t)(NT * KS * 64);
+        for (int idx = tid; idx < NT * KS * 64; idx += kQprepThreads) {
+            const int rho = idx & 1, ln = (idx >> 1) & 31, ks = (idx >> 6) % KS;
+            const int nt = (idx >> 6) / KS;
+            const int k = ks / KCH, c = ks % KCH;               // field position, k-chunk
             const int g = ln >> 2, t = ln & 3;
             const int head = 4 * nt + g / 2, piece = g & 1;     // columns (hi, lo) per head
-            const int e = 2 * ks + rho;
-            const int w = WPT * t + e / (2 * CPB), beta = (e / CPB) & 1, k = e % CPB;
-            const int dlo = (4 * w + beta) * CPB + k, dhi = (4 * w + 2 + beta) * CPB + k;
-            const float scale = ldexpf(1.f, eq + BK * (CPB - 1 - k));
             const float *qv = qt + (bi * G + head) * D;
+            const float qs2 = ldexpf(1.f, eqv[bi * G + head]);
             uint32_t packed = 0;
+            if (WPT >= 2 || rho == 0) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const float val = qv[half ? dhi : dlo] * scale;
-                const __half hi = __float2half_rn(val);
-                const __half pc = piece ? __float2half_rn(val - __half2float(hi)) : hi;
-                packed |= (uint32_t)__half_as_ushort(pc) << (16 * half);
+                for (int j = 0; j < 4; ++j) {
+                    // key slot 16 rho + 4t + j <-> byte 4 WPT t + 8c + 4 rho + j, field k
+                    const int byte = WPT >= 2 ? 4 * WPT * t + 8 * c + 4 * rho + j : 4 * t + j;
+                    const int qi = (int)rintf(qv[CPB * byte + k] * qs2);
+                    const int hi = (qi + 128) >> 8, lo = qi - 256 * hi;   // qi = 256 hi + lo
+                    packed |= (uint32_t)(uint8_t)(int8_t)(piece ? lo : hi) << (8 * j);
+                }
             }
             fr[idx] = packed;
         }
@@ -402,25 +394,26 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // q~ operand fragments and per-head constants
-    uint32_t qB[C::NT][C::KSTEPS][2];
+    uint32_t qB[C::NT][C::KS][2];
     {
         const uint32_t *fr = P.qfrag + pair * (size_t)C::QFRAG;
 #pragma unroll
         for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
-            for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                uint2 v = reinterpret_cast<const uint2 *>(fr)[(nt * C::KSTEPS + ks) * 32 + lane];
+            for (int ks = 0; ks < C::KS; ++ks) {
+                uint2 v = reinterpret_cast<const uint2 *>(fr)[(nt * C::KS + ks) * 32 + lane];
                 qB[nt][ks][0] = v.x;
                 qB[nt][ks][1] = v.y;
             }
     }
     // Thread (g, t) owns head 4nt + t of every n-tile nt (columns 2t = hi, 2t+1 = lo) and
     // tokens g, g+8 of every 16-token sub-tile.
-    const float cs = P.qscale[pair];
-    float wq[C::NT];
+    float cs[C::NT], wq[C::NT];
 #pragma unroll
-    for (int nt = 0; nt < C::NT; ++nt)
+    for (int nt = 0; nt < C::NT; ++nt) {
+        cs[nt] = P.qscale[(size_t)b * P.Hq + h * G + 4 * nt + t];
         wq[nt] = P.qw[(size_t)b * P.Hq + h * G + 4 * nt + t];
+    }
 
     float m_run[C::NT], l_run[C::NT], lz_run[C::NT];
     float O[C::MT][C::NT][4];
@@ -444,9 +437,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
         const uint32_t *vszw =
             reinterpret_cast<const uint32_t *>(st + C::KC_BYTES + C::SZ_BYTES + C::VC_BYTES);
 
-        // ---- scores S^T for 4 sub-tiles: independent chains interleaved per k-step.
-        //      Accumulator rows g and g+8 hold tokens ta and tb of the sub-tile (see below).
-        float S[4][C::NT][4];
+        // ---- scores S^T for 4 sub-tiles on int8 MMAs. A k-step takes one field position k
+        //      of every code byte, masked in place (uint8 c * 2^(BK k)); the field steps are
+        //      accumulated Horner-style (x 2^BK between them), so each score is the exact
+        //      integer 2^(BK(CPB-1)) * sum_j c_j q_int_j. Accumulator rows g and g+8 hold
+        //      tokens ta and tb of the sub-tile (see below).
+        int S[4][C::NT][4];
         uint32_t kw[4][2][C::WPT];
 #pragma unroll
         for (int stt = 0; stt < 4; ++stt) {
@@ -457,20 +453,38 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
             for (int nt = 0; nt < C::NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    S[stt][nt][i] = 0.f;
+                    S[stt][nt][i] = 0;
         }
 #pragma unroll
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        for (int k = 0; k < C::CPBK; ++k) {
+            if (k > 0) {
 #pragma unroll
-            for (int stt = 0; stt < 4; ++stt) {
-                const uint32_t a0 = ext_k<BK, C::CPBK>(kw[stt][0], 2 * ks);
-                const uint32_t a1 = ext_k<BK, C::CPBK>(kw[stt][1], 2 * ks);
-                const uint32_t a2 = ext_k<BK, C::CPBK>(kw[stt][0], 2 * ks + 1);
-                const uint32_t a3 = ext_k<BK, C::CPBK>(kw[stt][1], 2 * ks + 1);
+                for (int stt = 0; stt < 4; ++stt)
 #pragma unroll
-                for (int nt = 0; nt < C::NT; ++nt)
-                    mma_f16(S[stt][nt], a0, a1, a2, a3, qB[nt][ks][0], qB[nt][ks][1]);
+                    for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            S[stt][nt][i] *= (1 << BK);
             }
+            const uint32_t M = (((1u << BK) - 1u) * 0x01010101u) << (BK * k);
+#pragma unroll
+            for (int c = 0; c < C::KCH; ++c)
+#pragma unroll
+                for (int stt = 0; stt < 4; ++stt) {
+                    if constexpr (C::WPT >= 2) {
+                        const uint32_t a0 = kw[stt][0][2 * c] & M, a1 = kw[stt][1][2 * c] & M;
+                        const uint32_t a2 = kw[stt][0][2 * c + 1] & M, a3 = kw[stt][1][2 * c + 1] & M;
+#pragma unroll
+                        for (int nt = 0; nt < C::NT; ++nt)
+                            imma_k32(S[stt][nt], a0, a1, a2, a3, qB[nt][k * C::KCH + c][0],
+                                     qB[nt][k * C::KCH + c][1]);
+                    } else {
+                        const uint32_t a0 = kw[stt][0][0] & M, a1 = kw[stt][1][0] & M;
+#pragma unroll
+                        for (int nt = 0; nt < C::NT; ++nt)
+                            imma_k16(S[stt][nt], a0, a1, qB[nt][k][0]);
+                    }
+                }
         }
 
         // ---- logits (log2 units): hi + lo columns, then the per-token affine terms
@@ -485,12 +499,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
             for (int tk = 0; tk < 2; ++tk) {
                 const int tl = 16 * stt + (tk ? tb : ta);
                 const float2 sz = half2_bits_to_float2(kszw[tl]);
-                const float a = sz.x * cs;
                 const bool valid = FULL || (tok0 + tl < t_end);
 #pragma unroll
                 for (int nt = 0; nt < C::NT; ++nt) {
-                    const float v = S[stt][nt][2 * tk] + S[stt][nt][2 * tk + 1];
-                    float l2 = fmaf(a, v, sz.y * wq[nt]);
+                    // columns hi, lo of the head: q_int = 256 hi + lo (exact in int32)
+                    const float v = (float)(S[stt][nt][2 * tk] * 256 + S[stt][nt][2 * tk + 1]);
+                    float l2 = fmaf(sz.x * cs[nt], v, sz.y * wq[nt]);
                     if constexpr (!FULL)
                         l2 = valid ? l2 : -INFINITY;
                     L2[stt][tk][nt] = l2;

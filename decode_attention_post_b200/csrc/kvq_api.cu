@@ -128,7 +128,7 @@ static DecodeWorkspace decode_layout(int B, int Hkv, int Hq, int d, int nsplit)
     w.qfrag = off;
     off += up256((size_t)B * Hkv * decode_qfrag_words(d, G) * 4);
     w.qscale = off;
-    off += up256((size_t)B * Hkv * 4);
+    off += up256((size_t)B * Hq * 4);
     w.qw = off;
     off += up256((size_t)B * Hq * 4);
     w.part = off;
