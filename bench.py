@@ -36,7 +36,7 @@ METRIC = "2-bit KV decode attention: achieved HBM GB/s and % of B200 peak; appen
 CONFIG_IDX = 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one decode_kernel launch on this workload
 # (ncu --set full --clock-control none, profiles directory); None once the kernel changes.
-DECODE_TRAFFIC_BYTES = 549_279_744
+DECODE_TRAFFIC_BYTES = 546_765_312
 DECODE_TRAFFIC_KERNEL = "decode_kernel<128,4,2,2>"
 APPEND_CONFIG_IDX = 4
 
@@ -337,7 +337,7 @@ def run_gpu(args):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "2-bit codes -> f16 mma, f32 accumulate/softmax", "data": "synthetic",
+        "dtype": "2-bit codes -> int8 mma (keys), f16 mma (values), f32 softmax", "data": "synthetic",
         "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
                    "T_cap": cfg.T_cap, "seqlens": f"U[{cfg.seq_lo},{cfg.seq_hi}]",
                    "sum_seqlens": int(np.sum(w.seqlens)), "bits_k": cfg.bits_k,

@@ -342,6 +342,23 @@ def test_decode_edge_lengths():
     assert err == 0 and not out.any()
 
 
+@pytest.mark.parametrize("qscale", [1e-30, 1e-6, 1e3, 1e12])
+def test_decode_query_magnitude(qscale):
+    # the key product runs on q~ as per-head 16-bit fixed point: its exponent must follow
+    # the query's magnitude from tiny to huge (softmax over near-equal or one-hot logits)
+    cfg = small(synth.CONFIGS[2], T_cap=512)
+    seql = [512, 300]
+    oc, M = oracle_built_cache(cfg, 2, 512)
+    gc = upload_cache(oc, cfg)
+    q = synth.queries(cfg.with_(B=2)).astype(np.float64)
+    q[:, ::3] *= 1e-3                                   # heads of very different sizes
+    q = synth.as_dtype((q * qscale).astype(np.float32), "f32")
+    want = oracle.decode(q, M, oc, np.array(seql, np.int32))
+    out, err = gpu_decode(cfg, q, M, gc, seql)
+    assert err == 0
+    assert_close(out.cpu().numpy(), want, where=f"qscale={qscale}")
+
+
 def test_decode_seqlen_beyond_max_is_clamped_and_flagged():
     cfg = small(synth.CONFIGS[1], T_cap=256)
     oc, M = oracle_built_cache(cfg, 1, 256)
