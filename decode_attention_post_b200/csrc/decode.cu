@@ -317,7 +317,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     int *flag_smem = reinterpret_cast<int *>(bars_all + kDecodeWarps * kDecodeStages);
 
     const int h = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31;
+    // the warp index through a broadcast shuffle: the compiler then knows it is the same
+    // in every lane, keeps the ring and copy addresses in uniform registers and issues the
+    // bulk copies from them directly
+    const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
     const int g = lane >> 2, t = lane & 3;
     // Tokens of a 16-token sub-tile held in accumulator rows g and g+8: row 2i holds token
     // i and row 2i+1 token i+8 (i < 4), row 8+2i token i+4 and row 9+2i token i+12. After
@@ -355,38 +359,22 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     }
     __syncwarp();
 
-    // Block jj of this warp into stage s: lane 0 announces the stage's bytes, then lanes
-    // 0..3 each issue one bulk copy (K codes, K scale/zero, V codes, V scale/zero).
-    // Called by the whole warp.
+    // Block jj of this warp into stage s: lane 0 announces the stage's bytes and issues the
+    // four bulk copies (K codes, K scale/zero, V codes, V scale/zero). Called by the whole
+    // warp.
     auto issue = [&](int jj, int s) {
         const int tok0 = t_begin + (warp + jj * kDecodeWarps) * kDecodeBlock;
         unsigned char *st = wring + s * C::STAGE;
-        if (lane == 0)
+        if (lane == 0) {
             mbar_arrive_expect_tx_relaxed(&bars[s], C::STAGE);
-        __syncwarp();
-        if (lane < 4) {
-            const void *src;
-            unsigned char *dst;
-            uint32_t bytes;
-            if (lane == 0) {
-                src = kc + (size_t)tok0 * C::ROWK;
-                dst = st;
-                bytes = C::KC_BYTES;
-            } else if (lane == 1) {
-                src = ksz + (size_t)tok0 * 4;
-                dst = st + C::KC_BYTES;
-                bytes = C::SZ_BYTES;
-            } else if (lane == 2) {
-                src = vc + (size_t)tok0 * (D * BV / 8);
-                dst = st + C::KC_BYTES + C::SZ_BYTES;
-                bytes = C::VC_BYTES;
-            } else {
-                src = vsz + (size_t)tok0 * 4;
-                dst = st + C::KC_BYTES + C::SZ_BYTES + C::VC_BYTES;
-                bytes = C::SZ_BYTES;
-            }
-            bulk_g2s(dst, src, bytes, &bars[s]);
+            bulk_g2s(st, kc + (size_t)tok0 * C::ROWK, C::KC_BYTES, &bars[s]);
+            bulk_g2s(st + C::KC_BYTES, ksz + (size_t)tok0 * 4, C::SZ_BYTES, &bars[s]);
+            bulk_g2s(st + C::KC_BYTES + C::SZ_BYTES, vc + (size_t)tok0 * (D * BV / 8),
+                     C::VC_BYTES, &bars[s]);
+            bulk_g2s(st + C::KC_BYTES + C::SZ_BYTES + C::VC_BYTES, vsz + (size_t)tok0 * 4,
+                     C::SZ_BYTES, &bars[s]);
         }
+        __syncwarp();
     };
     for (int jj = 0; jj < kDecodeStages && jj < my_nblk; ++jj)
         issue(jj, jj);
