@@ -362,6 +362,7 @@ def run_gpu(args):
 
     if not args.no_extras:
         line["bf16_comparator"] = bf16_comparator(w, cfg, K, stream, dec_ms)
+        line["paged_decode"] = paged_decode(w, cfg, K, stream, dec_ms, dec_bytes)
         del w
         torch.cuda.empty_cache()
         line["chunk_append"] = chunk_append(device, stream)
@@ -384,6 +385,37 @@ def bf16_comparator(w, cfg, K, stream, dec_ms):
     nbytes = int(np.sum(w.seqlens)) * cfg.Hkv * cfg.d * 2 * 2 + 2 * cfg.B * cfg.Hq * cfg.d * 2
     return {"ms_per_launch": round(ms, 5), "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
             "bytes_per_launch": nbytes, "speedup_of_2bit_decode": round(ms / dec_ms, 2)}
+
+
+def paged_decode(w, cfg, K, stream, dec_ms, dec_bytes, page_tokens=256):
+    """The same decode over a page pool: the workload's cache moved into shuffled pages of
+    `page_tokens` positions (block table read by the kernels at every call)."""
+    import torch
+    import decode_attention_post_b200 as kvq
+    per = cfg.T_cap // page_tokens
+    num_pages = cfg.B * per + 64
+    perm = np.random.default_rng(1000 * cfg.idx + 7).permutation(num_pages)[:cfg.B * per]
+    table = torch.from_numpy(perm.reshape(cfg.B, per).astype(np.int32)).to(w.dev)
+    pc = kvq.KVCache.allocate_paged(num_pages, page_tokens, table, cfg.Hkv, cfg.d, w.qp,
+                                    device=w.dev, zero=False)
+    idx = table.reshape(-1).long()
+    for src, dst in zip((w.cache.k_codes, w.cache.k_sz, w.cache.v_codes, w.cache.v_sz),
+                        (pc.k_codes, pc.k_sz, pc.v_codes, pc.v_sz)):
+        tb = src.numel() // (cfg.B * cfg.Hkv * cfg.T_cap)
+        s5 = src.view(cfg.B, cfg.Hkv, per, page_tokens, tb).permute(0, 2, 1, 3, 4)
+        dst.view(num_pages, cfg.Hkv, page_tokens, tb).index_copy_(
+            0, idx, s5.reshape(cfg.B * per, cfg.Hkv, page_tokens, tb))
+    out = torch.empty_like(w.out)
+    fn = lambda: kvq.decode_attention(w.q, w.Tit, pc, w.seq_d, w.max_seqlen, out, w.ws,
+                                      dev_err=w.err)
+    ms = statistics.mean(time_events(fn, min(K, 500), stream))
+    w.decode()
+    torch.cuda.synchronize()
+    same = bool(torch.equal(out.view(torch.int16), w.out.view(torch.int16)))
+    del pc
+    return {"page_tokens": page_tokens, "num_pages": num_pages, "ms_per_launch": round(ms, 5),
+            "GB_s": round(dec_bytes / (ms * 1e-3) / 1e9, 1),
+            "time_vs_contiguous": round(ms / dec_ms, 4), "output_identical": same}
 
 
 def chunk_append(device, stream):

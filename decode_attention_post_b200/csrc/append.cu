@@ -15,7 +15,8 @@
 //      (ties to even), so they match the float64 definition bit for bit.
 //   5. Codes are gathered through shared memory and written as whole 32-bit words
 //      (K rows) or whole 16-bit halves (V tiles); every token owns whole bytes, so
-//      no read-modify-write is needed even for single-token appends.
+//      no read-modify-write is needed even for single-token appends. The token slot
+//      comes from the contiguous layout or, for a paged cache, the block table.
 #include "kvq_common.cuh"
 
 namespace kvq {
@@ -79,7 +80,7 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
                    int Hkv, int T_cap, int bits_k, int bits_v, int group, int kappa,
                    uint8_t *__restrict__ k_codes, uint32_t *__restrict__ k_sz,
                    uint8_t *__restrict__ v_codes, uint32_t *__restrict__ v_sz,
-                   const int32_t *__restrict__ pos, int32_t *dev_err)
+                   const int32_t *__restrict__ pos, int32_t *dev_err, PageMap pm)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     using Smem = AppendSmem<D, TPW>;
@@ -179,7 +180,12 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
                 continue;
             }
             const int t = p0 + i;
-            const size_t row = ((size_t)b * Hkv + h) * T_cap + t;
+            const long long row = cache_row(pm, b, h, Hkv, T_cap, t);
+            if (row < 0) {
+                if (lane == 0)
+                    flag(dev_err, KVQ_DEVERR_PAGE_RANGE);
+                continue;
+            }
             for (int gr = 0; gr < ng; ++gr) {
                 // group gr covers dims [gr*group, (gr+1)*group), i.e. r in [r0, r0+nr);
                 // dims outside the group are padded with +-inf so they are never picked.
@@ -237,9 +243,8 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
                     for (int s2 = 0; s2 < E; ++s2)
                         hv |= (uint32_t)sm.codes[warp][8 * (E * r + s2) + gq] << (bits * s2);
                     const size_t tile_base =
-                        (((size_t)b * Hkv + h) * (T_cap / kTileTokens) + t / kTileTokens) *
-                        (kTileTokens * D * bits / 8);
-                    const int off = v_half_offset(D, bits, t % kTileTokens, gq, r);
+                        (size_t)(row / kTileTokens) * (kTileTokens * D * bits / 8);
+                    const int off = v_half_offset(D, bits, (int)(row % kTileTokens), gq, r);
                     *reinterpret_cast<uint16_t *>(v_codes + tile_base + off) = (uint16_t)hv;
                 }
             }
@@ -279,7 +284,7 @@ cudaError_t launch_append_fp32(const void *k, const void *v, int in_bf16, const 
     append_fp32_kernel<D, TPW><<<grid, kAppendThreads, smem, st>>>(
         k, v, in_bf16, Tk, Tv, B, n, c->Hkv, c->T_cap, c->qp.bits_k, c->qp.bits_v, c->qp.group,
         kappa, (uint8_t *)c->k_codes, (uint32_t *)c->k_sz, (uint8_t *)c->v_codes,
-        (uint32_t *)c->v_sz, pos, dev_err);
+        (uint32_t *)c->v_sz, pos, dev_err, PageMap{c->block_table, c->page_tokens, c->num_pages});
     return cudaGetLastError();
 }
 

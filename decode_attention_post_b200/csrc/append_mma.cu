@@ -138,7 +138,7 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                   int Hkv, int T_cap, int bits_k, int bits_v, int group, int kappa,
                   uint8_t *__restrict__ k_codes, uint32_t *__restrict__ k_sz,
                   uint8_t *__restrict__ v_codes, uint32_t *__restrict__ v_sz,
-                  const int32_t *__restrict__ pos, int32_t *dev_err)
+                  const int32_t *__restrict__ pos, int32_t *dev_err, PageMap pm)
 {
     using Sm = MmaSmem<D>;
     constexpr int TS = Sm::TS, NT = D / 8, NV = 2 * NT;
@@ -258,12 +258,21 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                 i -= n;
                 ++b;
             }
+            long long row = 0;                        // token slot in the planes
             if (ok) {
                 p0 = pos[b];
                 if (p0 < 0 || (long)p0 + n > T_cap) {
                     if (i == 0 && t == 0)
                         flag(dev_err, KVQ_DEVERR_POS_RANGE);
                     ok = false;
+                } else {
+                    row = cache_row(pm, b, h, Hkv, T_cap, p0 + i);
+                    if (row < 0) {
+                        if (t == 0)
+                            flag(dev_err, KVQ_DEVERR_PAGE_RANGE);
+                        ok = false;
+                        row = 0;
+                    }
                 }
             }
             // this lane's values of the token: columns 8nt + 2t + {0, 1}
@@ -358,7 +367,6 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                     cq[e] = (uint32_t)c;
                 }
                 if (ok && t == 0) {
-                    const size_t row = ((size_t)b * Hkv + h) * T_cap + p0 + i;
                     const uint32_t pair = (uint32_t)__half_as_ushort(sh) |
                                           ((uint32_t)__half_as_ushort(zh) << 16);
                     (which ? v_sz : k_sz)[row * ng + gr] = pair;
@@ -366,7 +374,6 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
             }
 
             // ---- packed stores, built in registers
-            const size_t row = ((size_t)b * Hkv + h) * T_cap + p0 + i;
             if (!which) {
                 uint32_t *dst = reinterpret_cast<uint32_t *>(k_codes + row * (D * bits / 8));
                 if (bits == 2)
@@ -374,14 +381,13 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                 else
                     store_k_row<D, 4>(cq, dst, t, ok);
             } else if (ok) {
-                const int tpos = p0 + i;
                 unsigned char *tile_base =
-                    v_codes + (((size_t)b * Hkv + h) * (T_cap / kTileTokens) + tpos / kTileTokens) *
-                                  (kTileTokens * D * bits / 8);
+                    v_codes + (size_t)(row / kTileTokens) * (kTileTokens * D * bits / 8);
+                const int tok = (int)(row % kTileTokens);
                 if (bits == 2)
-                    store_v_halves<D, 2>(cq, tile_base, tpos % kTileTokens, t);
+                    store_v_halves<D, 2>(cq, tile_base, tok, t);
                 else
-                    store_v_halves<D, 4>(cq, tile_base, tpos % kTileTokens, t);
+                    store_v_halves<D, 4>(cq, tile_base, tok, t);
             }
         }
         __syncwarp();
@@ -417,7 +423,8 @@ cudaError_t launch_mma(const void *k, const void *v, const float *Tk, const floa
     append_mma_kernel<D><<<grid, kMmaWarps * 32, smem, st>>>(
         (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, Tk, Tv, B, n, c->Hkv, c->T_cap,
         c->qp.bits_k, c->qp.bits_v, c->qp.group, kappa, (uint8_t *)c->k_codes,
-        (uint32_t *)c->k_sz, (uint8_t *)c->v_codes, (uint32_t *)c->v_sz, pos, dev_err);
+        (uint32_t *)c->k_sz, (uint8_t *)c->v_codes, (uint32_t *)c->v_sz, pos, dev_err,
+        PageMap{c->block_table, c->page_tokens, c->num_pages});
     return cudaGetLastError();
 }
 

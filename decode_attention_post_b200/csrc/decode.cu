@@ -347,10 +347,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     unsigned char *wring = ring + warp * kDecodeStages * C::STAGE;
     uint64_t *bars = bars_all + warp * kDecodeStages;
 
-    const uint8_t *kc = P.k_codes + pair * (size_t)P.T_cap * C::ROWK;
-    const uint8_t *ksz = reinterpret_cast<const uint8_t *>(P.k_sz + pair * (size_t)P.T_cap);
-    const uint8_t *vc = P.v_codes + pair * (size_t)P.T_cap * (D * BV / 8);
-    const uint8_t *vsz = reinterpret_cast<const uint8_t *>(P.v_sz + pair * (size_t)P.T_cap);
+    const PageMap pm{P.block_table, P.page_tokens, P.num_pages};
 
     if (lane == 0) {
         for (int s = 0; s < kDecodeStages; ++s)
@@ -360,19 +357,30 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     __syncwarp();
 
     // Block jj of this warp into stage s: lane 0 announces the stage's bytes and issues the
-    // four bulk copies (K codes, K scale/zero, V codes, V scale/zero). Called by the whole
-    // warp.
+    // four bulk copies (K codes, K scale/zero, V codes, V scale/zero) of the block's 64
+    // token slots (contiguous, or one page-aligned run of a page: page_tokens is a
+    // multiple of 64). Called by the whole warp.
     auto issue = [&](int jj, int s) {
         const int tok0 = t_begin + (warp + jj * kDecodeWarps) * kDecodeBlock;
         unsigned char *st = wring + s * C::STAGE;
         if (lane == 0) {
+            long long row0;
+            if (!pm.table) {
+                row0 = (long long)pair * P.T_cap + tok0;
+            } else {
+                row0 = cache_row(pm, b, h, P.Hkv, P.T_cap, tok0);
+                if (row0 < 0) {                 // out-of-range page: flagged, read page 0
+                    flag(P.dev_err, KVQ_DEVERR_PAGE_RANGE);
+                    row0 = (long long)h * pm.page_tokens + tok0 % pm.page_tokens;
+                }
+            }
             mbar_arrive_expect_tx_relaxed(&bars[s], C::STAGE);
-            bulk_g2s(st, kc + (size_t)tok0 * C::ROWK, C::KC_BYTES, &bars[s]);
-            bulk_g2s(st + C::KC_BYTES, ksz + (size_t)tok0 * 4, C::SZ_BYTES, &bars[s]);
-            bulk_g2s(st + C::KC_BYTES + C::SZ_BYTES, vc + (size_t)tok0 * (D * BV / 8),
+            bulk_g2s(st, P.k_codes + row0 * C::ROWK, C::KC_BYTES, &bars[s]);
+            bulk_g2s(st + C::KC_BYTES, P.k_sz + row0, C::SZ_BYTES, &bars[s]);
+            bulk_g2s(st + C::KC_BYTES + C::SZ_BYTES, P.v_codes + row0 * (D * BV / 8),
                      C::VC_BYTES, &bars[s]);
-            bulk_g2s(st + C::KC_BYTES + C::SZ_BYTES + C::VC_BYTES, vsz + (size_t)tok0 * 4,
-                     C::SZ_BYTES, &bars[s]);
+            bulk_g2s(st + C::KC_BYTES + C::SZ_BYTES + C::VC_BYTES, P.v_sz + row0, C::SZ_BYTES,
+                     &bars[s]);
         }
         __syncwarp();
     };

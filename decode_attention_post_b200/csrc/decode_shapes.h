@@ -29,6 +29,9 @@ struct DecodeParams {
     void *out;
     int out_bf16;
     int32_t *dev_err;
+    const int32_t *block_table; // paged cache: [B][T_cap/page_tokens]; nullptr = contiguous
+    int page_tokens;
+    int num_pages;
 };
 
 struct DecodeLaunch {

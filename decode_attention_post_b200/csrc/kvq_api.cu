@@ -77,6 +77,16 @@ static kvq_status check_cache(const kvq_cache *c)
     if (!aligned(c->k_codes, 16) || !aligned(c->k_sz, 16) || !aligned(c->v_codes, 16) ||
         !aligned(c->v_sz, 16))
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "cache planes must be 16-byte aligned");
+    if (c->block_table) {
+        if (c->page_tokens <= 0 || c->page_tokens % kDecodeBlock || c->T_cap % c->page_tokens)
+            KVQ_FAIL(KVQ_ERR_INVALID_ARG,
+                     "page_tokens=%d must be a positive multiple of %d dividing T_cap=%d",
+                     c->page_tokens, kDecodeBlock, c->T_cap);
+        if (c->num_pages <= 0)
+            KVQ_FAIL(KVQ_ERR_INVALID_ARG, "num_pages=%d must be positive", c->num_pages);
+        if (!aligned(c->block_table, 4))
+            KVQ_FAIL(KVQ_ERR_INVALID_ARG, "block_table must be 4-byte aligned");
+    }
     return KVQ_OK;
 }
 
@@ -185,7 +195,12 @@ size_t kvq_cache_plane_bytes(const kvq_cache *c, int which)
     if (!c || c->B <= 0 || c->Hkv <= 0 || c->T_cap <= 0 || c->d <= 0 || c->qp.group <= 0 ||
         c->d % c->qp.group)
         return 0;
-    const size_t tok = (size_t)c->B * c->Hkv * c->T_cap;
+    size_t tok = (size_t)c->B * c->Hkv * c->T_cap;
+    if (c->block_table) {
+        if (c->page_tokens <= 0 || c->page_tokens % kDecodeBlock || c->num_pages <= 0)
+            return 0;
+        tok = (size_t)c->num_pages * c->Hkv * c->page_tokens;
+    }
     switch (which) {
     case 0: return tok * c->d * c->qp.bits_k / 8;
     case 1: return tok * (c->d / c->qp.group) * 4;
@@ -278,6 +293,9 @@ kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const 
     L.p.out = out;
     L.p.out_bf16 = out_dtype == KVQ_BF16;
     L.p.dev_err = dev_err;
+    L.p.block_table = c->block_table;
+    L.p.page_tokens = c->page_tokens;
+    L.p.num_pages = c->num_pages;
     L.q = q;
     L.q_bf16 = q_dtype == KVQ_BF16;
     L.M = Tk_invT;

@@ -40,6 +40,29 @@ __host__ __device__ __forceinline__ int v_half_offset(int d, int bits, int tok, 
     return lane * chunk + (p * W + r) * 4 + 2 * hi;
 }
 
+// Where the positions of a (sequence, KV head) live: contiguous planes [B][Hkv][T_cap]
+// (table == nullptr) or pages [page][Hkv][page_tokens] through a block table
+// [B][T_cap / page_tokens].
+struct PageMap {
+    const int32_t *table;
+    int page_tokens;
+    int num_pages;
+};
+
+// Token slot (row of the K-code and scale/zero planes; value tiles hold slots
+// 16i..16i+15) of position t of sequence b, KV head h. -1 if the block table holds a page
+// outside [0, num_pages).
+__device__ __forceinline__ long long cache_row(const PageMap &pm, int b, int h, int Hkv, int T_cap,
+                                               int t)
+{
+    if (!pm.table)
+        return ((long long)b * Hkv + h) * T_cap + t;
+    const int page = pm.table[(size_t)b * (T_cap / pm.page_tokens) + t / pm.page_tokens];
+    if ((unsigned)page >= (unsigned)pm.num_pages)
+        return -1;
+    return ((long long)page * Hkv + h) * pm.page_tokens + t % pm.page_tokens;
+}
+
 // Host-side: thread-local last error text.
 void set_error(const char *fmt, ...);
 

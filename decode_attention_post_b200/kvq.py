@@ -33,7 +33,8 @@ class _QParams(C.Structure):
 
 class _Cache(C.Structure):
     _fields_ = [("B", _I), ("Hkv", _I), ("T_cap", _I), ("d", _I), ("qp", _QParams),
-                ("k_codes", _P), ("k_sz", _P), ("v_codes", _P), ("v_sz", _P)]
+                ("k_codes", _P), ("k_sz", _P), ("v_codes", _P), ("v_sz", _P),
+                ("block_table", _P), ("page_tokens", _I), ("num_pages", _I)]
 
 
 class KvqError(RuntimeError):
@@ -130,20 +131,30 @@ class KVCache:
     """The four cache planes (caller-owned device memory) plus their shape.
 
     ``KVCache.allocate`` asks the library for each plane's size and allocates it with
-    torch; ``KVCache(planes=...)`` wraps existing uint8 tensors.
+    torch; ``KVCache(planes=...)`` wraps existing uint8 tensors. With ``block_table``
+    (int32 [B][T_cap/page_tokens] on the device) the planes are page pools of
+    ``num_pages`` pages (``KVCache.allocate_paged``).
     """
 
-    def __init__(self, B, Hkv, T_cap, d, qp: QParams, planes):
+    def __init__(self, B, Hkv, T_cap, d, qp: QParams, planes, block_table=None,
+                 page_tokens=0, num_pages=0):
         self.B, self.Hkv, self.T_cap, self.d, self.qp = B, Hkv, T_cap, d, qp
         self.k_codes, self.k_sz, self.v_codes, self.v_sz = planes
         for name, t in zip(("k_codes", "k_sz", "v_codes", "v_sz"), planes):
             _cuda(name, t, torch.uint8)
+        _cuda("block_table", block_table, torch.int32)
+        self.block_table, self.page_tokens, self.num_pages = block_table, page_tokens, num_pages
         self._desc = _Cache(B, Hkv, T_cap, d, qp._c(), _ptr(self.k_codes), _ptr(self.k_sz),
-                            _ptr(self.v_codes), _ptr(self.v_sz))
+                            _ptr(self.v_codes), _ptr(self.v_sz), _ptr(block_table),
+                            page_tokens if block_table is not None else 0,
+                            num_pages if block_table is not None else 0)
 
     @staticmethod
-    def plane_bytes(B, Hkv, T_cap, d, qp: QParams):
-        desc = _Cache(B, Hkv, T_cap, d, qp._c(), None, None, None, None)
+    def plane_bytes(B, Hkv, T_cap, d, qp: QParams, page_tokens=0, num_pages=0):
+        """Plane sizes; with page_tokens > 0, those of a pool of num_pages pages."""
+        paged = page_tokens > 0
+        desc = _Cache(B, Hkv, T_cap, d, qp._c(), None, None, None, None,
+                      C.c_void_p(16) if paged else None, page_tokens, num_pages)
         return [int(load().kvq_cache_plane_bytes(C.byref(desc), w)) for w in range(4)]
 
     @classmethod
@@ -155,8 +166,26 @@ class KVCache:
         planes = [make(n, dtype=torch.uint8, device=device) for n in sizes]
         return cls(B, Hkv, T_cap, d, qp, planes)
 
+    @classmethod
+    def allocate_paged(cls, num_pages, page_tokens, block_table, Hkv, d, qp: QParams,
+                       device="cuda", zero=True):
+        """A pool of num_pages pages; block_table int32 [B][pages per sequence] on the
+        device gives the page of every page_tokens positions of every sequence."""
+        B, per_seq = block_table.shape
+        T_cap = per_seq * page_tokens
+        sizes = cls.plane_bytes(B, Hkv, T_cap, d, qp, page_tokens, num_pages)
+        if min(sizes) <= 0:
+            raise ValueError("invalid paged cache shape")
+        make = torch.zeros if zero else torch.empty
+        planes = [make(n, dtype=torch.uint8, device=device) for n in sizes]
+        return cls(B, Hkv, T_cap, d, qp, planes, block_table, page_tokens, num_pages)
+
     def view_sequence(self, b: int) -> "KVCache":
         """The same cache restricted to sequence b (a B = 1 view of its planes)."""
+        if self.block_table is not None:
+            return KVCache(1, self.Hkv, self.T_cap, self.d, self.qp,
+                           (self.k_codes, self.k_sz, self.v_codes, self.v_sz),
+                           self.block_table[b:b + 1], self.page_tokens, self.num_pages)
         per = [p.numel() // self.B for p in (self.k_codes, self.k_sz, self.v_codes, self.v_sz)]
         planes = [p[b * n:(b + 1) * n] for p, n in zip((self.k_codes, self.k_sz, self.v_codes,
                                                          self.v_sz), per)]

@@ -65,6 +65,8 @@ typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
 #define KVQ_DEVERR_POS_RANGE      0x2   /* pos[b] < 0 or pos[b] + n > T_cap: sequence skipped */
 #define KVQ_DEVERR_NONFINITE      0x4   /* a group had a non-finite clip range: codes 0 */
 #define KVQ_DEVERR_WAIT_TIMEOUT   0x8   /* a bounded pipeline wait gave up: output invalid */
+#define KVQ_DEVERR_PAGE_RANGE     0x10  /* a block-table entry outside [0, num_pages): the
+                                           append skips the token, the decode reads page 0 */
 
 /*
  * Quantizer parameters (WUSH-KV summary, section 5.3; percentile clipping).
@@ -100,6 +102,19 @@ typedef struct {
  *  k_sz, v_sz [B][Hkv][T_cap][d/group] pairs of float16 (s_h, z_h), s_h first (4 bytes).
  * T_cap must be a multiple of 64; d must be 64 or 128. All planes 16-byte aligned.
  * qp must equal the parameters passed to kvq_quantize_append.
+ *
+ * Paged layout (optional; the serving layout of a block table, NOVA-KV page, "Three
+ * requirements", item 3: fixed-width tokens make pages of equal size). With
+ * block_table != NULL the planes are pools of num_pages pages of page_tokens positions:
+ *  k_codes [num_pages][Hkv][page_tokens][d*bits_k/8], v_codes [num_pages][Hkv]
+ *  [page_tokens/16][16*d*bits_v/8], k_sz, v_sz [num_pages][Hkv][page_tokens][d/group],
+ * each page holding every KV head of page_tokens consecutive positions of one sequence.
+ * block_table is device int32 [B][T_cap/page_tokens]: position t of sequence b lives in
+ * page block_table[b][t / page_tokens] at slot t % page_tokens. page_tokens must be a
+ * multiple of 64 dividing T_cap; T_cap is the per-sequence capacity. The table is read
+ * on the device at every call (it may change between calls); an entry outside
+ * [0, num_pages) sets KVQ_DEVERR_PAGE_RANGE. block_table == NULL: contiguous planes as
+ * above, page_tokens and num_pages ignored.
  */
 typedef struct {
     int B;
@@ -111,9 +126,13 @@ typedef struct {
     void *k_sz;
     void *v_codes;
     void *v_sz;
+    const int32_t *block_table; /* NULL = contiguous; else device [B][T_cap/page_tokens] */
+    int page_tokens;            /* paged: positions per page, a multiple of 64 */
+    int num_pages;              /* paged: pages in each pool plane */
 } kvq_cache;
 
-/* Size in bytes of plane `which` (0 k_codes, 1 k_sz, 2 v_codes, 3 v_sz); 0 if invalid. */
+/* Size in bytes of plane `which` (0 k_codes, 1 k_sz, 2 v_codes, 3 v_sz); 0 if invalid.
+ * Paged caches: the size of the page pool (num_pages pages). */
 KVQ_API size_t kvq_cache_plane_bytes(const kvq_cache *cache, int which);
 
 /*

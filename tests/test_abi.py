@@ -53,6 +53,44 @@ def test_plane_bytes_follow_layout():
     assert kb * 8 / (2 * 2 * 128 * 128) == 2.25
 
 
+def _paged_desc(page_tokens=64, num_pages=10, table=0x8000, T_cap=128, **kw):
+    desc, qp = _desc(T_cap=T_cap, **kw)
+    desc.block_table = table
+    desc.page_tokens = page_tokens
+    desc.num_pages = num_pages
+    return desc, qp
+
+
+def test_paged_plane_bytes_are_pool_sizes():
+    L = kvq.load()
+    desc, _ = _paged_desc(page_tokens=128, num_pages=7, T_cap=256, B=3, Hkv=2, bits_k=4,
+                          bits_v=2)
+    tok = 7 * 2 * 128                                  # pages x heads x slots per page
+    want = [tok * 64, tok * 4, tok * 32, tok * 4]
+    assert [L.kvq_cache_plane_bytes(C.byref(desc), w) for w in range(4)] == want
+    bad, _ = _paged_desc(page_tokens=96)
+    assert L.kvq_cache_plane_bytes(C.byref(bad), 0) == 0
+
+
+@pytest.mark.parametrize("mut", [
+    dict(page_tokens=0), dict(page_tokens=96), dict(page_tokens=256),   # not a divisor of T_cap
+    dict(num_pages=0), dict(table=0x8002),                              # misaligned table
+])
+def test_paged_cache_validation(mut):
+    desc, qp = _paged_desc(**mut)
+    assert _append(desc, qp) == 1
+    assert kvq.load().kvq_last_error()
+    assert _decode(desc) == 1
+
+
+def test_paged_cache_accepted_shapes():
+    # argument checks pass (n = 0 is a no-op: nothing is launched)
+    desc, qp = _paged_desc(page_tokens=64, num_pages=4)
+    assert _append(desc, qp, n=0) == 0
+    desc, qp = _paged_desc(page_tokens=128, num_pages=1)
+    assert _append(desc, qp, n=0) == 0
+
+
 def _append(desc, qp, n=4, dtype=0, k=0x2000, pos=0x3000):
     L = kvq.load()
     return L.kvq_quantize_append(k, k, dtype, None, None, C.byref(qp), C.byref(desc), pos, n,

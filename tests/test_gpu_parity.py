@@ -18,7 +18,7 @@ import torch
 
 import decode_attention_post_b200 as kvq
 import oracle
-from tests import synth
+from tests import paging, synth
 
 pytestmark = pytest.mark.gpu
 
@@ -506,3 +506,84 @@ def test_bf16_decode_matches_oracle(G, d):
         assert np.all(np.abs(g - want) <= 0.5 * ulp + MAX_ABS), splits
         rl2 = np.linalg.norm(g - want) / np.linalg.norm(want)
         assert rl2 <= 3e-3, (splits, rl2)      # bf16 rounding alone is about 1.5e-3
+
+
+# ----------------------------------------------------------------------------- paged cache
+
+
+def _paged(cfg, B, page_tokens, extra_pages, seed):
+    per = cfg.T_cap // page_tokens
+    num_pages = B * per + extra_pages
+    table = paging.random_table(np.random.default_rng(seed), B, per, num_pages)
+    tb = paging.token_bytes(cfg.d, cfg.bits_k, cfg.bits_v, cfg.group)
+    return table, num_pages, tb
+
+
+def paged_upload(oc, cfg, page_tokens, extra_pages=5, seed=0):
+    """The oracle's contiguous planes moved into a shuffled page pool on the GPU."""
+    table, num_pages, tb = _paged(cfg, oc.B, page_tokens, extra_pages, seed)
+    pools = paging.scatter([p.view(np.uint8) for p in oc.planes()], table, oc.Hkv, oc.T_cap,
+                           page_tokens, num_pages, tb)
+    gc = kvq.KVCache.allocate_paged(num_pages, page_tokens, t_(table), oc.Hkv, oc.d, qp_of(cfg))
+    for dst, src in zip((gc.k_codes, gc.k_sz, gc.v_codes, gc.v_sz), pools):
+        dst.copy_(torch.from_numpy(src))
+    return gc
+
+
+@pytest.mark.parametrize("page_tokens", [64, 256])
+def test_paged_decode_matches_oracle(page_tokens):
+    cfg = small(synth.CONFIGS[2], T_cap=1024)
+    seql = [1000, 1, 577]
+    oc, M = oracle_built_cache(cfg, 3, 1024)
+    gc = paged_upload(oc, cfg, page_tokens, seed=page_tokens)
+    q = synth.as_dtype(synth.queries(cfg.with_(B=3)), cfg.q_dtype)
+    want = oracle.decode(q, M, oc, np.array(seql, np.int32))
+    out, err = gpu_decode(cfg, q, M, gc, seql)
+    assert err == 0
+    assert_close(out.cpu().numpy(), want, where=f"paged {page_tokens}")
+
+
+@pytest.mark.parametrize("cfg,B,n,pos,dtype,with_T", [
+    (small(synth.CONFIGS[1], T_cap=512), 3, 1, [0, 100, 511], "bf16", True),    # decode-time
+    (small(synth.CONFIGS[1], T_cap=512), 3, 77, [0, 64, 435], "f32", False),
+    (small(synth.CONFIGS[4], T_cap=512), 2, 300, [0, 212], "bf16", True),       # tensor cores
+])
+def test_paged_append_matches_contiguous_bytes(cfg, B, n, pos, dtype, with_T):
+    """An append into a shuffled page pool, gathered back, is byte-identical to the same
+    append into contiguous planes (which the oracle pins), and leaves unused pages empty."""
+    k, v = _inputs(cfg, B, n, dtype)
+    Tk, Tv, _ = synth.transforms(cfg) if with_T else (None, None, None)
+    ref, err = gpu_append(cfg, k, v, Tk, Tv, pos)
+    assert err == 0
+    if not with_T:
+        oc = oracle.Cache(B, cfg.Hkv, cfg.T_cap, cfg.d, cfg.bits_k, cfg.bits_v, cfg.group)
+        oracle.quantize_append(k, v, None, None, cfg.bits_k, cfg.bits_v, cfg.group,
+                               cfg.clip_alpha, oc, pos)
+        for a, b in zip(planes_to_host(ref), oc.planes()):
+            assert np.array_equal(a, b.view(np.uint8))
+    page_tokens = 128
+    table, num_pages, tb = _paged(cfg, B, page_tokens, 4, n)
+    gc = kvq.KVCache.allocate_paged(num_pages, page_tokens, t_(table), cfg.Hkv, cfg.d,
+                                    qp_of(cfg))
+    gc, err = gpu_append(cfg, k, v, Tk, Tv, pos, cache=gc)
+    assert err == 0
+    back = paging.gather(planes_to_host(gc), table, cfg.Hkv, page_tokens, tb)
+    for name, a, b in zip(("k_codes", "k_sz", "v_codes", "v_sz"), back, planes_to_host(ref)):
+        assert np.array_equal(a, b), name
+    unused = sorted(set(range(num_pages)) - set(table.reshape(-1).tolist()))
+    for pool in planes_to_host(gc):
+        assert not pool.reshape(num_pages, -1)[unused].any()
+
+
+def test_paged_out_of_range_page_is_flagged():
+    cfg = small(synth.CONFIGS[2], T_cap=256)
+    seql = [256, 130]
+    oc, M = oracle_built_cache(cfg, 2, 256)
+    gc = paged_upload(oc, cfg, 64, extra_pages=0)
+    gc.block_table[1, 1] = gc.num_pages + 3                 # outside the pool
+    q = synth.as_dtype(synth.queries(cfg.with_(B=2)), cfg.q_dtype)
+    out, err = gpu_decode(cfg, q, M, gc, seql)
+    assert err & 0x10
+    k, v = _inputs(cfg, 2, 1, "bf16")
+    _, err = gpu_append(cfg, k, v, None, None, [0, 70], cache=gc)   # 70 -> page entry [1][1]
+    assert err & 0x10
