@@ -168,8 +168,10 @@ KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int Hq, int ma
  *        domain; 0 for an empty sequence.
  *   workspace: device buffer of at least kvq_decode_workspace_bytes(...) bytes,
  *              256-byte aligned, used as scratch (contents need not be initialised).
- * Computed as a split-K flash decode: scores and P.V on tensor cores with float32
- * accumulation, float32 online softmax, then a merge of the splits.
+ * Computed as a split-K flash decode: scores on int8 tensor cores (key codes against q~
+ * as per-head 16-bit fixed point, exact int32 accumulation), float32 online softmax, P.V
+ * on float16 tensor cores with float32 accumulation, then a merge of the splits.
+ * Paged caches (block_table != NULL) are read through the block table.
  */
 KVQ_API kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const float *Tk_invT,
                                 const kvq_cache *cache, const int32_t *seqlens, int max_seqlen,
