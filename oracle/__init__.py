@@ -57,6 +57,11 @@ def lib():
         L.oracle_bf16_decode.restype = I
         L.oracle_v_code_pos.argtypes = [I, I, I, I, P, P]
         L.oracle_k_code_pos.argtypes = [I, I, I, P, P]
+        L.oracle_window_quantized.argtypes = [I, I, I, I]
+        L.oracle_window_quantized.restype = I
+        L.oracle_window_decode.argtypes = [P, I, I, I, I, I, P, P, P, P, I, I, I, I, I,
+                                           P, P, P, P, P, I, I, I, P]
+        L.oracle_window_decode.restype = I
         L.oracle_set_threads.argtypes = [I]
         L.oracle_get_threads.restype = I
         _lib = L
@@ -328,6 +333,40 @@ def bf16_decode(q_bits, K_bits, V_bits, seqlens, Hkv, sel=None) -> np.ndarray:
                                  _p(selc), nsel, _p(out))
     if r:
         raise ValueError("oracle_bf16_decode: bad arguments")
+    return out
+
+
+def window_quantized(L, S_sink, S_keep, S_flush) -> int:
+    """Quantized middle length Q of a sequence of L positions (full-precision window)."""
+    r = lib().oracle_window_quantized(int(L), int(S_sink), int(S_keep), int(S_flush))
+    if r < 0:
+        raise ValueError("oracle_window_quantized: bad arguments")
+    return r
+
+
+def window_decode(q, M, Tv, k_all, v_all, cache: Cache, seqlens, S_sink, S_keep,
+                  S_flush) -> np.ndarray:
+    """float64 [B][Hq][d] decode with a full-precision window: positions [S_sink,
+    S_sink + Q) from the quantized cache, the others from k_all, v_all [B][T_cap][Hkv][d]
+    (float32 or bf16 bits) with T_v [Hkv][d][d] (or None) applied to their values."""
+    dq, din = _dt(q), _dt(k_all)
+    assert _dt(v_all) == din
+    q = np.ascontiguousarray(q)
+    k_all, v_all = np.ascontiguousarray(k_all), np.ascontiguousarray(v_all)
+    B, Hq, d = q.shape
+    assert k_all.shape == (B, cache.T_cap, cache.Hkv, d)
+    Mc = None if M is None else _c(M, np.float32)
+    Tvc = None if Tv is None else _c(Tv, np.float32)
+    seqlens = _c(seqlens, np.int32)
+    out = np.full((B, Hq, d), np.nan, np.float64)
+    r = lib().oracle_window_decode(_p(q), dq, B, Hq, cache.Hkv, d, _p(Mc), _p(Tvc),
+                                   _p(k_all), _p(v_all), din, cache.T_cap, cache.bits_k,
+                                   cache.bits_v, cache.group, _p(cache.k_codes),
+                                   _p(cache.k_sz), _p(cache.v_codes), _p(cache.v_sz),
+                                   _p(seqlens), int(S_sink), int(S_keep), int(S_flush),
+                                   _p(out))
+    if r:
+        raise ValueError("oracle_window_decode: bad arguments")
     return out
 
 

@@ -18,6 +18,9 @@
  *     of query heads, over all cached positions.
  *   - "Spend Bits Where Queries Look" (NOVA-KV project page), "Three requirements",
  *     item 3: every token occupies the same number of bits (fixed-width layout).
+ *   - WUSH-KV page, section 4.4: the full-precision window (first S_sink and newest
+ *     S_keep positions kept in full precision, the middle quantized in batches of
+ *     S_flush) -- the decode over such a sequence.
  * Every step the pages leave open is stated next to the code that fixes it.
  *
  * Arithmetic: all transform and attention arithmetic is float64. Where the quantizer
@@ -654,6 +657,119 @@ int oracle_bf16_decode(const uint16_t *q, int B, int Hq, int Hkv, int d,
             l += p;
             for (int j = 0; j < d; ++j)
                 o[j] += p * oracle_bf16_to_f64(vr[j]);
+        }
+        for (int j = 0; j < d; ++j)
+            out[((size_t)b * Hq + hq) * d + j] = l > 0 ? o[j] / l : 0.0;
+        free(logit);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ full-precision window */
+
+/*
+ * Full-precision window ("WUSH-KV: KV Cache Quantization with Data-Adaptive
+ * Transforms", section 4.4): the first S_sink positions and the newest S_keep positions
+ * of a sequence stay in full precision, and the middle positions that are neither are
+ * quantized in batches of S_flush, after the new chunk has been appended and attended
+ * in full precision. Reading (the page gives no formula): the flush runs after every
+ * append and quantizes the oldest S_flush eligible positions while at least S_flush are
+ * eligible, so a sequence of L positions has the quantized middle
+ * [S_sink, S_sink + Q) with Q = S_flush * floor(max(0, L - S_sink - S_keep) / S_flush).
+ * Returns Q, or -1 for invalid arguments.
+ */
+int oracle_window_quantized(int L, int S_sink, int S_keep, int S_flush)
+{
+    if (L < 0 || S_sink < 0 || S_keep < 0 || S_flush <= 0)
+        return -1;
+    int e = L - S_sink - S_keep;
+    return e > 0 ? (e / S_flush) * S_flush : 0;
+}
+
+/*
+ * Decode attention of a sequence with a full-precision window. For t < L = seqlens[b]:
+ *   quantized t (S_sink <= t < S_sink + Q):  logit = (1/sqrt(d)) (M q) . khat_t,
+ *                                             value = vhat_t (as oracle_decode);
+ *   full-precision t:                         logit = (1/sqrt(d)) q . k_t,
+ *                                             value = T_v v_t,
+ * k_t, v_t as given (post-RoPE, not transformed; q . k = (M q) . (T_k k) holds exactly
+ * for M = T_k^{-T}, so both kinds of logits are on the same scale), and T_v applied in
+ * float64 so that every value is in the value-transform domain, as the quantized ones
+ * are. out[b][hq] = sum_t p_t value_t / sum_t p_t with p_t = exp(logit_t - max); 0 if
+ * L = 0.
+ *   k, v: [B][T_cap][Hkv][d] in in_dtype (0 float32, 1 bfloat16 bits): the full-precision
+ *         tokens (only window positions are read). Tv: [Hkv][d][d] float32 or NULL = I.
+ *   cache planes: the quantized positions at their own positions.
+ */
+int oracle_window_decode(const void *q, int q_dtype, int B, int Hq, int Hkv, int d,
+                         const float *M, const float *Tv, const void *k, const void *v,
+                         int in_dtype, int T_cap, int bits_k, int bits_v, int group,
+                         const uint8_t *k_codes, const uint16_t *k_sz,
+                         const uint8_t *v_codes, const uint16_t *v_sz,
+                         const int32_t *seqlens, int S_sink, int S_keep, int S_flush,
+                         double *out)
+{
+    if (Hkv <= 0 || Hq % Hkv || d > 1024 || T_cap % 16 || S_sink < 0 || S_keep < 0 ||
+        S_flush <= 0)
+        return -1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > T_cap)
+            return -1;
+    oracle_cache c = {B, Hkv, T_cap, d, bits_k, bits_v, group,
+                      (uint8_t *)k_codes, (uint8_t *)v_codes, (uint16_t *)k_sz, (uint16_t *)v_sz};
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int u = 0; u < B * Hq; ++u) {
+        int b = u / Hq, hq = u % Hq, G = Hq / Hkv, h = hq / G;
+        int L = seqlens[b];
+        int Q = oracle_window_quantized(L, S_sink, S_keep, S_flush);
+        double sm = 1.0 / sqrt((double)d);
+        double qt[1024], qin[1024], o[1024], xv[1024], val[1024];
+        query_transform(q, q_dtype, M, Hq, Hkv, d, b, hq, qt);
+        for (int j = 0; j < d; ++j)
+            qin[j] = load_in(q, q_dtype, ((size_t)b * Hq + hq) * d + j);
+        double *logit = (double *)malloc(sizeof(double) * (L > 0 ? L : 1));
+        double m = -INFINITY;
+        for (int t = 0; t < L; ++t) {
+            int quant = t >= S_sink && t < S_sink + Q;
+            double acc = 0.0;
+            if (quant) {
+                load_token(&c, 0, b, h, t, xv);
+                for (int j = 0; j < d; ++j)
+                    acc += qt[j] * xv[j];
+            } else {
+                for (int j = 0; j < d; ++j)
+                    acc += qin[j] * load_in(k, in_dtype, (((size_t)b * T_cap + t) * Hkv + h) * d + j);
+            }
+            logit[t] = sm * acc;
+            if (logit[t] > m)
+                m = logit[t];
+        }
+        double l = 0.0;
+        for (int j = 0; j < d; ++j)
+            o[j] = 0.0;
+        for (int t = 0; t < L; ++t) {
+            int quant = t >= S_sink && t < S_sink + Q;
+            double p = exp(logit[t] - m);
+            l += p;
+            if (quant) {
+                load_token(&c, 1, b, h, t, val);
+            } else {
+                for (int j = 0; j < d; ++j)
+                    xv[j] = load_in(v, in_dtype, (((size_t)b * T_cap + t) * Hkv + h) * d + j);
+                if (Tv) {
+                    for (int i = 0; i < d; ++i) {
+                        const float *row = Tv + ((size_t)h * d + i) * d;
+                        double a = 0.0;
+                        for (int j = 0; j < d; ++j)
+                            a += (double)row[j] * xv[j];
+                        val[i] = a;
+                    }
+                } else {
+                    memcpy(val, xv, sizeof(double) * d);
+                }
+            }
+            for (int j = 0; j < d; ++j)
+                o[j] += p * val[j];
         }
         for (int j = 0; j < d; ++j)
             out[((size_t)b * Hq + hq) * d + j] = l > 0 ? o[j] / l : 0.0;
