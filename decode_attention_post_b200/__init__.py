@@ -8,6 +8,7 @@ PyTorch supplies device memory and streams only; no step of the path runs here.
 """
 from .kvq import (  # noqa: F401
     KVQ_DEVERR_NONFINITE,
+    KVQ_DEVERR_PAGE_RANGE,
     KVQ_DEVERR_POS_RANGE,
     KVQ_DEVERR_SEQLEN_CLAMPED,
     KVQ_DEVERR_WAIT_TIMEOUT,
@@ -19,6 +20,7 @@ from .kvq import (  # noqa: F401
     cache_plane_bytes,
     decode_attention,
     decode_attention_noalloc,
+    decode_attention_window,
     decode_workspace_bytes,
     library_path,
     load,

@@ -336,11 +336,15 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
             flag(P.dev_err, KVQ_DEVERR_SEQLEN_CLAMPED);
         seqlen = seqlen < 0 ? 0 : P.max_seqlen;
     }
+    const bool windowed = P.win_flush > 0;
+    if (windowed)                               // the cache holds the quantized middle only
+        seqlen = window_quantized(seqlen, P.win_sink, P.win_keep, P.win_flush);
     const int t_begin = sigma * P.split_tokens;
     if (t_begin >= seqlen)
         return;                                 // nothing here (the prologue zeroes empty ones)
     const int t_end = min(t_begin + P.split_tokens, seqlen);
     const int nsplit_b = (seqlen + P.split_tokens - 1) / P.split_tokens;
+    const int nmerge = nsplit_b + (windowed ? 1 : 0);   // partials merged for the pair
     const int nblk = (t_end - t_begin + kDecodeBlock - 1) / kDecodeBlock;
     const int my_nblk = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
 
@@ -641,7 +645,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     __syncthreads();
 
     // ---- merge warps; either finish the output or store this split's partial
-    float *part = P.part + (pair * P.nsplit + sigma) * (size_t)(G * (D + 2));
+    float *part = P.part + (pair * P.part_slots + sigma) * (size_t)(G * (D + 2));
     for (int idx = threadIdx.x; idx < G * D; idx += kDecodeWarps * 32) {
         const int head = idx / D, dim = idx % D;
         float Mx = -INFINITY;
@@ -658,7 +662,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
             L = fmaf(wt, lw[w * G + head], L);
             o = fmaf(wt, ow[(w * G + head) * D + dim], o);
         }
-        if (nsplit_b == 1) {
+        if (nmerge == 1) {
             const size_t oi = ((size_t)b * P.Hq + h * G + head) * D + dim;
             const float r = o / L;
             if (P.out_bf16)
@@ -673,30 +677,35 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
             }
         }
     }
-    if (nsplit_b == 1)
+    if (nmerge == 1)
         return;
-    // ---- the last split of the pair to finish merges all splits. The barrier orders
+    // ---- the last split of the pair to finish merges all splits (and the window's
+    //      partial, counted in the ticket before this kernel started). The barrier orders
     //      every thread's partial stores before thread 0's device-scope fence and ticket;
     //      the merging CTA's thread 0 fences after its ticket and the barrier orders that
     //      before every thread's loads.
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        const int last = (atomicAdd(&P.ticket[pair], 1) == nsplit_b - 1);
+        const int last = (atomicAdd(&P.ticket[pair], 1) == nmerge - 1);
         __threadfence();
         *flag_smem = last;
     }
     __syncthreads();
     if (!*flag_smem)
         return;
-    const float *pall = P.part + pair * P.nsplit * (size_t)(G * (D + 2));
+    const float *pall = P.part + pair * P.part_slots * (size_t)(G * (D + 2));
+    // slots 0 .. nsplit_b-1 hold the splits; the window's partial is in slot P.nsplit
     for (int idx = threadIdx.x; idx < G * D; idx += kDecodeWarps * 32) {
         const int head = idx / D, dim = idx % D;
         float Mx = -INFINITY;
-        for (int sg = 0; sg < nsplit_b; ++sg)
+        for (int i = 0; i < nmerge; ++i) {
+            const int sg = i < nsplit_b ? i : P.nsplit;
             Mx = fmaxf(Mx, __ldcg(pall + (size_t)sg * G * (D + 2) + head * (D + 2)));
+        }
         float L = 0.f, o = 0.f;
-        for (int sg = 0; sg < nsplit_b; ++sg) {
+        for (int i = 0; i < nmerge; ++i) {
+            const int sg = i < nsplit_b ? i : P.nsplit;
             const float *pp = pall + (size_t)sg * G * (D + 2) + head * (D + 2);
             const float wt = ex2(__ldcg(pp) - Mx);
             L = fmaf(wt, __ldcg(pp + 1), L);
@@ -748,6 +757,12 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
             L.p.out, L.p.out_bf16, const_cast<uint32_t *>(L.p.qfrag),
             const_cast<float *>(L.p.qscale), const_cast<float *>(L.p.qw), L.p.ticket);
         e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    }
+    // full-precision window: its partial and ticket count before the decode's merges
+    if (L.win) {
+        e = launch_window(*L.win, st);
         if (e != cudaSuccess)
             return e;
     }

@@ -32,10 +32,34 @@ struct DecodeParams {
     const int32_t *block_table; // paged cache: [B][T_cap/page_tokens]; nullptr = contiguous
     int page_tokens;
     int num_pages;
+    int part_slots;             // partial slots per (sequence, KV head): nsplit + 1
+    // full-precision window (win_flush = 0: none): the cache holds the quantized middle,
+    // seqlens are whole lengths, slot `nsplit` holds the window's partial
+    int win_sink, win_keep, win_flush;
 };
+
+// The window's attention: one CTA per (KV head, sequence) over the full-precision
+// positions, written as the extra partial of the pair (or as the output when nothing of
+// the sequence is quantized).
+struct WindowParams {
+    const void *q;              // bfloat16 [B][Hq][d]
+    const void *k_sink, *v_sink, *k_recent, *v_recent;
+    const float *T_v;
+    const int32_t *seqlens;
+    int B, Hkv, Hq, d, max_seqlen;
+    int S_sink, S_keep, S_flush;
+    float *part;
+    int part_slots, slot;
+    int *ticket;
+    void *out;
+    int out_bf16;
+};
+
+struct WindowParams;
 
 struct DecodeLaunch {
     DecodeParams p;
+    const WindowParams *win;    // full-precision window, launched between qprep and decode
     const void *q;
     int q_bf16;
     const float *M;
@@ -49,5 +73,13 @@ struct DecodeWorkspace {
 
 size_t decode_qfrag_words(int d, int G);
 cudaError_t launch_decode(const DecodeLaunch &L, cudaStream_t st);
+cudaError_t launch_window(const WindowParams &W, cudaStream_t st);
+
+// Quantized middle length of a sequence of L positions with a full-precision window.
+__host__ __device__ inline int window_quantized(int L, int S_sink, int S_keep, int S_flush)
+{
+    const int e = L - S_sink - S_keep;
+    return e > 0 ? (e / S_flush) * S_flush : 0;
+}
 
 }  // namespace kvq

@@ -141,8 +141,8 @@ static DecodeWorkspace decode_layout(int B, int Hkv, int Hq, int d, int nsplit)
     off += up256((size_t)B * Hq * 4);
     w.qw = off;
     off += up256((size_t)B * Hq * 4);
-    w.part = off;
-    off += up256((size_t)B * Hkv * nsplit * G * (d + 2) * 4);
+    w.part = off;                              // nsplit split slots + 1 window slot
+    off += up256((size_t)B * Hkv * (nsplit + 1) * G * (d + 2) * 4);
     w.ticket = off;
     off += up256((size_t)B * Hkv * 4);
     w.total = off;
@@ -250,13 +250,16 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *c, int Hq, int max_seqlen)
     return decode_layout(c->B, c->Hkv, Hq, c->d, ns).total;
 }
 
-kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const float *Tk_invT,
+// Shared by the plain and the windowed decode: argument checks beyond the cache shape,
+// workspace carving and launch. `win` (nullable) describes the full-precision window and
+// `qmax` is the longest quantized run the cache holds for max_seqlen.
+static kvq_status decode_common(const void *q, kvq_dtype q_dtype, int Hq, const float *Tk_invT,
                                 const kvq_cache *c, const int32_t *seqlens, int max_seqlen,
-                                void *out, kvq_dtype out_dtype, void *workspace, size_t ws_bytes,
-                                int32_t *dev_err, kvq_stream_t stream)
+                                int qmax, void *out, kvq_dtype out_dtype, void *workspace,
+                                size_t ws_bytes, int32_t *dev_err, kvq_stream_t stream,
+                                const kvq_window *win)
 {
-    g_last_error[0] = 0;
-    kvq_status s = check_decode_shape(c, Hq, max_seqlen);
+    kvq_status s = check_decode_shape(c, Hq, qmax);
     if (s != KVQ_OK)
         return s;
     if (!q || !seqlens || !out)
@@ -265,7 +268,7 @@ kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const 
         (out_dtype != KVQ_F32 && out_dtype != KVQ_BF16))
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "q_dtype/out_dtype must be KVQ_F32 or KVQ_BF16");
     int split_tokens = 0;
-    const int ns = choose_splits(c->B, c->Hkv, max_seqlen, &split_tokens);
+    const int ns = choose_splits(c->B, c->Hkv, qmax, &split_tokens);
     const DecodeWorkspace w = decode_layout(c->B, c->Hkv, Hq, c->d, ns);
     if (!workspace || !aligned(workspace, 256))
         KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
@@ -296,6 +299,10 @@ kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const 
     L.p.block_table = c->block_table;
     L.p.page_tokens = c->page_tokens;
     L.p.num_pages = c->num_pages;
+    L.p.part_slots = ns + 1;
+    L.p.win_sink = win ? win->S_sink : 0;
+    L.p.win_keep = win ? win->S_keep : 0;
+    L.p.win_flush = win ? win->S_flush : 0;
     L.q = q;
     L.q_bf16 = q_dtype == KVQ_BF16;
     L.M = Tk_invT;
@@ -303,10 +310,73 @@ kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const 
     L.G = Hq / c->Hkv;
     L.bits_k = c->qp.bits_k;
     L.bits_v = c->qp.bits_v;
+    WindowParams W;
+    L.win = nullptr;
+    if (win) {
+        W.q = q;
+        W.k_sink = win->k_sink;
+        W.v_sink = win->v_sink;
+        W.k_recent = win->k_recent;
+        W.v_recent = win->v_recent;
+        W.T_v = win->T_v;
+        W.seqlens = seqlens;
+        W.B = c->B;
+        W.Hkv = c->Hkv;
+        W.Hq = Hq;
+        W.d = c->d;
+        W.max_seqlen = max_seqlen;
+        W.S_sink = win->S_sink;
+        W.S_keep = win->S_keep;
+        W.S_flush = win->S_flush;
+        W.part = L.p.part;
+        W.part_slots = L.p.part_slots;
+        W.slot = ns;
+        W.ticket = L.p.ticket;
+        W.out = out;
+        W.out_bf16 = L.p.out_bf16;
+        L.win = &W;
+    }
     cudaError_t e = launch_decode(L, (cudaStream_t)stream);
     if (e != cudaSuccess)
         KVQ_FAIL(KVQ_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const float *Tk_invT,
+                                const kvq_cache *c, const int32_t *seqlens, int max_seqlen,
+                                void *out, kvq_dtype out_dtype, void *workspace, size_t ws_bytes,
+                                int32_t *dev_err, kvq_stream_t stream)
+{
+    g_last_error[0] = 0;
+    return decode_common(q, q_dtype, Hq, Tk_invT, c, seqlens, max_seqlen, max_seqlen, out,
+                         out_dtype, workspace, ws_bytes, dev_err, stream, nullptr);
+}
+
+kvq_status kvq_decode_attention_window(const void *q, kvq_dtype q_dtype, int Hq,
+                                       const float *Tk_invT, const kvq_cache *c,
+                                       const kvq_window *win, const int32_t *seqlens,
+                                       int max_seqlen, void *out, kvq_dtype out_dtype,
+                                       void *workspace, size_t ws_bytes, int32_t *dev_err,
+                                       kvq_stream_t stream)
+{
+    g_last_error[0] = 0;
+    if (!win)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "window is NULL");
+    if (win->S_sink < 0 || win->S_keep < 0 || win->S_flush <= 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "window S_sink=%d S_keep=%d S_flush=%d: need >= 0, >= 0, > 0",
+                 win->S_sink, win->S_keep, win->S_flush);
+    if ((long)win->S_sink + win->S_keep + win->S_flush > 2048)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "window of %ld positions: at most 2048 are implemented",
+                 (long)win->S_sink + win->S_keep + win->S_flush);
+    if ((win->S_sink > 0 && (!win->k_sink || !win->v_sink)) || !win->k_recent || !win->v_recent)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "a window buffer is NULL");
+    if (q_dtype != KVQ_BF16)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "the windowed decode takes bfloat16 queries");
+    if (max_seqlen < 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "max_seqlen=%d must be >= 0", max_seqlen);
+    const int qmax = window_quantized(max_seqlen, win->S_sink, win->S_keep, win->S_flush);
+    return decode_common(q, q_dtype, Hq, Tk_invT, c, seqlens, max_seqlen, qmax, out, out_dtype,
+                         workspace, ws_bytes, dev_err, stream, win);
 }
 
 size_t kvq_bf16_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seqlen)

@@ -1,0 +1,185 @@
+// Full-precision window of the read path ("WUSH-KV: KV Cache Quantization with
+// Data-Adaptive Transforms", section 4.4): attention over the positions a sequence keeps
+// in full precision -- the first S_sink positions and those after the quantized middle --
+// as one more partial (running max, sum of weights, weighted sum of values) next to the
+// splits of the quantized middle, merged by the decode kernel's last split.
+//
+// One CTA per (KV head, sequence), 128 threads, for the G query heads of the KV head:
+//   logit_t = log2(e)/sqrt(d) * q . k_t  (the query as given: q . k = (T_k^{-T} q) . (T_k k)),
+//   m = max_t logit_t, p_t = 2^(logit_t - m), l = sum_t p_t, o = T_v sum_t p_t v_t,
+// in float32 on CUDA cores (the window is a few hundred positions at most), T_v applied
+// so that o is in the value-transform domain like the quantized values. The logits are in
+// log2 units, as the decode kernel's partials. When nothing of the sequence is quantized
+// the partial is the whole attention and o / l is written as the output.
+#include "kvq_common.cuh"
+#include "kvq_ptx.cuh"
+#include "decode_shapes.h"
+
+#include <math.h>
+
+namespace kvq {
+
+namespace {
+
+constexpr int kWinThreads = 128;
+constexpr float kWinLog2e = 1.4426950408889634f;
+
+template <int D, int G>
+__global__ void __launch_bounds__(kWinThreads) window_kernel(WindowParams W)
+{
+    extern __shared__ __align__(16) float wsm[];
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int R = W.S_keep + W.S_flush;                 // recent ring slots
+    const int WMAX = W.S_sink + R;                      // window positions at most
+    float *qf = wsm;                                    // [G][D]
+    float *of = qf + G * D;                             // [G][D]
+    float *stat = of + G * D;                           // [G][2]: m, l
+    float *lg = stat + 2 * G;                           // [G][WMAX]: logits, then weights
+
+    int L = W.seqlens[b];
+    L = L < 0 ? 0 : (L > W.max_seqlen ? W.max_seqlen : L);
+    if (L == 0)
+        return;                                         // the q prologue wrote zeros
+    const int Q = window_quantized(L, W.S_sink, W.S_keep, W.S_flush);
+    const int nsink = min(W.S_sink, L);
+    const int rec0 = W.S_sink + Q;                      // first recent position
+    const int nrec = L > rec0 ? L - rec0 : 0;
+    const int nw = nsink + nrec;
+    const size_t pair = (size_t)b * W.Hkv + h;
+    const float sc = kWinLog2e * rsqrtf((float)D);
+
+    // row of window position w (w < nsink: sink, else recent ring slot)
+    auto k_row = [&](int w) -> const __nv_bfloat16 * {
+        if (w < nsink)
+            return reinterpret_cast<const __nv_bfloat16 *>(W.k_sink) +
+                   (pair * W.S_sink + w) * D;
+        const int t = rec0 + (w - nsink);
+        return reinterpret_cast<const __nv_bfloat16 *>(W.k_recent) + (pair * R + t % R) * D;
+    };
+    auto v_row = [&](int w) -> const __nv_bfloat16 * {
+        if (w < nsink)
+            return reinterpret_cast<const __nv_bfloat16 *>(W.v_sink) +
+                   (pair * W.S_sink + w) * D;
+        const int t = rec0 + (w - nsink);
+        return reinterpret_cast<const __nv_bfloat16 *>(W.v_recent) + (pair * R + t % R) * D;
+    };
+
+    for (int idx = tid; idx < G * D; idx += kWinThreads)
+        qf[idx] = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(
+            W.q)[((size_t)b * W.Hq + h * G + idx / D) * D + idx % D]);
+    __syncthreads();
+    // ---- logits: thread per (head, position)
+    for (int idx = tid; idx < G * nw; idx += kWinThreads) {
+        const int head = idx / nw, w = idx % nw;
+        const __nv_bfloat16 *kr = k_row(w);
+        const float *qh = qf + head * D;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < D; ++j)
+            acc = fmaf(qh[j], __bfloat162float(kr[j]), acc);
+        lg[head * WMAX + w] = sc * acc;
+    }
+    __syncthreads();
+    // ---- per head: max, weights 2^(logit - m), their sum
+    for (int head = warp; head < G; head += kWinThreads / 32) {
+        float m = -INFINITY;
+        for (int w = lane; w < nw; w += 32)
+            m = fmaxf(m, lg[head * WMAX + w]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float l = 0.f;
+        for (int w = lane; w < nw; w += 32) {
+            const float p = ex2(lg[head * WMAX + w] - m);
+            lg[head * WMAX + w] = p;
+            l += p;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            l += __shfl_xor_sync(0xffffffffu, l, off);
+        if (lane == 0) {
+            stat[2 * head] = m;
+            stat[2 * head + 1] = l;
+        }
+    }
+    __syncthreads();
+    // ---- sum_t p_t v_t (untransformed values): thread per (head, dim)
+    for (int idx = tid; idx < G * D; idx += kWinThreads) {
+        const int head = idx / D, j = idx % D;
+        float acc = 0.f;
+        for (int w = 0; w < nw; ++w)
+            acc = fmaf(lg[head * WMAX + w], __bfloat162float(v_row(w)[j]), acc);
+        of[idx] = acc;
+    }
+    __syncthreads();
+    // ---- o = T_v (sum p v), then the partial (or the output)
+    const float *Tv = W.T_v ? W.T_v + (size_t)h * D * D : nullptr;
+    float *part = W.part + (pair * W.part_slots + W.slot) * (size_t)(G * (D + 2));
+    for (int idx = tid; idx < G * D; idx += kWinThreads) {
+        const int head = idx / D, i = idx % D;
+        float o = of[idx];
+        if (Tv) {
+            const float *row = Tv + (size_t)i * D;
+            const float *oh = of + head * D;
+            float acc = 0.f;
+#pragma unroll 8
+            for (int j = 0; j < D; ++j)
+                acc = fmaf(row[j], oh[j], acc);
+            o = acc;
+        }
+        if (Q == 0) {
+            const size_t oi = ((size_t)b * W.Hq + h * G + head) * D + i;
+            const float r = o / stat[2 * head + 1];
+            if (W.out_bf16)
+                reinterpret_cast<__nv_bfloat16 *>(W.out)[oi] = __float2bfloat16_rn(r);
+            else
+                reinterpret_cast<float *>(W.out)[oi] = r;
+        } else {
+            part[head * (D + 2) + 2 + i] = o;
+            if (i == 0) {
+                part[head * (D + 2)] = stat[2 * head];
+                part[head * (D + 2) + 1] = stat[2 * head + 1];
+            }
+        }
+    }
+    if (Q > 0) {
+        // count this partial in the pair's ticket: the decode kernel's last split merges it
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(&W.ticket[pair], 1);
+        }
+    }
+}
+
+template <int D, int G>
+cudaError_t launch_window_t(const WindowParams &W, cudaStream_t st)
+{
+    const int WMAX = W.S_sink + W.S_keep + W.S_flush;
+    const size_t smem = (size_t)(2 * G * D + 2 * G + G * WMAX) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(window_kernel<D, G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    window_kernel<D, G><<<dim3(W.Hkv, W.B), kWinThreads, smem, st>>>(W);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_window(const WindowParams &W, cudaStream_t st)
+{
+    const int G = W.Hq / W.Hkv;
+    if (W.d == 128 && G == 4)
+        return launch_window_t<128, 4>(W, st);
+    if (W.d == 128 && G == 8)
+        return launch_window_t<128, 8>(W, st);
+    if (W.d == 64 && G == 4)
+        return launch_window_t<64, 4>(W, st);
+    if (W.d == 64 && G == 8)
+        return launch_window_t<64, 8>(W, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kvq

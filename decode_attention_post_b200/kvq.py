@@ -23,6 +23,7 @@ KVQ_DEVERR_SEQLEN_CLAMPED = 0x1
 KVQ_DEVERR_POS_RANGE = 0x2
 KVQ_DEVERR_NONFINITE = 0x4
 KVQ_DEVERR_WAIT_TIMEOUT = 0x8
+KVQ_DEVERR_PAGE_RANGE = 0x10
 
 _P, _I, _F, _S = C.c_void_p, C.c_int, C.c_float, C.c_size_t
 
@@ -35,6 +36,11 @@ class _Cache(C.Structure):
     _fields_ = [("B", _I), ("Hkv", _I), ("T_cap", _I), ("d", _I), ("qp", _QParams),
                 ("k_codes", _P), ("k_sz", _P), ("v_codes", _P), ("v_sz", _P),
                 ("block_table", _P), ("page_tokens", _I), ("num_pages", _I)]
+
+
+class _Window(C.Structure):
+    _fields_ = [("S_sink", _I), ("S_keep", _I), ("S_flush", _I), ("k_sink", _P),
+                ("v_sink", _P), ("k_recent", _P), ("v_recent", _P), ("T_v", _P)]
 
 
 class KvqError(RuntimeError):
@@ -70,6 +76,10 @@ def load():
     L.kvq_decode_attention.argtypes = [_P, _I, _I, _P, C.POINTER(_Cache), _P, _I, _P, _I, _P, _S,
                                        _P, _P]
     L.kvq_decode_attention_noalloc.restype = _I
+    L.kvq_decode_attention_window.argtypes = [_P, _I, _I, _P, C.POINTER(_Cache),
+                                              C.POINTER(_Window), _P, _I, _P, _I, _P, _S,
+                                              _P, _P]
+    L.kvq_decode_attention_window.restype = _I
     L.kvq_decode_attention_noalloc.argtypes = [_P, _I, _I, _P, C.POINTER(_Cache), _P, _I, _P,
                                                _I, _P, _P]
     L.kvq_bf16_decode_workspace_bytes.restype = _S
@@ -242,6 +252,34 @@ def decode_attention(q, Tk_invT, cache: KVCache, seqlens, max_seqlen: int, out, 
                                   _ptr(seqlens), int(max_seqlen), _ptr(out), _dt(out),
                                   _ptr(workspace), workspace.numel(), _ptr(dev_err),
                                   _stream(stream)), "kvq_decode_attention")
+
+
+def decode_attention_window(q, Tk_invT, cache: KVCache, S_sink: int, S_keep: int,
+                            S_flush: int, k_sink, v_sink, k_recent, v_recent, T_v, seqlens,
+                            max_seqlen: int, out, workspace, dev_err=None, stream=None):
+    """kvq_decode_attention_window: decode with a full-precision window. q bfloat16
+    [B][Hq][d]; k_sink, v_sink bfloat16 [B][Hkv][S_sink][d] (None when S_sink = 0);
+    k_recent, v_recent bfloat16 [B][Hkv][S_keep + S_flush][d] (position t at slot
+    t % (S_keep + S_flush)); T_v float32 [Hkv][d][d] or None; seqlens int32 [B] whole
+    lengths; the cache holds the quantized middle from its position 0."""
+    L = load()
+    _cuda("q", q)
+    _cuda("Tk_invT", Tk_invT, torch.float32)
+    for name, t in (("k_sink", k_sink), ("v_sink", v_sink), ("k_recent", k_recent),
+                    ("v_recent", v_recent)):
+        _cuda(name, t, torch.bfloat16)
+    _cuda("T_v", T_v, torch.float32)
+    _cuda("seqlens", seqlens, torch.int32)
+    _cuda("out", out)
+    _cuda("workspace", workspace, torch.uint8)
+    _cuda("dev_err", dev_err, torch.int32)
+    win = _Window(int(S_sink), int(S_keep), int(S_flush), _ptr(k_sink), _ptr(v_sink),
+                  _ptr(k_recent), _ptr(v_recent), _ptr(T_v))
+    _check(L.kvq_decode_attention_window(_ptr(q), _dt(q), int(q.shape[1]), _ptr(Tk_invT),
+                                         C.byref(cache.desc), C.byref(win), _ptr(seqlens),
+                                         int(max_seqlen), _ptr(out), _dt(out), _ptr(workspace),
+                                         workspace.numel(), _ptr(dev_err), _stream(stream)),
+           "kvq_decode_attention_window")
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20

@@ -192,6 +192,48 @@ KVQ_API kvq_status kvq_bf16_decode(const void *q, int Hq, const void *k, const v
                            kvq_stream_t stream);
 
 /*
+ * Full-precision window (WUSH-KV summary, section 4.4): the first S_sink positions and
+ * the newest S_keep positions of a sequence stay in full precision; the positions between
+ * are quantized in batches of S_flush. With L positions the quantized middle is
+ * [S_sink, S_sink + Q), Q = S_flush * floor(max(0, L - S_sink - S_keep) / S_flush)
+ * (the flush runs after every append). The caller keeps:
+ *   k_sink, v_sink:     bfloat16 [B][Hkv][S_sink][d], positions 0..S_sink-1 as given;
+ *   k_recent, v_recent: bfloat16 [B][Hkv][S_keep + S_flush][d], position t >= S_sink + Q
+ *                       at slot t % (S_keep + S_flush), as given (post-RoPE keys);
+ *   the quantized cache holding position S_sink + i at cache position i (i < Q), written
+ *   by kvq_quantize_append when a batch is flushed.
+ * T_v: [Hkv][d][d] float32 (NULL = identity), applied to the full-precision values so
+ * that the whole output is in the value-transform domain.
+ */
+typedef struct {
+    int S_sink;
+    int S_keep;
+    int S_flush;                /* > 0 */
+    const void *k_sink;
+    const void *v_sink;
+    const void *k_recent;
+    const void *v_recent;
+    const float *T_v;
+} kvq_window;
+
+/*
+ * Decode with a full-precision window: seqlens[b] = L (all positions of sequence b,
+ * L <= max_seqlen); full-precision positions attend with the query as given (q . k,
+ * = (T_k^{-T} q) . (T_k k)), quantized ones as in kvq_decode_attention; one softmax over
+ * all L positions. q must be bfloat16. The quantized middle of max_seqlen positions must
+ * fit the cache (Q(max_seqlen) <= T_cap); S_sink + S_keep + S_flush <= 2048. Workspace:
+ * kvq_decode_workspace_bytes(cache, Hq, m) for any m >= Q(max_seqlen) (m = T_cap always
+ * suffices). Other arguments and errors as in kvq_decode_attention.
+ */
+KVQ_API kvq_status kvq_decode_attention_window(const void *q, kvq_dtype q_dtype, int Hq,
+                                               const float *Tk_invT, const kvq_cache *cache,
+                                               const kvq_window *window,
+                                               const int32_t *seqlens, int max_seqlen,
+                                               void *out, kvq_dtype out_dtype, void *workspace,
+                                               size_t ws_bytes, int32_t *dev_err,
+                                               kvq_stream_t stream);
+
+/*
  * Allocation-free decode (no counterpart in the paper; an addition for callers that
  * cannot allocate device memory). Same arguments and result as kvq_decode_attention
  * minus the workspace: an inference engine that has reserved nearly all device memory

@@ -587,3 +587,73 @@ def test_paged_out_of_range_page_is_flagged():
     k, v = _inputs(cfg, 2, 1, "bf16")
     _, err = gpu_append(cfg, k, v, None, None, [0, 70], cache=gc)   # 70 -> page entry [1][1]
     assert err & 0x10
+
+
+# ----------------------------------------------------------------------------- full-precision window
+
+
+def _round64(x):
+    return max(64, (x + 63) // 64 * 64)
+
+
+@pytest.mark.parametrize("ci,S_sink,S_keep,S_flush,seql", [
+    (2, 4, 32, 64, [300, 20, 97]),        # quantized middles; one sequence entirely in the window
+    (2, 0, 0, 64, [256, 128, 64]),        # no window: every position quantized
+    (2, 64, 128, 128, [700, 300, 0]),     # an empty sequence
+    (4, 8, 64, 64, [500, 71]),            # GQA 8, d 64
+])
+def test_window_decode_matches_oracle(ci, S_sink, S_keep, S_flush, seql):
+    cfg = synth.CONFIGS[ci]
+    B, T = len(seql), _round64(max(seql))
+    c = cfg.with_(B=B, T_cap=T)
+    k, v = synth.kv_batch(c, 0, T)                       # [B][T][Hkv][d] float32
+    kb, vb = synth.as_dtype(k, "bf16"), synth.as_dtype(v, "bf16")
+    Tk, Tv, Tit = synth.transforms(cfg)
+    q = synth.as_dtype(synth.queries(c), "bf16")
+    # oracle: every position quantized at its own position; the window decode reads the
+    # middle from there and the rest in full precision
+    ofull = oracle.Cache(B, cfg.Hkv, T, cfg.d, cfg.bits_k, cfg.bits_v, cfg.group)
+    oracle.quantize_append(kb, vb, Tk, Tv, cfg.bits_k, cfg.bits_v, cfg.group, cfg.clip_alpha,
+                           ofull, np.zeros(B, np.int32))
+    want = oracle.window_decode(q, Tit, Tv, kb, vb, ofull, np.array(seql, np.int32), S_sink,
+                                S_keep, S_flush)
+    # GPU: the quantized middle of each sequence from cache position 0 (the oracle's codes
+    # for the same tokens), sink and recent ring in bfloat16
+    Qs = [oracle.window_quantized(L, S_sink, S_keep, S_flush) for L in seql]
+    Tc = _round64(max(Qs))
+    oc = oracle.Cache(B, cfg.Hkv, Tc, cfg.d, cfg.bits_k, cfg.bits_v, cfg.group)
+    for b, Qb in enumerate(Qs):
+        if Qb == 0:
+            continue
+        one = oracle.Cache(1, cfg.Hkv, Tc, cfg.d, cfg.bits_k, cfg.bits_v, cfg.group)
+        oracle.quantize_append(np.ascontiguousarray(kb[b:b + 1, S_sink:S_sink + Qb]),
+                               np.ascontiguousarray(vb[b:b + 1, S_sink:S_sink + Qb]), Tk, Tv,
+                               cfg.bits_k, cfg.bits_v, cfg.group, cfg.clip_alpha, one, [0])
+        for dst, src in zip(oc.planes(), one.planes()):
+            n = src.size
+            dst[b * n:(b + 1) * n] = src
+    gc = upload_cache(oc, cfg)
+    R = S_keep + S_flush
+    ks = np.zeros((B, cfg.Hkv, max(S_sink, 1), cfg.d), np.uint16)
+    vs = np.zeros_like(ks)
+    kr = np.zeros((B, cfg.Hkv, R, cfg.d), np.uint16)
+    vr = np.zeros_like(kr)
+    for b, L in enumerate(seql):
+        for t in range(min(S_sink, L)):
+            ks[b, :, t], vs[b, :, t] = kb[b, t], vb[b, t]
+        for t in range(S_sink + Qs[b], L):
+            kr[b, :, t % R], vr[b, :, t % R] = kb[b, t], vb[b, t]
+    out = torch.empty((B, cfg.Hq, cfg.d), dtype=torch.float32, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ws = torch.empty(kvq.decode_workspace_bytes(gc, cfg.Hq, Tc), dtype=torch.uint8, device=DEV)
+    kvq.decode_attention_window(t_(q), t_(Tit), gc, S_sink, S_keep, S_flush,
+                                t_(ks) if S_sink else None, t_(vs) if S_sink else None,
+                                t_(kr), t_(vr), t_(Tv), t_(np.array(seql, np.int32)),
+                                max(seql), out, ws, dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = out.cpu().numpy()
+    for b, L in enumerate(seql):
+        if L == 0:
+            assert not got[b].any()
+    assert_close(got, want, where=f"window {S_sink}/{S_keep}/{S_flush}")
