@@ -147,6 +147,47 @@ def test_decode_argument_errors():
     assert _decode(d2) == 2                    # decode implements group == d
 
 
+def _window_decode(desc, win, Hq=8, max_seqlen=64, qd=1, ws_bytes=1 << 30):
+    L = kvq.load()
+    return L.kvq_decode_attention_window(0x5000, qd, Hq, None, C.byref(desc),
+                                         None if win is None else C.byref(win), 0x7000,
+                                         max_seqlen, 0x6000, 1, 0x4000, ws_bytes, None, None)
+
+
+def _win(S_sink=4, S_keep=32, S_flush=64, ks=0x9000, vs=0x9000, kr=0xA000, vr=0xA000):
+    return K._Window(S_sink, S_keep, S_flush, ks, vs, kr, vr, None)
+
+
+def test_window_decode_argument_errors():
+    desc, _ = _desc(T_cap=128)
+    assert _window_decode(desc, None) == 1                        # no window
+    assert _window_decode(desc, _win(S_flush=0)) == 1
+    assert _window_decode(desc, _win(S_sink=-1)) == 1
+    assert _window_decode(desc, _win(S_keep=-2)) == 1
+    assert _window_decode(desc, _win(S_sink=1024, S_keep=1024, S_flush=64)) == 2   # > 2048
+    assert _window_decode(desc, _win(ks=0)) == 1                  # sink buffer missing
+    assert _window_decode(desc, _win(kr=0)) == 1                  # recent buffer missing
+    assert _window_decode(desc, _win(), qd=0) == 2                # float32 queries
+    # the quantized middle of max_seqlen must fit the cache: 4 + 32 + 128 fits, + 64 not
+    assert _window_decode(desc, _win(), max_seqlen=4 + 32 + 192 + 63) == 3
+    assert _window_decode(desc, _win(), ws_bytes=16) == 4
+    assert kvq.load().kvq_last_error()
+
+
+def test_window_quantized_middle_matches_the_oracle_reading():
+    import oracle
+    # the library's host-side reading (through the capacity check) equals the oracle's:
+    # max_seqlen whose middle is exactly T_cap passes the shape checks, one batch more fails
+    desc, _ = _desc(T_cap=128)
+    for S_sink, S_keep, S_flush in [(4, 32, 64), (0, 0, 64), (64, 128, 128), (3, 5, 16)]:
+        win = _win(S_sink, S_keep, S_flush)
+        L_ok = S_sink + S_keep + 128 + S_flush - 1
+        assert oracle.window_quantized(L_ok, S_sink, S_keep, S_flush) == 128
+        assert _window_decode(desc, win, max_seqlen=L_ok, ws_bytes=16) == 4   # shape ok
+        assert oracle.window_quantized(L_ok + 1, S_sink, S_keep, S_flush) > 128
+        assert _window_decode(desc, win, max_seqlen=L_ok + 1, ws_bytes=16) == 3
+
+
 def test_workspace_sizes_positive_and_monotone():
     L = kvq.load()
     desc, _ = _desc(B=4, Hkv=8, T_cap=16384)
