@@ -50,7 +50,6 @@ struct Cfg {
     static constexpr int KS = (8 / BK) * KCH;        // int8 k-steps of the Q.K contraction
     static constexpr int MT = D / 16;                // m-tiles (output dims) of P.V
     static constexpr int NT = (2 * G) / 8;           // n-tiles of (hi, lo) x G columns
-    static constexpr int COLS = 2 * G;
     static constexpr int ROWK = D * BK / 8;          // bytes per K row (token)
     static constexpr int WPT = D * BK / 128;         // K words per thread per token
     static constexpr int CPBK = 8 / BK;              // code fields per byte (K)
@@ -66,7 +65,9 @@ struct Cfg {
     static constexpr int QFRAG = NT * KS * 32 * 2;
     static constexpr int RING = kDecodeWarps * kDecodeStages * STAGE;
     static constexpr int MERGE = kDecodeWarps * G * (D + 2) * 4;
-    static constexpr int SMEM = (RING > MERGE ? RING : MERGE) + kDecodeWarps * kDecodeStages * 8 + 16;
+    // ring (or merge area), stage barriers, one test-hook barrier per warp, merge flag
+    static constexpr int SMEM =
+        (RING > MERGE ? RING : MERGE) + kDecodeWarps * (kDecodeStages + 1) * 8 + 16;
     // resident CTAs per SM the register budget targets: kDecodeMinBlocks, or fewer when
     // shared memory (227 KB per SM, 1 KB reserved per CTA) holds fewer
     static constexpr int SMEM_FIT = (227 * 1024) / (SMEM + 1024);
@@ -314,7 +315,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     unsigned char *ring = smem_raw;
     uint64_t *bars_all =
         reinterpret_cast<uint64_t *>(smem_raw + (C::RING > C::MERGE ? C::RING : C::MERGE));
-    int *flag_smem = reinterpret_cast<int *>(bars_all + kDecodeWarps * kDecodeStages);
+    uint64_t *stall_bars = bars_all + kDecodeWarps * kDecodeStages;
+    int *flag_smem = reinterpret_cast<int *>(stall_bars + kDecodeWarps);
 
     const int h = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
     const int lane = threadIdx.x & 31;
@@ -356,6 +358,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     if (lane == 0) {
         for (int s = 0; s < kDecodeStages; ++s)
             mbar_init(&bars[s], 1);
+        mbar_init(&stall_bars[warp], 1);
         mbar_fence_init();
     }
     __syncwarp();
@@ -429,6 +432,16 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
                 O[m][nt][i] = 0.f;
     }
     bool timed_out = false;
+    if (P.stall_test_ns > 0 && my_nblk > 0) {
+        // failure-path test hook: a bounded wait on a barrier that nothing arrives at; on
+        // giving up, the same path as a real timeout -- wait (bounded, normal limit) for
+        // this warp's copies in flight, skip the blocks, flag the error
+        if (!mbar_wait_bounded(&stall_bars[warp], 0, (uint64_t)P.stall_test_ns)) {
+            timed_out = true;
+            for (int k2 = 0; k2 < kDecodeStages && k2 < my_nblk; ++k2)
+                mbar_wait_bounded(&bars[k2], 0);
+        }
+    }
 
     // One 64-token block. FULL: every token is below t_end (no per-token masking).
     auto block = [&](const unsigned char *st, int tok0, auto full_tag) {
@@ -584,7 +597,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
         __syncwarp();
     };
 
-    for (int jj = 0; jj < my_nblk; ++jj) {
+    for (int jj = 0; !timed_out && jj < my_nblk; ++jj) {
         const int s = jj % kDecodeStages;
         if (!mbar_wait_bounded(&bars[s], (jj / kDecodeStages) & 1)) {
             timed_out = true;
@@ -617,8 +630,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
         }
 
     __syncthreads();                             // all warps are done with the ring
-    for (int s = 0; s < kDecodeStages && lane == 0; ++s)
-        mbar_inval(&bars[s]);
+    if (lane == 0) {
+        for (int s = 0; s < kDecodeStages; ++s)
+            mbar_inval(&bars[s]);
+        mbar_inval(&stall_bars[warp]);
+    }
     float *mw = reinterpret_cast<float *>(ring);                 // [W][G]
     float *lw = mw + kDecodeWarps * G;                           // [W][G]
     float *ow = lw + kDecodeWarps * G;                           // [W][G][D]
@@ -695,17 +711,17 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     if (!*flag_smem)
         return;
     const float *pall = P.part + pair * P.part_slots * (size_t)(G * (D + 2));
-    // slots 0 .. nsplit_b-1 hold the splits; the window's partial is in slot P.nsplit
+    // slots 0 .. nsplit_b-1 hold the splits; the window's partial is in the last slot
     for (int idx = threadIdx.x; idx < G * D; idx += kDecodeWarps * 32) {
         const int head = idx / D, dim = idx % D;
         float Mx = -INFINITY;
         for (int i = 0; i < nmerge; ++i) {
-            const int sg = i < nsplit_b ? i : P.nsplit;
+            const int sg = i < nsplit_b ? i : P.part_slots - 1;
             Mx = fmaxf(Mx, __ldcg(pall + (size_t)sg * G * (D + 2) + head * (D + 2)));
         }
         float L = 0.f, o = 0.f;
         for (int i = 0; i < nmerge; ++i) {
-            const int sg = i < nsplit_b ? i : P.nsplit;
+            const int sg = i < nsplit_b ? i : P.part_slots - 1;
             const float *pp = pall + (size_t)sg * G * (D + 2) + head * (D + 2);
             const float wt = ex2(__ldcg(pp) - Mx);
             L = fmaf(wt, __ldcg(pp + 1), L);
@@ -718,23 +734,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
         else
             reinterpret_cast<float *>(P.out)[oi] = r;
     }
-}
-
-// cudaFuncSetAttribute applies to the current device: remember it per device.
-template <typename F>
-cudaError_t ensure_dynamic_smem(F *func, int bytes, unsigned long long &done_mask)
-{
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (done_mask & bit)
-        return cudaSuccess;
-    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess)
-        done_mask |= bit;
-    return e;
 }
 
 template <int D, int G, int BK, int BV>
@@ -767,7 +766,9 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
             return e;
     }
     // decode: CTA (KV head, sequence, split), splits slowest so that the short last
-    // splits of the sequences run last; a programmatic dependent of the prologue
+    // splits of the sequences run last; a programmatic dependent of the kernel launched
+    // just before it (qprep, or the window kernel, which never triggers its dependents
+    // early, so its partial and ticket are complete before this grid's wait returns)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(L.p.Hkv, L.p.B, L.p.nsplit);
     cfg.blockDim = dim3(kDecodeWarps * 32);

@@ -32,10 +32,14 @@ struct DecodeParams {
     const int32_t *block_table; // paged cache: [B][T_cap/page_tokens]; nullptr = contiguous
     int page_tokens;
     int num_pages;
-    int part_slots;             // partial slots per (sequence, KV head): nsplit + 1
+    int part_slots;             // partial slots per (sequence, KV head): split slots
+                                // (>= nsplit) + 1, the last one for the window's partial
     // full-precision window (win_flush = 0: none): the cache holds the quantized middle,
-    // seqlens are whole lengths, slot `nsplit` holds the window's partial
+    // seqlens are whole lengths, the last slot holds the window's partial
     int win_sink, win_keep, win_flush;
+    // > 0: failure-path test hook, each warp first waits this long on a barrier that
+    // nothing arrives at, then takes the timeout path (KVQ_TEST_STALL_NS in kvq.h)
+    long long stall_test_ns;
 };
 
 // The window's attention: one CTA per (KV head, sequence) over the full-precision

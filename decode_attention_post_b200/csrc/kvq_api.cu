@@ -108,19 +108,31 @@ static int num_sms()
     return sms;
 }
 
-// Splits along the tokens so that about 4 waves of the resident CTAs per SM cover the
-// (sequence, KV head) pairs; each split is a whole number of 64-token blocks.
-// KVQ_DECODE_SPLITS overrides the count (tuning).
-static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens)
+// Target number of splits per (sequence, KV head), before clamping to the blocks of the
+// sequence: about 4 waves of the resident CTAs per SM over the pairs.
+// KVQ_DECODE_SPLITS overrides it (tuning).
+static long target_splits(int B, int Hkv)
 {
-    const int blocks = max_seqlen > 0 ? (max_seqlen + kDecodeBlock - 1) / kDecodeBlock : 1;
     const long pairs = (long)B * Hkv;
     const long target = (long)num_sms() * kDecodeMinBlocks * 4;
     long ns = (target + pairs - 1) / pairs;
     if (const char *e = getenv("KVQ_DECODE_SPLITS"))
         ns = atol(e);
-    if (ns < 1)
-        ns = 1;
+    return ns < 1 ? 1 : ns;
+}
+
+static int blocks_of(int max_seqlen)
+{
+    return max_seqlen > 0 ? (max_seqlen + kDecodeBlock - 1) / kDecodeBlock : 1;
+}
+
+// Splits along the tokens; each split is a whole number of 64-token blocks. The count
+// is ceil(blocks / ceil(blocks / ns)) with ns = min(target, blocks), which is at most ns;
+// it is not monotonic in max_seqlen (75 blocks over 74 target splits give 38 splits).
+static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens)
+{
+    const int blocks = blocks_of(max_seqlen);
+    long ns = target_splits(B, Hkv);
     if (ns > blocks)
         ns = blocks;
     const int bps = (int)((blocks + ns - 1) / ns);
@@ -128,9 +140,19 @@ static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens)
     return (blocks + bps - 1) / bps;
 }
 
+// Split partial slots the workspace holds: min(target, blocks), an upper bound of
+// choose_splits that never decreases as max_seqlen grows, so a workspace sized for a
+// longer max_seqlen always serves a shorter one.
+static int split_slots(int B, int Hkv, int max_seqlen)
+{
+    const long ns = target_splits(B, Hkv);
+    const int blocks = blocks_of(max_seqlen);
+    return (int)(ns < blocks ? ns : blocks);
+}
+
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-static DecodeWorkspace decode_layout(int B, int Hkv, int Hq, int d, int nsplit)
+static DecodeWorkspace decode_layout(int B, int Hkv, int Hq, int d, int nslots)
 {
     const int G = Hq / Hkv;
     DecodeWorkspace w;
@@ -141,8 +163,8 @@ static DecodeWorkspace decode_layout(int B, int Hkv, int Hq, int d, int nsplit)
     off += up256((size_t)B * Hq * 4);
     w.qw = off;
     off += up256((size_t)B * Hq * 4);
-    w.part = off;                              // nsplit split slots + 1 window slot
-    off += up256((size_t)B * Hkv * (nsplit + 1) * G * (d + 2) * 4);
+    w.part = off;                              // nslots split slots + 1 window slot
+    off += up256((size_t)B * Hkv * (nslots + 1) * G * (d + 2) * 4);
     w.ticket = off;
     off += up256((size_t)B * Hkv * 4);
     w.total = off;
@@ -245,9 +267,7 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *c, int Hq, int max_seqlen)
 {
     if (check_decode_shape(c, Hq, max_seqlen) != KVQ_OK)
         return 0;
-    int split_tokens = 0;
-    const int ns = choose_splits(c->B, c->Hkv, max_seqlen, &split_tokens);
-    return decode_layout(c->B, c->Hkv, Hq, c->d, ns).total;
+    return decode_layout(c->B, c->Hkv, Hq, c->d, split_slots(c->B, c->Hkv, max_seqlen)).total;
 }
 
 // Shared by the plain and the windowed decode: argument checks beyond the cache shape,
@@ -269,7 +289,8 @@ static kvq_status decode_common(const void *q, kvq_dtype q_dtype, int Hq, const 
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "q_dtype/out_dtype must be KVQ_F32 or KVQ_BF16");
     int split_tokens = 0;
     const int ns = choose_splits(c->B, c->Hkv, qmax, &split_tokens);
-    const DecodeWorkspace w = decode_layout(c->B, c->Hkv, Hq, c->d, ns);
+    const int nslots = split_slots(c->B, c->Hkv, qmax);     // >= ns
+    const DecodeWorkspace w = decode_layout(c->B, c->Hkv, Hq, c->d, nslots);
     if (!workspace || !aligned(workspace, 256))
         KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
     if (ws_bytes < w.total)
@@ -299,10 +320,13 @@ static kvq_status decode_common(const void *q, kvq_dtype q_dtype, int Hq, const 
     L.p.block_table = c->block_table;
     L.p.page_tokens = c->page_tokens;
     L.p.num_pages = c->num_pages;
-    L.p.part_slots = ns + 1;
+    L.p.part_slots = nslots + 1;
     L.p.win_sink = win ? win->S_sink : 0;
     L.p.win_keep = win ? win->S_keep : 0;
     L.p.win_flush = win ? win->S_flush : 0;
+    L.p.stall_test_ns = 0;
+    if (const char *e = getenv("KVQ_TEST_STALL_NS"))
+        L.p.stall_test_ns = atoll(e);
     L.q = q;
     L.q_bf16 = q_dtype == KVQ_BF16;
     L.M = Tk_invT;
@@ -330,7 +354,7 @@ static kvq_status decode_common(const void *q, kvq_dtype q_dtype, int Hq, const 
         W.S_flush = win->S_flush;
         W.part = L.p.part;
         W.part_slots = L.p.part_slots;
-        W.slot = ns;
+        W.slot = nslots;
         W.ticket = L.p.ticket;
         W.out = out;
         W.out_bf16 = L.p.out_bf16;

@@ -66,6 +66,25 @@ __device__ __forceinline__ long long cache_row(const PageMap &pm, int b, int h, 
 // Host-side: thread-local last error text.
 void set_error(const char *fmt, ...);
 
+// Host-side: cudaFuncSetAttribute(MaxDynamicSharedMemorySize) applies to the current
+// device; `done_mask` remembers per device (ordinal mod 64) that it has been set, so the
+// driver call happens once per kernel and device, before any stream capture.
+template <typename F>
+cudaError_t ensure_dynamic_smem(F *func, int bytes, unsigned long long &done_mask)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done_mask & bit)
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        done_mask |= bit;
+    return e;
+}
+
 }  // namespace kvq
 
 #define KVQ_FAIL(code, ...)                 \

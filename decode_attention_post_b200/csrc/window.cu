@@ -11,6 +11,12 @@
 // so that o is in the value-transform domain like the quantized values. The logits are in
 // log2 units, as the decode kernel's partials. When nothing of the sequence is quantized
 // the partial is the whole attention and o / l is written as the output.
+//
+// Ordering with the decode grid that follows: that grid is a programmatic dependent of
+// this kernel and its last split reads this partial and counts this kernel's ticket
+// increment. This kernel therefore never issues griddepcontrol.launch_dependents: the
+// dependent grid's griddepcontrol.wait then returns only after this grid has completed
+// and its writes are visible.
 #include "kvq_common.cuh"
 #include "kvq_ptx.cuh"
 #include "decode_shapes.h"
@@ -153,16 +159,25 @@ __global__ void __launch_bounds__(kWinThreads) window_kernel(WindowParams W)
     }
 }
 
+constexpr int kWinMaxPositions = 2048;       // S_sink + S_keep + S_flush limit (host-checked)
+
+template <int D, int G>
+constexpr size_t window_smem_bytes(int positions)
+{
+    return (size_t)(2 * G * D + 2 * G + G * positions) * sizeof(float);
+}
+
 template <int D, int G>
 cudaError_t launch_window_t(const WindowParams &W, cudaStream_t st)
 {
     const int WMAX = W.S_sink + W.S_keep + W.S_flush;
-    const size_t smem = (size_t)(2 * G * D + 2 * G + G * WMAX) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(window_kernel<D, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // the attribute is set once per device for the largest window, so every call fits
+    static unsigned long long attr_done = 0;
+    cudaError_t e = ensure_dynamic_smem(window_kernel<D, G>,
+                                        (int)window_smem_bytes<D, G>(kWinMaxPositions), attr_done);
     if (e != cudaSuccess)
         return e;
-    window_kernel<D, G><<<dim3(W.Hkv, W.B), kWinThreads, smem, st>>>(W);
+    window_kernel<D, G><<<dim3(W.Hkv, W.B), kWinThreads, window_smem_bytes<D, G>(WMAX), st>>>(W);
     return cudaGetLastError();
 }
 

@@ -64,7 +64,13 @@ typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
 #define KVQ_DEVERR_SEQLEN_CLAMPED 0x1   /* seqlens[b] < 0 or > max_seqlen: clamped */
 #define KVQ_DEVERR_POS_RANGE      0x2   /* pos[b] < 0 or pos[b] + n > T_cap: sequence skipped */
 #define KVQ_DEVERR_NONFINITE      0x4   /* a group had a non-finite clip range: codes 0 */
-#define KVQ_DEVERR_WAIT_TIMEOUT   0x8   /* a bounded pipeline wait gave up: output invalid */
+#define KVQ_DEVERR_WAIT_TIMEOUT   0x8   /* a bounded pipeline wait (about 1 s) gave up: the
+                                           output is invalid; the warp waited for its own
+                                           copies in flight and stopped. For tests of this
+                                           path, the environment variable KVQ_TEST_STALL_NS
+                                           (read at every decode call) makes each decode warp
+                                           first wait that many ns on a barrier nothing
+                                           arrives at and then take the same path. */
 #define KVQ_DEVERR_PAGE_RANGE     0x10  /* a block-table entry outside [0, num_pages): the
                                            append skips the token, the decode reads page 0 */
 
@@ -154,7 +160,8 @@ KVQ_API kvq_status kvq_quantize_append(const void *k_post_rope, const void *v, k
                                kvq_stream_t stream);
 
 /* Workspace bytes kvq_decode_attention needs for this cache shape, Hq query heads and
- * sequences of at most max_seqlen tokens (0 if the arguments are invalid). */
+ * sequences of at most max_seqlen tokens (0 if the arguments are invalid). The size never
+ * decreases as max_seqlen grows, so a workspace sized for T_cap serves every call. */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache *cache, int Hq, int max_seqlen);
 
 /*
@@ -223,7 +230,8 @@ typedef struct {
  * all L positions. q must be bfloat16. The quantized middle of max_seqlen positions must
  * fit the cache (Q(max_seqlen) <= T_cap); S_sink + S_keep + S_flush <= 2048. Workspace:
  * kvq_decode_workspace_bytes(cache, Hq, m) for any m >= Q(max_seqlen) (m = T_cap always
- * suffices). Other arguments and errors as in kvq_decode_attention.
+ * suffices, as that size never decreases with m). Other arguments and errors as in
+ * kvq_decode_attention.
  */
 KVQ_API kvq_status kvq_decode_attention_window(const void *q, kvq_dtype q_dtype, int Hq,
                                                const float *Tk_invT, const kvq_cache *cache,

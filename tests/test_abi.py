@@ -199,6 +199,40 @@ def test_workspace_sizes_positive_and_monotone():
     assert L.kvq_bf16_decode_workspace_bytes(4, 32, 8, 96, 16384) == 0
 
 
+def test_workspace_never_shrinks_across_a_split_boundary():
+    """With 32 (sequence, KV head) pairs the split target is 74 (148 SMs x 4 CTAs x 4 waves
+    / 32): 74 blocks of 64 tokens give 74 splits and 75 blocks only 38. The workspace must
+    not shrink at that boundary, so that a size query for any longer max_seqlen (e.g.
+    T_cap, as the windowed decode allows) covers every shorter call."""
+    L = kvq.load()
+    desc, _ = _desc(B=4, Hkv=8, T_cap=16384)
+    sizes = [L.kvq_decode_workspace_bytes(C.byref(desc), 32, m)
+             for m in range(64, 16385, 64)]
+    assert all(0 < a <= b for a, b in zip(sizes, sizes[1:]))
+    assert L.kvq_decode_workspace_bytes(C.byref(desc), 32, 74 * 64) == \
+        L.kvq_decode_workspace_bytes(C.byref(desc), 32, 75 * 64)
+
+
+def test_window_decode_accepts_a_workspace_sized_for_t_cap():
+    """The header's promise: kvq_decode_workspace_bytes(cache, Hq, m) for any m >= the
+    quantized middle of max_seqlen (m = T_cap always) is enough. The windowed decode needs
+    the size for its quantized middle, one byte less is rejected (KVQ_ERR_WORKSPACE, 4)
+    before anything is launched; the T_cap size is at least that."""
+    import oracle
+    L = kvq.load()
+    desc, _ = _desc(B=4, Hkv=8, T_cap=16384)
+    ws_cap = L.kvq_decode_workspace_bytes(C.byref(desc), 32, 16384)
+    for S_sink, S_keep, S_flush in [(0, 0, 64), (4, 60, 64), (64, 256, 128)]:
+        for mid_blocks in (1, 37, 74, 75, 149, 255):
+            max_seqlen = S_sink + S_keep + mid_blocks * 64
+            qmax = oracle.window_quantized(max_seqlen, S_sink, S_keep, S_flush)
+            need = L.kvq_decode_workspace_bytes(C.byref(desc), 32, qmax)
+            assert 0 < need <= ws_cap
+            r = _window_decode(desc, _win(S_sink, S_keep, S_flush), Hq=32,
+                               max_seqlen=max_seqlen, ws_bytes=need - 1)
+            assert r == 4, (S_sink, S_keep, S_flush, mid_blocks)
+
+
 def test_bf16_decode_argument_errors():
     L = kvq.load()
     args = dict(q=0x1000, Hq=32, k=0x2000, v=0x3000, B=2, Hkv=8, T_cap=128, d=128,

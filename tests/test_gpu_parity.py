@@ -280,6 +280,9 @@ DECODE_CASES = [
     ("gqa4-k4v2", small(synth.CONFIGS[3], T_cap=1280), 2, [1280, 700]),
     ("gqa8-d64", small(synth.CONFIGS[4], T_cap=768), 2, [768, 333]),
     ("gqa4-v4", small(synth.CONFIGS[1], T_cap=512, bits_v=4), 2, [512, 129]),
+    ("gqa8-d128", small(synth.CONFIGS[1], T_cap=640, Hq=64), 2, [640, 321]),
+    ("gqa8-d128-k4v4", small(synth.CONFIGS[1], T_cap=384, Hq=64, bits_k=4, bits_v=4), 2,
+     [384, 70]),
 ]
 
 
@@ -308,6 +311,27 @@ def test_decode_split_invariance(splits, monkeypatch):
     out, err = gpu_decode(cfg, q, M, gc, seql)
     assert err == 0
     assert_close(out.cpu().numpy(), want, where=f"splits={splits}")
+
+
+def test_decode_wait_timeout_is_flagged_and_the_context_stays_usable(monkeypatch):
+    """Failure path of the bounded pipeline waits, made to run out without a fault: the
+    test hook KVQ_TEST_STALL_NS makes every decode warp first wait 1 ms on a barrier that
+    nothing arrives at. Each warp then takes the timeout path (waits for its own copies
+    in flight, skips its blocks) and the call flags KVQ_DEVERR_WAIT_TIMEOUT. The next
+    call without the hook gives the oracle's result, so the context is intact."""
+    cfg = small(synth.CONFIGS[2], T_cap=1024)
+    oc, M = oracle_built_cache(cfg, 2, 1024)
+    gc = upload_cache(oc, cfg)
+    q = synth.as_dtype(synth.queries(cfg.with_(B=2)), cfg.q_dtype)
+    seql = [1024, 517]
+    want = oracle.decode(q, M, oc, np.array(seql, np.int32))
+    monkeypatch.setenv("KVQ_TEST_STALL_NS", "1000000")
+    _, err = gpu_decode(cfg, q, M, gc, seql)
+    assert err & kvq.KVQ_DEVERR_WAIT_TIMEOUT
+    monkeypatch.delenv("KVQ_TEST_STALL_NS")
+    out, err = gpu_decode(cfg, q, M, gc, seql)
+    assert err == 0
+    assert_close(out.cpu().numpy(), want, where="after the timeout test")
 
 
 @pytest.mark.parametrize("splits", ["1", "3", "100"])
