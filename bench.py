@@ -39,6 +39,7 @@ CONFIG_IDX = 2
 DECODE_TRAFFIC_BYTES = None
 DECODE_TRAFFIC_KERNEL = "decode_kernel<128,4,2,2>"
 APPEND_CONFIG_IDX = 4
+DECODE_CONFIGS = (1, 3, 4)       # further decode shapes timed as extras
 
 
 def step_bytes(cfg, seqlens):
@@ -209,6 +210,65 @@ class Workload:
         self.decode()
 
 
+class E2EStep:
+    """One serving step through the public API with host buffers: a single pinned host
+    staging buffer holds q, the new token's k and v, seqlens and positions; one
+    cudaMemcpyAsync moves it into a device staging buffer whose views are the step's
+    inputs; append + decode run; the bf16 output is copied back to pinned host memory.
+    The sequence is captured once in a CUDA graph and replayed."""
+
+    def __init__(self, w):
+        import torch
+        parts = [w.q, w.knew, w.vnew, w.seq_d, w.pos]
+        sizes = [t.numel() * t.element_size() for t in parts]
+        offs = np.concatenate([[0], np.cumsum([(n + 255) // 256 * 256 for n in sizes])])
+        self.stage_d = torch.empty(int(offs[-1]), dtype=torch.uint8, device=w.dev)
+        self.stage_h = torch.empty(int(offs[-1]), dtype=torch.uint8).pin_memory()
+        views = []
+        for t, o, n in zip(parts, offs[:-1], sizes):
+            hv = self.stage_h[int(o):int(o) + n].view(t.dtype).view(t.shape)
+            hv.copy_(t.cpu())
+            views.append(self.stage_d[int(o):int(o) + n].view(t.dtype).view(t.shape))
+        self.q, self.knew, self.vnew, self.seq_d, self.pos = views
+        self.w = w
+        self.out_h = torch.empty(w.out.shape, dtype=w.out.dtype).pin_memory()
+        self.h2d_bytes = int(sum(sizes))
+        self.d2h_bytes = self.out_h.numel() * self.out_h.element_size()
+
+    def step(self):
+        import decode_attention_post_b200 as kvq
+        w = self.w
+        self.stage_d.copy_(self.stage_h, non_blocking=True)
+        kvq.quantize_append(self.knew, self.vnew, w.Tk, w.Tv, w.qp, w.cache, self.pos, n=1,
+                            dev_err=w.err)
+        kvq.decode_attention(self.q, w.Tit, w.cache, self.seq_d, w.max_seqlen, w.out, w.ws,
+                             dev_err=w.err)
+        self.out_h.copy_(w.out, non_blocking=True)
+
+    def time(self, iters, stream, barrier):
+        import torch
+        for _ in range(3):
+            self.step()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        del g
+        return e0.elapsed_time(e1) / iters
+
+
 def time_events(fn, iters, stream, per_graph=1):
     """Mean device time of one fn() call: fn is captured `per_graph` times into a CUDA
     graph, each replay is bracketed by CUDA events on the launching stream, so host
@@ -300,38 +360,14 @@ def run_gpu(args):
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     dev_err = int(w.err.item())
 
-    # ---- end to end through the public API with pinned host buffers
-    q_h = w.q.cpu().pin_memory()
-    k_h, v_h = w.knew.cpu().pin_memory(), w.vnew.cpu().pin_memory()
-    s_h, p_h = w.seq_d.cpu().pin_memory(), w.pos.cpu().pin_memory()
-    out_h = torch.empty_like(w.out, device="cpu").pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, s_h, p_h))
-    d2h = out_h.numel() * out_h.element_size()
-
-    def e2e_step():
-        w.q.copy_(q_h, non_blocking=True)
-        w.knew.copy_(k_h, non_blocking=True)
-        w.vnew.copy_(v_h, non_blocking=True)
-        w.seq_d.copy_(s_h, non_blocking=True)
-        w.pos.copy_(p_h, non_blocking=True)
-        w.step()
-        out_h.copy_(w.out, non_blocking=True)
-
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    Ke = min(K, 500)
-    barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(Ke):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / Ke
+    # ---- end to end through the public API: the step's inputs (q, the new token's k and
+    #      v, seqlens, positions) packed in one pinned host buffer and moved by one
+    #      host->device copy, the step, and the output read back to pinned host memory;
+    #      the whole sequence is replayed as a CUDA graph
+    e2e = E2EStep(w)
+    e2e_ms = max_over_ranks(e2e.time(min(K, 500), stream, barrier))
     e2e_value = weak_scaling_gbs(dec_bytes + app_bytes, e2e_ms, world)
+    h2d, d2h = e2e.h2d_bytes, e2e.d2h_bytes
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -354,7 +390,9 @@ def run_gpu(args):
         "append_decode_time": {"append_ms": round(app_ms, 5), "decode_ms": round(dec_ms, 5),
                                "append_tok_per_s": round(cfg.B / (app_ms * 1e-3), 1)},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "one pinned staging buffer -> one H2D copy, append + decode, D2H of "
+                       "the output; replayed as a CUDA graph"},
         "gpu_launches": 3 * K,
         "dev_err": dev_err,
         "clocks": clocks,
@@ -366,12 +404,93 @@ def run_gpu(args):
         del w
         torch.cuda.empty_cache()
         line["chunk_append"] = chunk_append(device, stream)
+        line["append_config0"] = append_config0(device, stream)
+        line["decode_configs"] = [decode_config_line(i, device, stream, peak)
+                                  for i in DECODE_CONFIGS]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def build_cache(cfg, device, append_n=None):
+    """The workload's cache filled by the library's own quantize-append from the seeded
+    synthetic keys and values, one sequence at a time (seqlens as drawn)."""
+    import torch
+    import decode_attention_post_b200 as kvq
+    qp = kvq.QParams(cfg.bits_k, cfg.bits_v, cfg.group, cfg.clip_alpha)
+    cache = kvq.KVCache.allocate(cfg.B, cfg.Hkv, cfg.T_cap, cfg.d, qp, device=device)
+    seql = synth.seqlens(cfg)
+    Tk, Tv, Tit = synth.transforms(cfg)
+    g = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    Tk, Tv, Tit = g(Tk), g(Tv), g(Tit)
+    zero = torch.zeros(1, dtype=torch.int32, device=device)
+    for b in range(cfg.B):
+        n = int(seql[b])
+        kd = g(synth.keys(cfg, b, 0, n)).to(torch.bfloat16)
+        vd = g(synth.values(cfg, b, 0, n)).to(torch.bfloat16)
+        kvq.quantize_append(kd[None], vd[None], Tk, Tv, qp, cache.view_sequence(b), zero)
+        del kd, vd
+    torch.cuda.synchronize()
+    return cache, seql, Tit
+
+
+def decode_bytes(cfg, seql):
+    ng = cfg.d // cfg.group
+    per_tok = cfg.Hkv * (cfg.d * cfg.bits_k // 8 + 4 * ng + cfg.d * cfg.bits_v // 8 + 4 * ng)
+    return int(np.sum(seql)) * per_tok + 2 * cfg.B * cfg.Hq * cfg.d * 2
+
+
+def decode_config_line(idx, device, stream, peak):
+    """Decode call (q prologue + split-K decode) at one more workload shape."""
+    import torch
+    import decode_attention_post_b200 as kvq
+    cfg = synth.CONFIGS[idx]
+    cache, seql, Tit = build_cache(cfg, device)
+    q = torch.from_numpy(synth.queries(cfg)).to(device).to(torch.bfloat16)
+    sd = torch.from_numpy(seql).to(device)
+    out = torch.empty((cfg.B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=device)
+    ws = torch.empty(kvq.decode_workspace_bytes(cache, cfg.Hq, cfg.T_cap), dtype=torch.uint8,
+                     device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    fn = lambda: kvq.decode_attention(q, Tit, cache, sd, cfg.T_cap, out, ws, dev_err=err)
+    ms = statistics.mean(time_events(fn, 200, stream))
+    nbytes = decode_bytes(cfg, seql)
+    res = {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
+           "bits_k": cfg.bits_k, "bits_v": cfg.bits_v,
+           "seqlens": f"U[{cfg.seq_lo},{cfg.seq_hi}]", "sum_seqlens": int(np.sum(seql)),
+           "bytes_per_launch": nbytes, "ms_per_launch": round(ms, 5),
+           "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+           "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4),
+           "dev_err": int(err.item())}
+    del cache, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def append_config0(device, stream):
+    """Prefill append of the tiny float32 workload (1 sequence, 2048 tokens, 1 KV head,
+    d 128): float32 CUDA-core transform path."""
+    import torch
+    import decode_attention_post_b200 as kvq
+    cfg = synth.CONFIGS[0]
+    qp = kvq.QParams(cfg.bits_k, cfg.bits_v, cfg.group, cfg.clip_alpha)
+    cache = kvq.KVCache.allocate(cfg.B, cfg.Hkv, cfg.T_cap, cfg.d, qp, device=device)
+    Tk, Tv, _ = synth.transforms(cfg)
+    k, v = synth.kv_batch(cfg, 0, cfg.T_cap)
+    g = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    kd, vd, Tk, Tv = g(k), g(v), g(Tk), g(Tv)
+    pos = torch.zeros(cfg.B, dtype=torch.int32, device=device)
+    fn = lambda: kvq.quantize_append(kd, vd, Tk, Tv, qp, cache, pos)
+    ms = statistics.mean(time_events(fn, 50, stream))
+    tokheads = cfg.B * cfg.T_cap * cfg.Hkv
+    nbytes = tokheads * (2 * cfg.d * 4 + cfg.d * (cfg.bits_k + cfg.bits_v) // 8 + 8) + \
+        2 * cfg.Hkv * cfg.d * cfg.d * 4
+    return {"workload": cfg.name, "ms": round(ms, 4),
+            "tok_per_s": round(cfg.B * cfg.T_cap / (ms * 1e-3), 1),
+            "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "bytes": nbytes}
 
 
 def bf16_comparator(w, cfg, K, stream, dec_ms):
@@ -490,21 +609,31 @@ class OracleSample:
 
 
 def cpu_baseline(cfg, budget_s=12.0):
+    """The float64 oracle on the host cores: all threads, then one thread (a quarter of
+    the budget), on one sequence of the workload."""
     import oracle
     s = OracleSample(cfg, 1)
-    t = time.perf_counter()
-    s.step()
-    one = time.perf_counter() - t
-    reps = max(1, int(budget_s / max(one, 1e-3)))
-    t = time.perf_counter()
-    for _ in range(reps):
+    cores = oracle.get_threads()
+
+    def timed(budget):
+        t = time.perf_counter()
         s.step()
-    el = (time.perf_counter() - t) / reps
+        one = time.perf_counter() - t
+        reps = max(1, int(budget / max(one, 1e-3)))
+        t = time.perf_counter()
+        for _ in range(reps):
+            s.step()
+        return (time.perf_counter() - t) / reps, reps
+    el, reps = timed(budget_s)
+    oracle.set_threads(1)
+    el1, reps1 = timed(budget_s / 4)
+    oracle.set_threads(cores)
     return {"value": round(s.bytes() / el / 1e9, 4), "unit": "GB/s",
-            "cores": oracle.get_threads(), "kind": "oracle",
+            "cores": cores, "kind": "oracle",
+            "single_thread_value": round(s.bytes() / el1 / 1e9, 5),
             "sample": f"1 of {cfg.B} sequences (seqlen {int(s.seqlens[0])}), all {cfg.Hq} "
-                      f"query heads: append 1 token + decode, {reps} reps, "
-                      f"{el:.3f} s per step"}
+                      f"query heads: append 1 token + decode, {reps} reps at {cores} threads "
+                      f"({el:.3f} s per step), {reps1} reps at 1 thread ({el1:.3f} s)"}
 
 
 def run_reference(args):
@@ -547,6 +676,44 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def profile_case(name):
+    """One kernel's workload on its own, a few launches, for an ncu capture of that kernel
+    (the command is recorded in the profiles directory). Prints one JSON line."""
+    import torch
+    import decode_attention_post_b200 as kvq
+    torch.cuda.set_device(0)
+    device, stream = "cuda:0", torch.cuda.current_stream()
+    peak, _ = peaks()
+    if name == "chunk_append":
+        res = chunk_append(device, stream)
+    elif name == "append_config0":
+        res = append_config0(device, stream)
+    elif name.startswith("decode_config"):
+        res = decode_config_line(int(name[len("decode_config"):]), device, stream, peak)
+    elif name == "bf16_config1":
+        # the uncompressed comparator at the batch-16 / 16K shape (1.07 GB of bf16 K and V);
+        # its time does not depend on the values, so they are drawn on the device
+        cfg = synth.CONFIGS[1]
+        gen = torch.Generator(device=device)
+        gen.manual_seed(1000 * cfg.idx + synth.STREAM_CACHE)
+        shape = (cfg.B, cfg.Hkv, cfg.T_cap, cfg.d)
+        kb = torch.randn(shape, generator=gen, device=device).to(torch.bfloat16)
+        vb = torch.randn(shape, generator=gen, device=device).to(torch.bfloat16)
+        q = torch.from_numpy(synth.queries(cfg)).to(device).to(torch.bfloat16)
+        sd = torch.from_numpy(synth.seqlens(cfg)).to(device)
+        out = torch.empty((cfg.B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=device)
+        ws = torch.empty(kvq.bf16_decode_workspace_bytes(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.T_cap),
+                         dtype=torch.uint8, device=device)
+        fn = lambda: kvq.bf16_decode(q, kb, vb, sd, cfg.T_cap, out, ws)
+        ms = statistics.mean(time_events(fn, 20, stream))
+        nbytes = int(np.sum(synth.seqlens(cfg))) * cfg.Hkv * cfg.d * 4 + 2 * cfg.B * cfg.Hq * cfg.d * 2
+        res = {"workload": cfg.name, "ms": round(ms, 5),
+               "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "bytes": nbytes}
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    print(json.dumps({"case": name, **res}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -556,8 +723,13 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip bf16 comparator and chunk append")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile-case", default=None,
+                    help="run one kernel's workload alone (chunk_append, append_config0, "
+                         "decode_config1/3/4, bf16_config1) for an ncu capture")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.profile_case:
+        profile_case(args.profile_case)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

@@ -25,4 +25,5 @@ from .kvq import (  # noqa: F401
     library_path,
     load,
     quantize_append,
+    window_append,
 )

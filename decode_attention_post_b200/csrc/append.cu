@@ -73,6 +73,64 @@ __device__ __forceinline__ float order_stat(const float (&vals)[NV], int kappa, 
     return m;
 }
 
+// Where flattened token (b, i) of the call comes from and goes to.
+//  plain append (ring_k == nullptr): input row (b, i) of in[B][n][Hkv][D], written at cache
+//    position pos[b] + i; the sequence is out of range unless 0 <= pos[b], pos[b] + n <= T_cap.
+//  window flush (kvq_window_append, WUSH-KV section 4.4): sequence b had len[b] positions
+//    and receives n_new more; the call quantizes the positions that leave the
+//    full-precision window, [S_sink + Q(len), S_sink + Q(len + n_new)) with Q the
+//    quantized-middle length, i.e. i < Q(len + n_new) - Q(len) (larger i: nothing to do).
+//    Position t = S_sink + Q(len) + i comes from the recent ring (slot t % R of
+//    ring[B][Hkv][R][D]) when t < len, else from the new tokens (row t - len of
+//    in[B][n_new][Hkv][D]); it is written at cache position Q(len) + i. Out of range
+//    unless Q(len + n_new) <= T_cap.
+struct TokenMap {
+    const void *ring_k, *ring_v;
+    const int32_t *len;
+    int S_sink, S_keep, S_flush, R, n_new;
+};
+
+struct TokenSlot {
+    bool active;        // the token is written by this call
+    bool bad_range;     // its sequence is out of range (flagged once, skipped)
+    int first;          // i == 0 of its sequence
+    size_t src;         // element offset of its input row
+    const void *base;   // buffer holding the row
+    int dst;            // cache position
+};
+
+__device__ __forceinline__ TokenSlot token_slot(const TokenMap &tm, const void *in, int which,
+                                                const int32_t *pos, int b, int i, int n, int h,
+                                                int Hkv, int D, int T_cap)
+{
+    TokenSlot ts;
+    ts.first = i == 0;
+    if (!tm.ring_k) {
+        const int p0 = pos[b];
+        ts.bad_range = p0 < 0 || (long)p0 + n > T_cap;
+        ts.active = !ts.bad_range;
+        ts.base = in;
+        ts.src = (((size_t)b * n + i) * Hkv + h) * D;
+        ts.dst = p0 + i;
+        return ts;
+    }
+    const int L = tm.len[b];
+    const int qo = L < 0 ? 0 : window_quantized(L, tm.S_sink, tm.S_keep, tm.S_flush);
+    const int qn = L < 0 ? 0 : window_quantized(L + tm.n_new, tm.S_sink, tm.S_keep, tm.S_flush);
+    ts.bad_range = L < 0 || qn > T_cap;
+    ts.active = !ts.bad_range && i < qn - qo;
+    const int t = tm.S_sink + qo + i;
+    if (t < L) {
+        ts.base = which ? tm.ring_v : tm.ring_k;
+        ts.src = (((size_t)b * Hkv + h) * tm.R + t % tm.R) * D;
+    } else {
+        ts.base = in;
+        ts.src = (((size_t)b * tm.n_new + (t - L)) * Hkv + h) * D;
+    }
+    ts.dst = qo + i;
+    return ts;
+}
+
 template <int D, int TPW>
 __global__ void __launch_bounds__(kAppendThreads)
 append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in, int in_bf16,
@@ -80,9 +138,10 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
                    int Hkv, int T_cap, int bits_k, int bits_v, int group, int kappa,
                    uint8_t *__restrict__ k_codes, uint32_t *__restrict__ k_sz,
                    uint8_t *__restrict__ v_codes, uint32_t *__restrict__ v_sz,
-                   const int32_t *__restrict__ pos, int32_t *dev_err, PageMap pm)
+                   const int32_t *__restrict__ pos, int32_t *dev_err, PageMap pm, TokenMap tm)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ int tile_active;
     using Smem = AppendSmem<D, TPW>;
     constexpr int kTokPerWarp = TPW;
     constexpr int kTokPerTile = Smem::kTokPerTile;
@@ -100,7 +159,9 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
     const int ng = D / group;
     const int qmax = (1 << bits) - 1;
 
-    if (T) {
+    // T_h staged transposed; a window flush stages it only once the CTA meets a tile with
+    // work (most CTAs of a decode-time flush have none)
+    auto stage_T = [&]() {
         // 16 independent float4 loads in flight per thread, then transposed stores
         const float4 *Th4 = reinterpret_cast<const float4 *>(T + (size_t)h * D * D);
         constexpr int N4 = D * D / 4 / kAppendThreads;
@@ -114,11 +175,36 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
             sm.Tt[(j + 2) * (D + 1) + i] = v4.z;
             sm.Tt[(j + 3) * (D + 1) + i] = v4.w;
         }
+    };
+    bool T_staged = false;
+    if (T && !tm.ring_k) {
+        stage_T();
+        T_staged = true;
     }
 
     for (long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         const long u0 = tile * kTokPerTile;
         __syncthreads();                        // previous tile's readers are done
+        if (tm.ring_k) {
+            // window flush: most sequences flush nothing in a call; skip tiles without work
+            if (threadIdx.x == 0)
+                tile_active = 0;
+            __syncthreads();
+            if (threadIdx.x < kTokPerTile && u0 + threadIdx.x < total) {
+                const long u = u0 + threadIdx.x;
+                const TokenSlot ts = token_slot(tm, in, which, pos, (int)(u / n), (int)(u % n), n,
+                                                h, Hkv, D, T_cap);
+                if (ts.active || (ts.bad_range && ts.first))
+                    tile_active = 1;
+            }
+            __syncthreads();
+            if (!tile_active)
+                continue;
+            if (T && !T_staged) {               // uniform: every thread saw tile_active
+                stage_T();
+                T_staged = true;
+            }
+        }
 #pragma unroll
         for (int it = 0; it < (kTokPerTile * D + kAppendThreads - 1) / kAppendThreads; ++it) {
             const int idx = threadIdx.x + kAppendThreads * it;
@@ -128,8 +214,10 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
             const long u = u0 + tk;
             float x = 0.f;
             if (u < total) {
-                const long b = u / n, i = u % n;
-                x = load_in(in, in_bf16, (((size_t)b * n + i) * Hkv + h) * D + j);
+                const TokenSlot ts = token_slot(tm, in, which, pos, (int)(u / n), (int)(u % n), n,
+                                                h, Hkv, D, T_cap);
+                if (ts.active)
+                    x = load_in(ts.base, in_bf16, ts.src + j);
             }
             sm.X[tk][j] = x;
         }
@@ -173,13 +261,15 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
             if (u >= total)
                 break;
             const int b = (int)(u / n), i = (int)(u % n);
-            const int p0 = pos[b];
-            if (p0 < 0 || (long)p0 + n > T_cap) {
-                if (i == 0 && lane == 0)
+            const TokenSlot ts = token_slot(tm, in, which, pos, b, i, n, h, Hkv, D, T_cap);
+            if (ts.bad_range) {
+                if (ts.first && lane == 0)
                     flag(dev_err, KVQ_DEVERR_POS_RANGE);
                 continue;
             }
-            const int t = p0 + i;
+            if (!ts.active)
+                continue;
+            const int t = ts.dst;
             const long long row = cache_row(pm, b, h, Hkv, T_cap, t);
             if (row < 0) {
                 if (lane == 0)
@@ -256,7 +346,8 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
 template <int D, int TPW>
 cudaError_t launch_append_fp32(const void *k, const void *v, int in_bf16, const float *Tk,
                                const float *Tv, int B, int n, const kvq_cache *c, int kappa,
-                               const int32_t *pos, int32_t *dev_err, cudaStream_t st)
+                               const int32_t *pos, int32_t *dev_err, cudaStream_t st,
+                               const TokenMap &tm = TokenMap{})
 {
     using Smem = AppendSmem<D, TPW>;
     const size_t smem = sizeof(Smem);
@@ -278,13 +369,16 @@ cudaError_t launch_append_fp32(const void *k, const void *v, int in_bf16, const 
         want = 1;
     // at least 8 tiles per CTA once the T staging cost matters
     long gx = tiles < want ? tiles : want;
-    if (tiles > want * 8)
+    if (tm.ring_k)                          // window flush: most tiles have no work
+        gx = tiles < want * 4 ? tiles : want * 4;
+    else if (tiles > want * 8)
         gx = (tiles + 7) / 8 < 65535 ? (tiles + 7) / 8 : 65535;
     dim3 grid((unsigned)gx, (unsigned)c->Hkv, 2);
     append_fp32_kernel<D, TPW><<<grid, kAppendThreads, smem, st>>>(
         k, v, in_bf16, Tk, Tv, B, n, c->Hkv, c->T_cap, c->qp.bits_k, c->qp.bits_v, c->qp.group,
         kappa, (uint8_t *)c->k_codes, (uint32_t *)c->k_sz, (uint8_t *)c->v_codes,
-        (uint32_t *)c->v_sz, pos, dev_err, PageMap{c->block_table, c->page_tokens, c->num_pages});
+        (uint32_t *)c->v_sz, pos, dev_err, PageMap{c->block_table, c->page_tokens, c->num_pages},
+        tm);
     return cudaGetLastError();
 }
 
@@ -293,6 +387,35 @@ cudaError_t launch_append_fp32(const void *k, const void *v, int in_bf16, const 
 cudaError_t append_mma(const void *k, const void *v, const float *Tk, const float *Tv, int B,
                        int n, const kvq_cache *c, int kappa, const int32_t *pos, int32_t *dev_err,
                        cudaStream_t st);
+
+// Window flush of kvq_window_append: the positions leaving the full-precision window
+// (from the recent ring or the n_new new tokens) through the float32 CUDA-core path; the
+// flattened list holds S_flush * ceil(n_new / S_flush) entries per sequence, the most any
+// sequence can flush in one call.
+cudaError_t window_flush_launch(const void *k_new, const void *v_new, const float *Tk,
+                                const float *Tv, int B, int n_new, const kvq_cache *c, int kappa,
+                                const void *ring_k, const void *ring_v, const int32_t *len,
+                                int S_sink, int S_keep, int S_flush, int32_t *dev_err,
+                                cudaStream_t st)
+{
+    TokenMap tm;
+    tm.ring_k = ring_k;
+    tm.ring_v = ring_v;
+    tm.len = len;
+    tm.S_sink = S_sink;
+    tm.S_keep = S_keep;
+    tm.S_flush = S_flush;
+    tm.R = S_keep + S_flush;
+    tm.n_new = n_new;
+    const long nmax = (long)S_flush * ((n_new + S_flush - 1) / S_flush);
+    if (nmax > 0x7fffffffL / (B > 0 ? B : 1))
+        return cudaErrorInvalidValue;
+    if (c->d == 64)
+        return launch_append_fp32<64, 4>(k_new, v_new, 1, Tk, Tv, B, (int)nmax, c, kappa, nullptr,
+                                         dev_err, st, tm);
+    return launch_append_fp32<128, 4>(k_new, v_new, 1, Tk, Tv, B, (int)nmax, c, kappa, nullptr,
+                                      dev_err, st, tm);
+}
 
 // Chunks of bfloat16 inputs with both transforms go to the tensor-core kernel; float32
 // inputs, identity transforms, small (decode-time) appends and unaligned inputs use the

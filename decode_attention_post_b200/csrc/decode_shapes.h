@@ -79,11 +79,5 @@ size_t decode_qfrag_words(int d, int G);
 cudaError_t launch_decode(const DecodeLaunch &L, cudaStream_t st);
 cudaError_t launch_window(const WindowParams &W, cudaStream_t st);
 
-// Quantized middle length of a sequence of L positions with a full-precision window.
-__host__ __device__ inline int window_quantized(int L, int S_sink, int S_keep, int S_flush)
-{
-    const int e = L - S_sink - S_keep;
-    return e > 0 ? (e / S_flush) * S_flush : 0;
-}
 
 }  // namespace kvq

@@ -14,6 +14,15 @@ namespace kvq {
 cudaError_t append_launch(const void *k, const void *v, int in_bf16, const float *Tk,
                           const float *Tv, int B, int n, const kvq_cache *c, int kappa,
                           const int32_t *pos, int32_t *dev_err, cudaStream_t st);
+cudaError_t window_flush_launch(const void *k_new, const void *v_new, const float *Tk,
+                                const float *Tv, int B, int n_new, const kvq_cache *c, int kappa,
+                                const void *ring_k, const void *ring_v, const int32_t *len,
+                                int S_sink, int S_keep, int S_flush, int32_t *dev_err,
+                                cudaStream_t st);
+cudaError_t launch_window_store(const void *k_new, const void *v_new, int B, int n, int Hkv,
+                                int d, const int32_t *len, int S_sink, int S_keep, int S_flush,
+                                int T_cap, void *k_sink, void *v_sink, void *k_ring, void *v_ring,
+                                cudaStream_t st);
 cudaError_t launch_bf16_decode(const void *q, int Hq, const void *k, const void *v, int B,
                                int Hkv, int T_cap, int d, const int32_t *seqlens, int max_seqlen,
                                void *out, void *ws, int nsplit, int split_tokens,
@@ -376,14 +385,9 @@ kvq_status kvq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const 
                          out_dtype, workspace, ws_bytes, dev_err, stream, nullptr);
 }
 
-kvq_status kvq_decode_attention_window(const void *q, kvq_dtype q_dtype, int Hq,
-                                       const float *Tk_invT, const kvq_cache *c,
-                                       const kvq_window *win, const int32_t *seqlens,
-                                       int max_seqlen, void *out, kvq_dtype out_dtype,
-                                       void *workspace, size_t ws_bytes, int32_t *dev_err,
-                                       kvq_stream_t stream)
+// Window parameters shared by the windowed decode and the windowed append.
+static kvq_status check_window(const kvq_window *win)
 {
-    g_last_error[0] = 0;
     if (!win)
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "window is NULL");
     if (win->S_sink < 0 || win->S_keep < 0 || win->S_flush <= 0)
@@ -394,6 +398,68 @@ kvq_status kvq_decode_attention_window(const void *q, kvq_dtype q_dtype, int Hq,
                  (long)win->S_sink + win->S_keep + win->S_flush);
     if ((win->S_sink > 0 && (!win->k_sink || !win->v_sink)) || !win->k_recent || !win->v_recent)
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "a window buffer is NULL");
+    return KVQ_OK;
+}
+
+kvq_status kvq_window_append(const void *k_new, const void *v_new, kvq_dtype in_dtype,
+                             const float *T_k, const float *T_v, const kvq_qparams *qp,
+                             kvq_cache *cache, const kvq_window *win, const int32_t *seqlens,
+                             int n, int32_t *dev_err, kvq_stream_t stream)
+{
+    g_last_error[0] = 0;
+    kvq_status s = check_cache(cache);
+    if (s != KVQ_OK)
+        return s;
+    s = check_qparams(qp, cache->d);
+    if (s != KVQ_OK)
+        return s;
+    if (!same_qp(qp, &cache->qp))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "qparams differ from the cache's qparams");
+    s = check_window(win);
+    if (s != KVQ_OK)
+        return s;
+    if (in_dtype != KVQ_BF16)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "the windowed append takes bfloat16 keys and values");
+    if (n < 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "n=%d is negative", n);
+    if (n == 0)
+        return KVQ_OK;
+    if (!k_new || !v_new || !seqlens)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "k_new, v_new and seqlens must not be NULL");
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(win->k_recent, 16) ||
+        !aligned(win->v_recent, 16) ||
+        (win->S_sink > 0 && (!aligned(win->k_sink, 16) || !aligned(win->v_sink, 16))))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "bfloat16 token and window buffers must be 16-byte aligned");
+    if ((long)cache->B * n > 0x7fffffffL / 4)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "B * n = %ld new tokens in one call is too many",
+                 (long)cache->B * n);
+    cudaStream_t st = (cudaStream_t)stream;
+    // the flush reads ring slots that the store below may overwrite: flush first
+    cudaError_t e = window_flush_launch(k_new, v_new, T_k, T_v, cache->B, n, cache,
+                                        kappa_of(qp->clip_alpha, qp->group), win->k_recent,
+                                        win->v_recent, seqlens, win->S_sink, win->S_keep,
+                                        win->S_flush, dev_err, st);
+    if (e != cudaSuccess)
+        KVQ_FAIL(KVQ_ERR_CUDA, "window flush launch: %s", cudaGetErrorString(e));
+    e = launch_window_store(k_new, v_new, cache->B, n, cache->Hkv, cache->d, seqlens,
+                            win->S_sink, win->S_keep, win->S_flush, cache->T_cap, win->k_sink,
+                            win->v_sink, win->k_recent, win->v_recent, st);
+    if (e != cudaSuccess)
+        KVQ_FAIL(KVQ_ERR_CUDA, "window store launch: %s", cudaGetErrorString(e));
+    return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention_window(const void *q, kvq_dtype q_dtype, int Hq,
+                                       const float *Tk_invT, const kvq_cache *c,
+                                       const kvq_window *win, const int32_t *seqlens,
+                                       int max_seqlen, void *out, kvq_dtype out_dtype,
+                                       void *workspace, size_t ws_bytes, int32_t *dev_err,
+                                       kvq_stream_t stream)
+{
+    g_last_error[0] = 0;
+    kvq_status ws = check_window(win);
+    if (ws != KVQ_OK)
+        return ws;
     if (q_dtype != KVQ_BF16)
         KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "the windowed decode takes bfloat16 queries");
     if (max_seqlen < 0)

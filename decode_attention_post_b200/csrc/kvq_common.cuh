@@ -40,6 +40,16 @@ __host__ __device__ __forceinline__ int v_half_offset(int d, int bits, int tok, 
     return lane * chunk + (p * W + r) * 4 + 2 * hi;
 }
 
+// Quantized middle length of a sequence of L positions with a full-precision window
+// (WUSH-KV section 4.4): the flush runs after every append and quantizes the oldest
+// S_flush eligible positions while at least S_flush are eligible, so the middle
+// [S_sink, S_sink + Q) holds Q = S_flush * floor(max(0, L - S_sink - S_keep) / S_flush).
+__host__ __device__ inline int window_quantized(int L, int S_sink, int S_keep, int S_flush)
+{
+    const int e = L - S_sink - S_keep;
+    return e > 0 ? (e / S_flush) * S_flush : 0;
+}
+
 // Where the positions of a (sequence, KV head) live: contiguous planes [B][Hkv][T_cap]
 // (table == nullptr) or pages [page][Hkv][page_tokens] through a block table
 // [B][T_cap / page_tokens].

@@ -80,6 +80,9 @@ def load():
                                               C.POINTER(_Window), _P, _I, _P, _I, _P, _S,
                                               _P, _P]
     L.kvq_decode_attention_window.restype = _I
+    L.kvq_window_append.argtypes = [_P, _P, _I, _P, _P, C.POINTER(_QParams), C.POINTER(_Cache),
+                                    C.POINTER(_Window), _P, _I, _P, _P]
+    L.kvq_window_append.restype = _I
     L.kvq_decode_attention_noalloc.argtypes = [_P, _I, _I, _P, C.POINTER(_Cache), _P, _I, _P,
                                                _I, _P, _P]
     L.kvq_bf16_decode_workspace_bytes.restype = _S
@@ -280,6 +283,34 @@ def decode_attention_window(q, Tk_invT, cache: KVCache, S_sink: int, S_keep: int
                                          int(max_seqlen), _ptr(out), _dt(out), _ptr(workspace),
                                          workspace.numel(), _ptr(dev_err), _stream(stream)),
            "kvq_decode_attention_window")
+
+
+def window_append(k_new, v_new, T_k, T_v, qp: QParams, cache: KVCache, S_sink: int,
+                  S_keep: int, S_flush: int, k_sink, v_sink, k_recent, v_recent, seqlens,
+                  n=None, dev_err=None, stream=None):
+    """kvq_window_append: append n bfloat16 tokens k_new, v_new [B][n][Hkv][d] to sequences
+    of seqlens (int32 [B], lengths before the call; not updated) with a full-precision
+    window: sink k_sink, v_sink [B][Hkv][S_sink][d] (None when S_sink = 0), recent ring
+    k_recent, v_recent [B][Hkv][S_keep + S_flush][d], positions leaving the window
+    quantized into the cache at position t - S_sink."""
+    L = load()
+    _cuda("k_new", k_new, torch.bfloat16)
+    _cuda("v_new", v_new, torch.bfloat16)
+    _cuda("T_k", T_k, torch.float32)
+    _cuda("T_v", T_v, torch.float32)
+    for name, t in (("k_sink", k_sink), ("v_sink", v_sink), ("k_recent", k_recent),
+                    ("v_recent", v_recent)):
+        _cuda(name, t, torch.bfloat16)
+    _cuda("seqlens", seqlens, torch.int32)
+    _cuda("dev_err", dev_err, torch.int32)
+    if n is None:
+        n = k_new.shape[1]
+    win = _Window(int(S_sink), int(S_keep), int(S_flush), _ptr(k_sink), _ptr(v_sink),
+                  _ptr(k_recent), _ptr(v_recent), None)
+    qpc = qp._c()
+    _check(L.kvq_window_append(_ptr(k_new), _ptr(v_new), KVQ_BF16, _ptr(T_k), _ptr(T_v),
+                               C.byref(qpc), C.byref(cache.desc), C.byref(win), _ptr(seqlens),
+                               int(n), _ptr(dev_err), _stream(stream)), "kvq_window_append")
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20

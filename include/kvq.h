@@ -216,10 +216,10 @@ typedef struct {
     int S_sink;
     int S_keep;
     int S_flush;                /* > 0 */
-    const void *k_sink;
-    const void *v_sink;
-    const void *k_recent;
-    const void *v_recent;
+    void *k_sink;               /* read by the decode, written by kvq_window_append */
+    void *v_sink;
+    void *k_recent;
+    void *v_recent;
     const float *T_v;
 } kvq_window;
 
@@ -240,6 +240,34 @@ KVQ_API kvq_status kvq_decode_attention_window(const void *q, kvq_dtype q_dtype,
                                                void *out, kvq_dtype out_dtype, void *workspace,
                                                size_t ws_bytes, int32_t *dev_err,
                                                kvq_stream_t stream);
+
+/*
+ * Write path with a full-precision window (WUSH-KV summary, section 4.4): append n new
+ * tokens to every sequence and quantize the positions that leave the window, so that the
+ * state afterwards is the one kvq_decode_attention_window reads for L + n positions.
+ *   k_new, v_new: bfloat16 [B][n][Hkv][d], post-RoPE keys and values of positions
+ *                 [L_b, L_b + n), L_b = seqlens[b] (device int32 [B], lengths BEFORE the
+ *                 call; the library does not update them).
+ *   window: S_sink, S_keep, S_flush and the sink / recent-ring buffers (written here);
+ *           T_v is not used (the values go through T_v in the quantizer).
+ *   T_k, T_v, qp, cache: as in kvq_quantize_append.
+ * Per sequence: new positions t < S_sink are copied to the sink; the positions
+ * [S_sink + Q(L_b), S_sink + Q(L_b + n)) (Q as above) are transformed, clipped, quantized
+ * and written at cache positions [Q(L_b), Q(L_b + n)), each read from the recent ring
+ * (t < L_b) or from the new tokens (t >= L_b); the new positions still in the window
+ * (t >= S_sink + Q(L_b + n)) are copied to ring slot t % (S_keep + S_flush). The flush
+ * reading is the one of the windowed decode: after every append, the oldest S_flush
+ * eligible positions are quantized while at least S_flush are eligible. The quantization
+ * uses the float32 CUDA-core transform; its codes equal those of kvq_quantize_append on
+ * the same tokens through that path (fewer than 256 tokens in one call).
+ * A sequence with L_b < 0 or Q(L_b + n) > T_cap is skipped and flagged
+ * (KVQ_DEVERR_POS_RANGE). All bf16 buffers 16-byte aligned. n == 0 is a no-op.
+ */
+KVQ_API kvq_status kvq_window_append(const void *k_new, const void *v_new, kvq_dtype in_dtype,
+                                     const float *T_k, const float *T_v, const kvq_qparams *qp,
+                                     kvq_cache *cache, const kvq_window *window,
+                                     const int32_t *seqlens, int n, int32_t *dev_err,
+                                     kvq_stream_t stream);
 
 /*
  * Allocation-free decode (no counterpart in the paper; an addition for callers that

@@ -174,6 +174,29 @@ def test_window_decode_argument_errors():
     assert kvq.load().kvq_last_error()
 
 
+def _window_append(desc, qp, win, dtype=1, n=1, k=0x5000, seqlens=0x7000):
+    L = kvq.load()
+    return L.kvq_window_append(k, 0x6000, dtype, None, None, C.byref(qp), C.byref(desc),
+                               None if win is None else C.byref(win), seqlens, n, None, None)
+
+
+def test_window_append_argument_errors():
+    desc, qp = _desc(T_cap=128)
+    assert _window_append(desc, qp, None) == 1                     # no window
+    assert _window_append(desc, qp, _win(S_flush=0)) == 1
+    assert _window_append(desc, qp, _win(S_sink=1024, S_keep=1024, S_flush=64)) == 2
+    assert _window_append(desc, qp, _win(kr=0)) == 1
+    assert _window_append(desc, qp, _win(), dtype=0) == 2          # float32 tokens
+    assert _window_append(desc, qp, _win(), n=-1) == 1
+    assert _window_append(desc, qp, _win(), k=0) == 1
+    assert _window_append(desc, qp, _win(), seqlens=0) == 1
+    assert _window_append(desc, qp, _win(), k=0x5002) == 1         # misaligned
+    other = K._QParams(4, 2, 128, 0.01)
+    assert _window_append(desc, other, _win()) == 1                # qparams differ
+    assert _window_append(desc, qp, _win(), n=0, k=0) == 0         # nothing to do
+    assert kvq.load().kvq_last_error() == b""
+
+
 def test_window_quantized_middle_matches_the_oracle_reading():
     import oracle
     # the library's host-side reading (through the capacity check) equals the oracle's:
