@@ -43,6 +43,12 @@ def lib():
         L.oracle_quantize_append.argtypes = [P, P, I, P, P, I, I, I, I, I, I, I, F, I, P,
                                              P, P, P, P, P, P]
         L.oracle_quantize_append.restype = I
+        L.oracle_quantize_append_q.argtypes = [P, P, I, P, P, I, I, I, I, I, I, I, F, I, I, P,
+                                               P, P, P, P, P, P]
+        L.oracle_quantize_append_q.restype = I
+        L.oracle_quantize_group_quest.argtypes = [P, I, I, P, P, P]
+        L.oracle_quest_delta.argtypes = [I]
+        L.oracle_quest_delta.restype = F
         L.oracle_pack_tokens.argtypes = [I] * 11 + [P] * 8
         L.oracle_pack_tokens.restype = I
         L.oracle_unpack_tokens.argtypes = [I] * 11 + [P] * 8
@@ -128,6 +134,21 @@ def quantize_group(x, bits: int, kap: int):
     s = np.zeros(1, np.uint16)
     z = np.zeros(1, np.uint16)
     lib().oracle_quantize_group(_p(x), x.shape[0], bits, kap, _p(codes), _p(s), _p(z))
+    return codes, int(s[0]), int(z[0])
+
+
+def quest_delta(bits: int) -> float:
+    """The QuEST INT step in units of the group RMS (float32)."""
+    return float(lib().oracle_quest_delta(int(bits)))
+
+
+def quantize_group_quest(x, bits: int):
+    """QuEST INT codes (uint8 [g]), s_h, z_h (float16 bit patterns) of one group."""
+    x = _c(x, np.float32)
+    codes = np.empty(x.shape[0], np.uint8)
+    s = np.zeros(1, np.uint16)
+    z = np.zeros(1, np.uint16)
+    lib().oracle_quantize_group_quest(_p(x), x.shape[0], bits, _p(codes), _p(s), _p(z))
     return codes, int(s[0]), int(z[0])
 
 
@@ -251,8 +272,9 @@ class Cache:
 # ------------------------------------------------------------------ write path
 
 def quantize_append(k, v, T_k, T_v, bits_k, bits_v, group, clip_alpha, cache: Cache, pos,
-                    return_transformed=False):
-    """k, v: [B][n][Hkv][d] float32 or bf16 bits; T_k/T_v float32 [Hkv][d][d] or None."""
+                    return_transformed=False, quantizer=0):
+    """k, v: [B][n][Hkv][d] float32 or bf16 bits; T_k/T_v float32 [Hkv][d][d] or None.
+    quantizer 0 = percentile-clipped affine, 1 = QuEST INT (clip_alpha unused)."""
     dt = _dt(k)
     assert _dt(v) == dt
     k, v = np.ascontiguousarray(k), np.ascontiguousarray(v)
@@ -262,8 +284,9 @@ def quantize_append(k, v, T_k, T_v, bits_k, bits_v, group, clip_alpha, cache: Ca
     pos = _c(pos, np.int32)
     kt = np.empty((B, n, Hkv, d), np.float32) if return_transformed else None
     vt = np.empty((B, n, Hkv, d), np.float32) if return_transformed else None
-    r = lib().oracle_quantize_append(_p(k), _p(v), dt, _p(Tk), _p(Tv), B, n, Hkv, d, bits_k,
-                                     bits_v, group, float(clip_alpha), cache.T_cap, _p(pos),
+    r = lib().oracle_quantize_append_q(_p(k), _p(v), dt, _p(Tk), _p(Tv), B, n, Hkv, d, bits_k,
+                                     bits_v, group, float(clip_alpha), int(quantizer),
+                                     cache.T_cap, _p(pos),
                                      _p(cache.k_codes), _p(cache.k_sz), _p(cache.v_codes),
                                      _p(cache.v_sz), _p(kt), _p(vt))
     if r:

@@ -195,6 +195,60 @@ void oracle_quantize_group(const float *x, int g, int bits, int kappa,
     *z_h = zh;
 }
 
+/*
+ * QuEST INT quantizer ("WUSH-KV: KV Cache Quantization with Data-Adaptive Transforms",
+ * section 4.3 and the attention-stage comparison of section 5.1): each token's group of
+ * channels is quantized with RMS-based clipped levels. The page gives no constants; the
+ * reading here: a symmetric uniform grid of 2^b levels at (c - (2^b - 1)/2) * step,
+ * c = 0 .. 2^b - 1, with step = delta_b * RMS(x), delta_b the uniform step that minimises
+ * the mean squared error for a unit Gaussian (Max, 1960: 0.9957 for 4 levels, 0.3352 for
+ * 16 levels); values beyond the outer levels clip to them. In the cache's affine form:
+ *   ms  = sum_j x_j^2 / g                      (float64)
+ *   rms = f32(sqrt(ms))
+ *   s   = f32(rms * delta_b)                   (float32 product, delta_b a float32 constant)
+ *   s_h = f16(s),  z_h = f16(-(2^b - 1)/2 * s_h)   (the product is exact in float32)
+ *   c   = clamp(rint(f32(f32(x - z) / s)), 0, 2^b - 1) with z, s read back from f16, as
+ *         the percentile quantizer; s_h == 0 gives all codes 0.
+ * The decode is unchanged: x^ = z_h + c s_h.
+ */
+float oracle_quest_delta(int bits)
+{
+    return bits == 2 ? 0.9957f : bits == 4 ? 0.3352f : 0.0f;
+}
+
+void oracle_quantize_group_quest(const float *x, int g, int bits, uint8_t *codes, uint16_t *s_h,
+                                 uint16_t *z_h)
+{
+    double ms = 0.0;
+    for (int i = 0; i < g; ++i)
+        ms += (double)x[i] * (double)x[i];
+    ms /= (double)g;
+    float rms = (float)sqrt(ms);
+    int qmax = (1 << bits) - 1;
+    float s = f32((double)rms * (double)oracle_quest_delta(bits));
+    uint16_t sh = oracle_f32_to_f16(s);
+    double sf = oracle_f16_to_f64(sh);
+    float zq = f32(-0.5 * (double)qmax * sf);
+    uint16_t zh = oracle_f32_to_f16(zq);
+    double zf = oracle_f16_to_f64(zh);
+    for (int i = 0; i < g; ++i) {
+        int c = 0;
+        if (sf != 0.0) {
+            float diff = f32((double)x[i] - zf);
+            float y = f32((double)diff / sf);
+            double r = rint((double)y);
+            if (r < 0)
+                r = 0;
+            if (r > qmax)
+                r = qmax;
+            c = (int)r;
+        }
+        codes[i] = (uint8_t)c;
+    }
+    *s_h = sh;
+    *z_h = zh;
+}
+
 /* ------------------------------------------------------------------ cache layout */
 /*
  * Fixed width per token ("Spend Bits Where Queries Look", Three requirements, item 3).
@@ -371,6 +425,14 @@ static double load_in(const void *p, int dtype, size_t i)
  * kt_out / vt_out (nullable): the float32 transformed inputs, [B][n][Hkv][d].
  * Returns 0, or -1 on an argument error.
  */
+int oracle_quantize_append_q(const void *k, const void *v, int in_dtype,
+                             const float *T_k, const float *T_v,
+                             int B, int n, int Hkv, int d, int bits_k, int bits_v, int group,
+                             float clip_alpha, int quantizer, int T_cap, const int32_t *pos,
+                             uint8_t *k_codes, uint16_t *k_sz, uint8_t *v_codes, uint16_t *v_sz,
+                             float *kt_out, float *vt_out);
+
+/* The percentile-clipped quantizer (quantizer 0); see oracle_quantize_append_q. */
 int oracle_quantize_append(const void *k, const void *v, int in_dtype,
                            const float *T_k, const float *T_v,
                            int B, int n, int Hkv, int d, int bits_k, int bits_v, int group,
@@ -378,6 +440,22 @@ int oracle_quantize_append(const void *k, const void *v, int in_dtype,
                            uint8_t *k_codes, uint16_t *k_sz, uint8_t *v_codes, uint16_t *v_sz,
                            float *kt_out, float *vt_out)
 {
+    return oracle_quantize_append_q(k, v, in_dtype, T_k, T_v, B, n, Hkv, d, bits_k, bits_v,
+                                    group, clip_alpha, 0, T_cap, pos, k_codes, k_sz, v_codes,
+                                    v_sz, kt_out, vt_out);
+}
+
+/* quantizer: 0 = percentile-clipped affine (OSCAR-style, clip_alpha), 1 = QuEST INT
+ * (RMS-based symmetric grid, clip_alpha unused). */
+int oracle_quantize_append_q(const void *k, const void *v, int in_dtype,
+                             const float *T_k, const float *T_v,
+                             int B, int n, int Hkv, int d, int bits_k, int bits_v, int group,
+                             float clip_alpha, int quantizer, int T_cap, const int32_t *pos,
+                             uint8_t *k_codes, uint16_t *k_sz, uint8_t *v_codes, uint16_t *v_sz,
+                             float *kt_out, float *vt_out)
+{
+    if (quantizer != 0 && quantizer != 1)
+        return -1;
     if (d <= 0 || d > 1024 || group <= 0 || d % group || (bits_k != 2 && bits_k != 4) ||
         (bits_v != 2 && bits_v != 4) || T_cap % 16 || d % 64 ||
         2 * oracle_kappa(clip_alpha, group) >= group)
@@ -421,9 +499,14 @@ int oracle_quantize_append(const void *k, const void *v, int in_dtype,
             if (dump)
                 memcpy(dump + base, xf, sizeof(float) * d);
             int kappa = oracle_kappa(clip_alpha, group);
-            for (int gr = 0; gr < ng; ++gr)
-                oracle_quantize_group(xf + gr * group, group, bits, kappa, codes + gr * group,
-                                      &sz[2 * gr], &sz[2 * gr + 1]);
+            for (int gr = 0; gr < ng; ++gr) {
+                if (quantizer == 1)
+                    oracle_quantize_group_quest(xf + gr * group, group, bits, codes + gr * group,
+                                                &sz[2 * gr], &sz[2 * gr + 1]);
+                else
+                    oracle_quantize_group(xf + gr * group, group, bits, kappa, codes + gr * group,
+                                          &sz[2 * gr], &sz[2 * gr + 1]);
+            }
             store_token(&c, which, b, h, pos[b] + i, codes, sz);
         }
     }

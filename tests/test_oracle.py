@@ -439,3 +439,111 @@ def test_end_to_end_chain_against_numpy_restatement():
     for hq in range(4):
         want = _two_pass(q[0, hq].astype(np.float64), Tit[0].astype(np.float64), kh, vh, 90, 128)
         np.testing.assert_allclose(out[0, hq], want, rtol=1e-11, atol=1e-12)
+
+
+# ----------------------------------------------------------------- QuEST INT quantizer
+# ("WUSH-KV: KV Cache Quantization with Data-Adaptive Transforms", section 4.3)
+
+def test_quest_hand_worked_examples():
+    n = 0
+    for bits, xs, sh, zh, codes, packed in _rows("quest_hand_worked.txt"):
+        x = np.array([float(v) for v in xs.split()], np.float32)
+        c, s, z = oracle.quantize_group_quest(x, int(bits))
+        assert s == int(sh, 16), (xs, hex(s))
+        assert z == int(zh, 16), (xs, hex(z))
+        assert c.tolist() == [int(v) for v in codes.split()]
+        assert oracle.pack_k_row(c, int(bits)).tolist() == [int(v, 16) for v in packed.split()]
+        n += 1
+    assert n == 4
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_quest_step_minimises_the_gaussian_mse(bits):
+    """The step constant is the uniform step with the least mean squared error for a unit
+    Gaussian, found here by numerical integration and minimisation (independent of the
+    oracle and of any table): 2^b levels at (c - (2^b - 1)/2) step, cells split at the
+    midpoints, the outer cells open."""
+    from scipy import integrate, optimize, stats
+    N = 1 << bits
+
+    def mse(step):
+        levels = (np.arange(N) - (N - 1) / 2) * step
+        edges = np.concatenate([[-np.inf], (levels[:-1] + levels[1:]) / 2, [np.inf]])
+        tot = 0.0
+        for c in range(N):
+            f = lambda x, y=levels[c]: (x - y) ** 2 * stats.norm.pdf(x)
+            tot += integrate.quad(f, edges[c], edges[c + 1])[0]
+        return tot
+    best = optimize.minimize_scalar(mse, bounds=(0.05, 2.0), method="bounded",
+                                    options={"xatol": 1e-7}).x
+    assert abs(best - oracle.quest_delta(bits)) < 5e-4, best
+
+
+@pytest.mark.parametrize("bits,mse_opt", [(2, 0.1188), (4, 0.01154)])
+def test_quest_gaussian_mse_is_the_textbook_optimum(bits, mse_opt):
+    """On unit-Gaussian groups of 128 the quantizer's mean squared error is close to the
+    optimal uniform quantizer's (Max 1960: 0.1188 for 4 levels, 0.01154 for 16); the
+    per-group RMS keeps it a few percent lower (a sample's largest values sit closer to
+    its own RMS, fewer overload errors). A grid shifted by half a step, a missing clip or
+    a wrong RMS moves it far outside 6%."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((3000, 128)).astype(np.float32)
+    err = 0.0
+    for row in x:
+        c, sh, zh = oracle.quantize_group_quest(row, bits)
+        s, z = oracle.f16_bits_to_f64([sh, zh])
+        err += np.sum((row.astype(np.float64) - (z + c * s)) ** 2)
+    mse = err / x.size
+    assert abs(mse - mse_opt) / mse_opt < 0.06, mse
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_quest_grid_and_error_bound(bits):
+    """Levels sit symmetrically (up to the float16 zero-point) around 0 with step
+    delta_b * rms; entries inside the grid are within s/2 of their reconstruction, entries
+    outside clip to the outer level."""
+    rng = np.random.default_rng(6 + bits)
+    qmax = (1 << bits) - 1
+    for _ in range(200):
+        g = int(rng.choice([32, 64, 128]))
+        x = (rng.standard_normal(g) * rng.lognormal(0, 2)).astype(np.float32)
+        c, sh, zh = oracle.quantize_group_quest(x, bits)
+        s, z = oracle.f16_bits_to_f64([sh, zh])
+        rms = np.float32(np.sqrt(np.mean(x.astype(np.float64) ** 2)))
+        s_ref = np.float32(rms * np.float32(oracle.quest_delta(bits)))
+        assert abs(s - s_ref) <= s_ref * 2.0 ** -11                      # f16 rounding of s
+        assert abs(z + qmax / 2 * s) <= abs(z) * 2.0 ** -11 + 1e-30     # z = -(2^b-1)/2 s
+        xh = z + c * s
+        inside = (x >= z) & (x <= z + qmax * s)
+        assert np.all(np.abs(x[inside] - xh[inside]) <= s / 2 * (1 + 2.0 ** -20))
+        assert np.all(c[x < z] == 0) and np.all(c[x > z + qmax * s] == qmax)
+
+
+def test_quest_scale_invariance():
+    """Scaling a group by a power of two scales s_h and z_h by it and keeps every code."""
+    rng = np.random.default_rng(9)
+    for bits in (2, 4):
+        for _ in range(50):
+            x = rng.standard_normal(64).astype(np.float32)
+            c0, s0, z0 = oracle.quantize_group_quest(x, bits)
+            c1, s1, z1 = oracle.quantize_group_quest(x * np.float32(8.0), bits)
+            a0, b0 = oracle.f16_bits_to_f64([s0, z0])
+            a1, b1 = oracle.f16_bits_to_f64([s1, z1])
+            assert np.array_equal(c0, c1) and a1 == 8 * a0 and b1 == 8 * b0
+
+
+def test_quest_append_uses_the_groupwise_quantizer():
+    """quantize_append with quantizer 1 stores exactly the QuEST codes and (s, z) of each
+    transformed token group."""
+    rng = np.random.default_rng(10)
+    k = rng.standard_normal((1, 5, 2, 128)).astype(np.float32)
+    v = rng.standard_normal((1, 5, 2, 128)).astype(np.float32)
+    oc = oracle.Cache(1, 2, 64, 128, 4, 2, 128)
+    oracle.quantize_append(k, v, None, None, 4, 2, 128, 0.0, oc, [3], quantizer=1)
+    for h in range(2):
+        kc, vc, ksz, vsz = oc.unpack_tokens(0, h, 3, 5)
+        for i in range(5):
+            c, s, z = oracle.quantize_group_quest(k[0, i, h], 4)
+            assert kc[i].tolist() == c.tolist() and ksz[i, 0].tolist() == [s, z]
+            c, s, z = oracle.quantize_group_quest(v[0, i, h], 2)
+            assert vc[i].tolist() == c.tolist() and vsz[i, 0].tolist() == [s, z]
