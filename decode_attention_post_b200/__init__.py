@@ -12,6 +12,8 @@ from .kvq import (  # noqa: F401
     KVQ_DEVERR_POS_RANGE,
     KVQ_DEVERR_SEQLEN_CLAMPED,
     KVQ_DEVERR_WAIT_TIMEOUT,
+    KVQ_QUANT_PERCENTILE,
+    KVQ_QUANT_QUEST,
     KvqError,
     KVCache,
     QParams,

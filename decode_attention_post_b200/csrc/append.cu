@@ -10,7 +10,8 @@
 //   2. Each warp transforms 4 tokens: lane l owns output dims l + 32r, so the d x d
 //      product is register-tiled 4 tokens x d/32 dims with fused multiply-add.
 //   3. Per group, the order statistics x_(kappa) and x_(g-1-kappa) come from kappa+1
-//      rounds of a warp-wide min (max) with removal of one instance (exact, ties safe).
+//      rounds of a warp-wide min (max) with removal of one instance (exact, ties safe);
+//      for the QuEST INT quantizer, the group RMS from a float64 sum of squares.
 //   4. Scale, zero-point and codes use IEEE float32 division (__fdiv_rn) and rintf
 //      (ties to even), so they match the float64 definition bit for bit.
 //   5. Codes are gathered through shared memory and written as whole 32-bit words
@@ -280,21 +281,41 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
                 // group gr covers dims [gr*group, (gr+1)*group), i.e. r in [r0, r0+nr);
                 // dims outside the group are padded with +-inf so they are never picked.
                 const int r0 = gr * group / 32, nr = group / 32;
-                float vmin[R], vmax[R];
+                __half sh, zh;
+                bool finite;
+                if (kappa == kQuestClip) {
+                    // QuEST INT: s = f32(rms * delta_b), z = -(2^b - 1)/2 * s_h; the sum of
+                    // squares in float64 (each square exact), reduced over the warp
+                    double ss = 0.0;
 #pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const bool ing = r >= r0 && r < r0 + nr;
-                    vmin[r] = ing ? acc[q][r] : INFINITY;
-                    vmax[r] = ing ? acc[q][r] : -INFINITY;
+                    for (int r = 0; r < R; ++r)
+                        if (r >= r0 && r < r0 + nr)
+                            ss = fma((double)acc[q][r], (double)acc[q][r], ss);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1)
+                        ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                    const float rms = __double2float_rn(sqrt(ss / (double)group));
+                    const float s = __fmul_rn(rms, quest_delta(bits));
+                    sh = __float2half_rn(s);
+                    zh = __float2half_rn(__fmul_rn(-0.5f * (float)qmax, __half2float(sh)));
+                    finite = isfinite(s);
+                } else {
+                    float vmin[R], vmax[R];
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const bool ing = r >= r0 && r < r0 + nr;
+                        vmin[r] = ing ? acc[q][r] : INFINITY;
+                        vmax[r] = ing ? acc[q][r] : -INFINITY;
+                    }
+                    const float lo = order_stat<R, false>(vmin, kappa, lane);
+                    const float hi = order_stat<R, true>(vmax, kappa, lane);
+                    const float range = __fsub_rn(hi, lo);
+                    const float s = __fdiv_rn(range, (float)qmax);
+                    sh = __float2half_rn(s);
+                    zh = __float2half_rn(lo);
+                    finite = isfinite(range) && isfinite(s);
                 }
-                const float lo = order_stat<R, false>(vmin, kappa, lane);
-                const float hi = order_stat<R, true>(vmax, kappa, lane);
-                const float range = __fsub_rn(hi, lo);
-                const float s = __fdiv_rn(range, (float)qmax);
-                const __half sh = __float2half_rn(s);
-                const __half zh = __float2half_rn(lo);
                 const float sf = __half2float(sh), zf = __half2float(zh);
-                const bool finite = isfinite(range) && isfinite(s);
                 if (!finite && lane == 0)
                     flag(dev_err, KVQ_DEVERR_NONFINITE);
 #pragma unroll

@@ -10,7 +10,8 @@
 //   X~[16 tok x d] = X[16 x d] . (T_hi + T_lo)^T on mma.sync m16n8k16 (bf16, f32 acc);
 //   the inputs are bfloat16, so X is exact and only T is split.
 //   Each token's d values sit in the 4 lanes of a quad: order statistics by a quad-wide
-//   min/max (kappa = 0) or a top-2 merge (kappa = 1) or kappa+1 extraction rounds.
+//   min/max (kappa = 0) or a top-2 merge (kappa = 1) or kappa+1 extraction rounds; the
+//   QuEST INT quantizer takes the group RMS from a float64 sum of squares instead.
 //   s = f32(f32(hi - lo) / qmax), s_h = f16(s), z_h = f16(lo), as the definition; codes
 //   c = clamp(rint(f32(x - z)/s)) computed as (x - z) * rcp_rn(s), which differs from the
 //   IEEE quotient by under 2 ulp; a value within 2^-20 of a rounding tie is recomputed
@@ -285,8 +286,22 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
             uint32_t cq[NV];                          // codes of this lane's columns
             for (int gr = 0; gr < ng; ++gr) {
                 const int c0 = gr * group, c1 = c0 + group;    // columns of this group
-                float lo, hi;
-                if (kappa == 0) {
+                float lo = 0.f, hi = 0.f;
+                float quest_s = 0.f;
+                if (kappa == kQuestClip) {
+                    // QuEST INT: float64 sum of squares of the group over the quad
+                    double ss = 0.0;
+#pragma unroll
+                    for (int e = 0; e < NV; ++e) {
+                        const int col = 8 * (e >> 1) + 2 * t + (e & 1);
+                        if (col >= c0 && col < c1)
+                            ss = fma((double)x[e], (double)x[e], ss);
+                    }
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+                    const float rms = __double2float_rn(sqrt(ss / (double)group));
+                    quest_s = __fmul_rn(rms, quest_delta(bits));
+                } else if (kappa == 0) {
                     lo = INFINITY;
                     hi = -INFINITY;
 #pragma unroll
@@ -337,12 +352,20 @@ append_mma_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *_
                     lo = quad_order_stat<NV, false>(vmin, kappa, lane);
                     hi = quad_order_stat<NV, true>(vmax, kappa, lane);
                 }
-                const float range = __fsub_rn(hi, lo);
-                const float s = __fdiv_rn(range, (float)qmax);
-                const __half sh = __float2half_rn(s);
-                const __half zh = __float2half_rn(lo);
+                __half sh, zh;
+                bool finite;
+                if (kappa == kQuestClip) {
+                    sh = __float2half_rn(quest_s);
+                    zh = __float2half_rn(__fmul_rn(-0.5f * (float)qmax, __half2float(sh)));
+                    finite = isfinite(quest_s);
+                } else {
+                    const float range = __fsub_rn(hi, lo);
+                    const float s = __fdiv_rn(range, (float)qmax);
+                    sh = __float2half_rn(s);
+                    zh = __float2half_rn(lo);
+                    finite = isfinite(range) && isfinite(s);
+                }
                 const float sf = __half2float(sh), zf = __half2float(zh);
-                const bool finite = isfinite(range) && isfinite(s);
                 if (ok && !finite && t == 0)
                     flag(dev_err, KVQ_DEVERR_NONFINITE);
                 const bool zero = !finite || sf == 0.f;

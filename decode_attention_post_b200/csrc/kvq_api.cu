@@ -46,6 +46,13 @@ static int kappa_of(float alpha, int group)
     return k < 0 ? 0 : (int)k;
 }
 
+// What the append kernels take as their clip parameter: the order-statistic index of the
+// percentile quantizer, or kQuestClip for the QuEST INT quantizer.
+static int clip_param(const kvq_qparams *qp)
+{
+    return qp->quantizer == KVQ_QUANT_QUEST ? kQuestClip : kappa_of(qp->clip_alpha, qp->group);
+}
+
 static kvq_status check_qparams(const kvq_qparams *qp, int d)
 {
     if (!qp)
@@ -56,6 +63,11 @@ static kvq_status check_qparams(const kvq_qparams *qp, int d)
     if (qp->group <= 0 || d % qp->group || qp->group % 32)
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "group=%d must divide d=%d and be a multiple of 32",
                  qp->group, d);
+    if (qp->quantizer != KVQ_QUANT_PERCENTILE && qp->quantizer != KVQ_QUANT_QUEST)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "quantizer=%d is not KVQ_QUANT_PERCENTILE or KVQ_QUANT_QUEST",
+                 qp->quantizer);
+    if (qp->quantizer == KVQ_QUANT_QUEST)
+        return KVQ_OK;                         // clip_alpha is not used
     if (!(qp->clip_alpha >= 0.f) || !(qp->clip_alpha < 0.5f))
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "clip_alpha=%g must be in [0, 0.5)", (double)qp->clip_alpha);
     const int kap = kappa_of(qp->clip_alpha, qp->group);
@@ -102,7 +114,8 @@ static kvq_status check_cache(const kvq_cache *c)
 static bool same_qp(const kvq_qparams *a, const kvq_qparams *b)
 {
     return a->bits_k == b->bits_k && a->bits_v == b->bits_v && a->group == b->group &&
-           a->clip_alpha == b->clip_alpha;
+           a->quantizer == b->quantizer &&
+           (a->quantizer == KVQ_QUANT_QUEST || a->clip_alpha == b->clip_alpha);
 }
 
 static int num_sms()
@@ -265,7 +278,7 @@ kvq_status kvq_quantize_append(const void *k, const void *v, kvq_dtype in_dtype,
     if (!k || !v || !pos)
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "k, v and pos must not be NULL");
     cudaError_t e = append_launch(k, v, in_dtype == KVQ_BF16, T_k, T_v, cache->B, n, cache,
-                                kappa_of(qp->clip_alpha, qp->group), pos, dev_err,
+                                clip_param(qp), pos, dev_err,
                                 (cudaStream_t)stream);
     if (e != cudaSuccess)
         KVQ_FAIL(KVQ_ERR_CUDA, "append launch: %s", cudaGetErrorString(e));
@@ -436,7 +449,7 @@ kvq_status kvq_window_append(const void *k_new, const void *v_new, kvq_dtype in_
     cudaStream_t st = (cudaStream_t)stream;
     // the flush reads ring slots that the store below may overwrite: flush first
     cudaError_t e = window_flush_launch(k_new, v_new, T_k, T_v, cache->B, n, cache,
-                                        kappa_of(qp->clip_alpha, qp->group), win->k_recent,
+                                        clip_param(qp), win->k_recent,
                                         win->v_recent, seqlens, win->S_sink, win->S_keep,
                                         win->S_flush, dev_err, st);
     if (e != cudaSuccess)

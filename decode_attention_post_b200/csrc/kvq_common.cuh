@@ -11,6 +11,14 @@
 namespace kvq {
 
 constexpr int kTileTokens = 16;      // V codes are stored in 16-token tiles
+constexpr int kQuestClip = -1;       // clip parameter of the append kernels: QuEST INT
+
+// QuEST INT step in units of the group RMS: the uniform step of least mean squared
+// error for a unit Gaussian with 2^bits levels (4 levels: 0.9957, 16 levels: 0.3352).
+__host__ __device__ inline float quest_delta(int bits)
+{
+    return bits == 2 ? 0.9957f : 0.3352f;
+}
 constexpr int kCapAlign = 64;        // T_cap granularity (whole decode blocks)
 
 // Bits of the device error word (see kvq.h).

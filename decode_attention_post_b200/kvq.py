@@ -19,6 +19,7 @@ _LIB_PATH = os.path.join(_HERE, "libkvq.so")
 _lib = None
 
 KVQ_F32, KVQ_BF16 = 0, 1
+KVQ_QUANT_PERCENTILE, KVQ_QUANT_QUEST = 0, 1
 KVQ_DEVERR_SEQLEN_CLAMPED = 0x1
 KVQ_DEVERR_POS_RANGE = 0x2
 KVQ_DEVERR_NONFINITE = 0x4
@@ -29,7 +30,8 @@ _P, _I, _F, _S = C.c_void_p, C.c_int, C.c_float, C.c_size_t
 
 
 class _QParams(C.Structure):
-    _fields_ = [("bits_k", _I), ("bits_v", _I), ("group", _I), ("clip_alpha", _F)]
+    _fields_ = [("bits_k", _I), ("bits_v", _I), ("group", _I), ("clip_alpha", _F),
+                ("quantizer", _I)]
 
 
 class _Cache(C.Structure):
@@ -131,13 +133,15 @@ def _cuda(name, t, dtype=None):
 
 @dataclasses.dataclass(frozen=True)
 class QParams:
+    """kvq_qparams: quantizer KVQ_QUANT_PERCENTILE (clip_alpha used) or KVQ_QUANT_QUEST."""
     bits_k: int = 2
     bits_v: int = 2
     group: int = 128
     clip_alpha: float = 0.01
+    quantizer: int = KVQ_QUANT_PERCENTILE
 
     def _c(self):
-        return _QParams(self.bits_k, self.bits_v, self.group, self.clip_alpha)
+        return _QParams(self.bits_k, self.bits_v, self.group, self.clip_alpha, self.quantizer)
 
 
 class KVCache:

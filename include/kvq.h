@@ -75,23 +75,38 @@ typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
                                            append skips the token, the decode reads page 0 */
 
 /*
- * Quantizer parameters (WUSH-KV summary, section 5.3; percentile clipping).
- * For a group of `group` consecutive dims of one token, with kappa = floor(clip_alpha *
- * (group - 1)) computed in double on the host:
+ * Quantizer parameters. Two quantizers write the same cache format (x^ = z_h + c s_h):
+ *
+ * quantizer = KVQ_QUANT_PERCENTILE (0): OSCAR-style percentile-clipped affine quantizer
+ * (WUSH-KV summary, section 5.3). For a group of `group` consecutive dims of one token,
+ * with kappa = floor(clip_alpha * (group - 1)) computed in double on the host:
  *   lo = x_(kappa), hi = x_(group-1-kappa)          order statistics, 0-indexed ascending
  *   s  = f32(f32(hi - lo) / (2^bits - 1))           IEEE float32 division
  *   s_h = f16_rn(s), z_h = f16_rn(lo)               stored as the pair (s_h, z_h)
  *   c  = clamp(rint(f32(f32(x - z_h) / s_h)), 0, 2^bits - 1), rint ties-to-even;
  *        s_h == 0 gives c = 0 for the whole group.
- * Dequantization is x^ = z_h + c * s_h.
- * Supported: bits_k, bits_v in {2, 4}; group divides d and is a multiple of 32;
- * 0 <= kappa <= 8 and 2*kappa < group.
+ * Dequantization is x^ = z_h + c * s_h. Supported: 0 <= kappa <= 8 and 2*kappa < group.
+ *
+ * quantizer = KVQ_QUANT_QUEST (1): QuEST INT, RMS-based clipped levels (WUSH-KV summary,
+ * section 4.3; each token's group of channels quantized on its own). The page gives no
+ * constants; this library's reading is a symmetric uniform grid of 2^bits levels whose
+ * step is delta_b times the group RMS, delta_b the uniform step of least mean squared
+ * error for a unit Gaussian (0.9957 at 2 bits, 0.3352 at 4 bits):
+ *   rms = f32(sqrt(sum_j x_j^2 / group))            sum of squares in float64
+ *   s   = f32(rms * delta_b),  s_h = f16_rn(s),  z_h = f16_rn(-(2^bits - 1)/2 * s_h)
+ *   c   = clamp(rint(f32(f32(x - z_h) / s_h)), 0, 2^bits - 1)  as above.
+ * clip_alpha is not used.
+ *
+ * Supported: bits_k, bits_v in {2, 4}; group divides d and is a multiple of 32.
  */
+#define KVQ_QUANT_PERCENTILE 0
+#define KVQ_QUANT_QUEST      1
 typedef struct {
     int bits_k;
     int bits_v;
     int group;
     float clip_alpha;
+    int quantizer;              /* KVQ_QUANT_PERCENTILE or KVQ_QUANT_QUEST */
 } kvq_qparams;
 
 /*
