@@ -36,7 +36,7 @@ METRIC = "2-bit KV decode attention: achieved HBM GB/s and % of B200 peak; appen
 CONFIG_IDX = 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one decode_kernel launch on this workload
 # (ncu --set full --clock-control none, profiles directory); None once the kernel changes.
-DECODE_TRAFFIC_BYTES = None
+DECODE_TRAFFIC_BYTES = 546872832
 DECODE_TRAFFIC_KERNEL = "decode_kernel<128,4,2,2>"
 APPEND_CONFIG_IDX = 4
 DECODE_CONFIGS = (1, 3, 4)       # further decode shapes timed as extras

@@ -20,6 +20,8 @@
 //      comes from the contiguous layout or, for a paged cache, the block table.
 #include "kvq_common.cuh"
 
+#include <stdlib.h>
+
 namespace kvq {
 
 namespace {
@@ -438,9 +440,14 @@ cudaError_t window_flush_launch(const void *k_new, const void *v_new, const floa
                                       dev_err, st, tm);
 }
 
-// Chunks of bfloat16 inputs with both transforms go to the tensor-core kernel; float32
-// inputs, identity transforms, small (decode-time) appends and unaligned inputs use the
-// float32 CUDA-core kernel.
+cudaError_t append_tc(const void *k, const void *v, const float *Tk, const float *Tv, int B, int n,
+                      const kvq_cache *c, int clip, const int32_t *pos, int32_t *dev_err,
+                      cudaStream_t st);
+
+// Chunks of bfloat16 inputs with both transforms go to the tcgen05 tensor-core kernel
+// (KVQ_APPEND_PATH=mma selects the warp-level mma.sync kernel instead, for comparison);
+// float32 inputs, identity transforms, small (decode-time) appends and unaligned inputs
+// use the float32 CUDA-core kernel.
 cudaError_t append_launch(const void *k, const void *v, int in_bf16, const float *Tk,
                           const float *Tv, int B, int n, const kvq_cache *c, int kappa,
                           const int32_t *pos, int32_t *dev_err, cudaStream_t st)
@@ -448,8 +455,12 @@ cudaError_t append_launch(const void *k, const void *v, int in_bf16, const float
     const long tokens = (long)B * n;
     const bool a16 = ((uintptr_t)k % 16 == 0) && ((uintptr_t)v % 16 == 0) &&
                      ((uintptr_t)Tk % 16 == 0) && ((uintptr_t)Tv % 16 == 0);
-    if (in_bf16 && Tk && Tv && a16 && tokens >= 256)
-        return append_mma(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
+    if (in_bf16 && Tk && Tv && a16 && tokens >= 256) {
+        const char *path = getenv("KVQ_APPEND_PATH");
+        if ((path && path[0] == 'm') || tokens > 0x7fffff00L)
+            return append_mma(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
+        return append_tc(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
+    }
     const bool small = tokens <= 2048;
     if (c->d == 64)
         return small ? launch_append_fp32<64, 1>(k, v, in_bf16, Tk, Tv, B, n, c, kappa, pos, dev_err, st)

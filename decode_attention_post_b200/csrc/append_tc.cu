@@ -1,0 +1,560 @@
+// Write path for chunks of bfloat16 keys/values on the 5th-generation tensor cores
+// ("WUSH-KV: KV Cache Quantization with Data-Adaptive Transforms", sections 4.2, 4.3 and
+// 5.3; "Spend Bits Where Queries Look", "Three requirements", item 3).
+//
+// CTA = (KV head, one of {K, V}, slice of the 128-token tiles of the flattened
+// (sequence, new token) list), 6 warps with fixed roles:
+//   warp 4, one lane   TMA: each 128-token input tile [128 x d] bf16 lands in a 3-stage
+//                      shared-memory ring in the 128-byte-swizzled K-major layout (3-D
+//                      tensor map over [tokens][Hkv][d], no multicast);
+//   warp 5, one lane   tcgen05.mma: X~[128 x d] = X . T_hi^T + X . T_lo^T into one float32
+//                      TMEM accumulator (T split into two bfloat16 pieces, 16 significant
+//                      bits; X is bfloat16, hence exact), M = 128, N = d, K = 16 per
+//                      instruction; two accumulator buffers so that the next tile's MMAs
+//                      overlap this tile's epilogue;
+//   warps 0-3          epilogue: thread r owns token r of the tile; tcgen05.ld brings its
+//                      d transformed values into registers, then per group the clip range
+//                      (order statistics, or the RMS for the QuEST INT quantizer), the
+//                      float16 scale and zero-point, the codes (reciprocal multiply with an
+//                      IEEE-division fallback within 2^-20 of a rounding tie, so the codes
+//                      are those of the definition bit for bit) and the fixed-width stores
+//                      (one K row, or the token's halves of its 16-token V tile).
+// T (the B operand, N = d output dims x K = d input dims, K-major) is converted and
+// swizzled into shared memory once per CTA. Every wait is bounded; a wait that gives up
+// flags KVQ_DEVERR_WAIT_TIMEOUT, the CTA waits (bounded) for its copies and MMAs in flight,
+// frees its TMEM and stops.
+#include "kvq_common.cuh"
+#include "kvq_ptx.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+namespace kvq {
+
+namespace {
+
+constexpr int kTcTile = 128;                       // tokens per tile (MMA M)
+constexpr int kTcEpiWarps = 4;
+constexpr int kTcThreads = (kTcEpiWarps + 2) * 32; // epilogue warps + TMA warp + MMA warp
+constexpr int kTcStages = 3;
+constexpr int kTcKBlock = 64;                      // bf16 per 128-byte swizzled row
+
+template <int D>
+struct TcCfg {
+    static constexpr int KB = D / kTcKBlock;                  // 128-byte K blocks
+    static constexpr int A_BLOCK = kTcTile * kTcKBlock * 2;   // 16 KB: one K block of a tile
+    static constexpr int A_BYTES = KB * A_BLOCK;              // one input stage
+    static constexpr int B_BLOCK = D * kTcKBlock * 2;         // one K block of T_hi or T_lo
+    static constexpr int B_BYTES = KB * B_BLOCK;
+    static constexpr int OFF_B_HI = kTcStages * A_BYTES;
+    static constexpr int OFF_B_LO = OFF_B_HI + B_BYTES;
+    static constexpr int OFF_BAR = OFF_B_LO + B_BYTES;
+    static constexpr int SMEM = OFF_BAR + 128 + 1024;         // barriers + alignment slack
+    static constexpr int TMEM_COLS = 2 * D;                   // two accumulator buffers
+    // CTAs per SM: shared memory allows it, TMEM (512 columns) and registers must too
+    static constexpr int PER_SM = D == 64 ? 3 : 1;
+    static_assert(PER_SM * TMEM_COLS <= 512, "TMEM oversubscribed");
+    static_assert(PER_SM * (SMEM + 1024) <= 228 * 1024, "shared memory oversubscribed");
+};
+
+struct TcParams {
+    const float *Tk, *Tv;
+    int B, n, Hkv, T_cap, bits_k, bits_v;
+    int clip;                   // order-statistic index kappa, or kQuestClip
+    uint8_t *k_codes;
+    uint32_t *k_sz;
+    uint8_t *v_codes;
+    uint32_t *v_sz;
+    const int32_t *pos;
+    int32_t *dev_err;
+    PageMap pm;
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// 32 TMEM columns of this thread's lane as floats (load and wait in one statement, so
+// that nothing reads the registers before the load has completed).
+__device__ __forceinline__ void tmem_ld32_f(uint32_t taddr, float *x)
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        x[i] = __uint_as_float(r[i]);
+}
+
+// Code of x for the float16 pair (s, z): clamp(rint(f32(f32(x - z) / s)), 0, qmax).
+// The quotient is taken as a reciprocal multiply (within 2 ulp of the IEEE quotient);
+// within 2^-20 of a rounding tie it is recomputed with IEEE division.
+__device__ __forceinline__ uint32_t code_of(float x, float zf, float sf, float rc, bool zero,
+                                            float qmax)
+{
+    if (zero)
+        return 0u;
+    const float dlt = __fsub_rn(x, zf);
+    float y = __fmul_rn(dlt, rc);
+    float k = rintf(y);
+    if (fabsf(y - k) >= 0.5f - 9.5367431640625e-07f * fmaxf(fabsf(y), 1.f)) {
+        y = __fdiv_rn(dlt, sf);
+        k = rintf(y);
+    }
+    return (uint32_t)fminf(fmaxf(k, 0.f), qmax);
+}
+
+// Clip range (lo, hi) of the GS values x[0..GS) by order statistics kappa and GS-1-kappa.
+template <int GS>
+__device__ __forceinline__ void clip_range(const float *x, int kappa, float &lo, float &hi)
+{
+    if (kappa == 0) {
+        lo = x[0];
+        hi = x[0];
+#pragma unroll
+        for (int j = 1; j < GS; ++j) {
+            lo = fminf(lo, x[j]);
+            hi = fmaxf(hi, x[j]);
+        }
+    } else if (kappa == 1) {
+        float m1 = INFINITY, m2 = INFINITY, M1 = -INFINITY, M2 = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < GS; ++j) {
+            const float v = x[j];
+            m2 = fminf(m2, fmaxf(m1, v));
+            m1 = fminf(m1, v);
+            M2 = fmaxf(M2, fminf(M1, v));
+            M1 = fmaxf(M1, v);
+        }
+        lo = m2;
+        hi = M2;
+    } else {
+        // kappa <= 8: the 9 smallest and 9 largest by insertion
+        float sm[9], lg[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+            sm[i] = INFINITY;
+            lg[i] = -INFINITY;
+        }
+#pragma unroll
+        for (int j = 0; j < GS; ++j) {
+            float a = x[j], b = x[j];
+#pragma unroll
+            for (int i = 0; i < 9; ++i) {
+                const float s0 = fminf(sm[i], a), s1 = fmaxf(sm[i], a);
+                sm[i] = s0;
+                a = s1;
+                const float l0 = fmaxf(lg[i], b), l1 = fminf(lg[i], b);
+                lg[i] = l0;
+                b = l1;
+            }
+        }
+        lo = sm[0];
+        hi = lg[0];
+#pragma unroll
+        for (int i = 1; i < 9; ++i)
+            if (i == kappa) {
+                lo = sm[i];
+                hi = lg[i];
+            }
+    }
+}
+
+template <int D, int GS>
+__global__ void __launch_bounds__(kTcThreads, TcCfg<D>::PER_SM)
+append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 TcParams P)
+{
+    using C = TcCfg<D>;
+    constexpr int NG = D / GS;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    uint64_t *empty = full + kTcStages;
+    uint64_t *accf = empty + kTcStages;
+    uint64_t *acce = accf + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int h = blockIdx.y, which = blockIdx.z;
+    const CUtensorMap *tmap = which ? &tm_v : &tm_k;
+    const float *T = which ? P.Tv : P.Tk;
+    const int bits = which ? P.bits_v : P.bits_k;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long total = (long)P.B * P.n;
+    const long ntiles = (total + kTcTile - 1) / kTcTile;
+    const int my_tiles =
+        blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&accf[a], 1);
+            mbar_init(&acce[a], kTcEpiWarps * 32);
+        }
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0)
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+
+    // ---- T_h -> bf16 (hi, lo) in the K-major 128-byte-swizzled layout: row i (output dim)
+    //      of K block kb at kb*B_BLOCK + (i/8)*1024 + (i%8)*128, 16-byte chunk c of the row
+    //      at position c ^ (i % 8)
+    for (int c = threadIdx.x; c < D * D / 8; c += kTcThreads) {
+        const int i = c / (D / 8), j0 = 8 * (c % (D / 8));
+        const float4 *src = reinterpret_cast<const float4 *>(T + ((size_t)h * D + i) * D + j0);
+        const float4 f0 = src[0], f1 = src[1];
+        const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * e]);
+            const __nv_bfloat16 h1 = __float2bfloat16_rn(v[2 * e + 1]);
+            const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * e] - __bfloat162float(h0));
+            const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * e + 1] - __bfloat162float(h1));
+            hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+            lw[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+        }
+        const int kb = j0 / kTcKBlock, chunk = (j0 % kTcKBlock) / 8;
+        const int off = kb * C::B_BLOCK + (i / 8) * 1024 + (i % 8) * 128 + ((chunk ^ (i % 8)) * 16);
+        *reinterpret_cast<uint4 *>(smem + C::OFF_B_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4 *>(smem + C::OFF_B_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    fence_proxy_async_smem();           // generic stores -> operands of the tensor core
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    int issued = 0, consumed = 0;       // TMA lane: tiles loaded; MMA lane: tiles multiplied
+    if (warp == kTcEpiWarps) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(tmap);
+            for (int k = 0; k < my_tiles && !*abort_flag; ++k) {
+                const int s = k % kTcStages;
+                if (!mbar_wait_bounded(&empty[s], ((k / kTcStages) & 1) ^ 1)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                const long tile = blockIdx.x + (long)k * gridDim.x;
+                mbar_arrive_expect_tx(&full[s], C::A_BYTES);
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_3d(smem + s * C::A_BYTES + kb * C::A_BLOCK, tmap, kb * kTcKBlock, h,
+                                (int)(tile * kTcTile), &full[s]);
+                issued = k + 1;
+            }
+        }
+    } else if (warp == kTcEpiWarps + 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16_f32(kTcTile, D);
+            for (int k = 0; k < my_tiles && !*abort_flag; ++k) {
+                const int s = k % kTcStages, a = k & 1;
+                if (!mbar_wait_bounded(&acce[a], ((k >> 1) & 1) ^ 1) ||
+                    !mbar_wait_bounded(&full[s], (k / kTcStages) & 1)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(a * D);
+                const unsigned char *As = smem + s * C::A_BYTES;
+#pragma unroll
+                for (int piece = 0; piece < 2; ++piece)
+#pragma unroll
+                    for (int kb = 0; kb < C::KB; ++kb)
+#pragma unroll
+                        for (int kk = 0; kk < kTcKBlock / 16; ++kk) {
+                            const uint64_t ad = umma_desc_sw128_kmajor(As + kb * C::A_BLOCK + kk * 32);
+                            const uint64_t bd = umma_desc_sw128_kmajor(
+                                smem + (piece ? C::OFF_B_LO : C::OFF_B_HI) + kb * C::B_BLOCK + kk * 32);
+                            umma_bf16(d_tmem, ad, bd, idesc, (piece | kb | kk) != 0);
+                        }
+                umma_commit(&empty[s]);     // the stage may be refilled once these are done
+                umma_commit(&accf[a]);      // the accumulator is complete
+                consumed = k + 1;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int r = warp * 32 + lane;                     // token row of the tile
+        const uint32_t qmax_i = (1u << bits) - 1u;
+        const float qmax = (float)qmax_i;
+        const int ng = NG;
+        for (int k = 0; k < my_tiles; ++k) {
+            const int a = k & 1;
+            if (*abort_flag || !mbar_wait_bounded(&accf[a], (k >> 1) & 1)) {
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            float x[D];
+            const uint32_t taddr = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(a * D);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c)
+                tmem_ld32_f(taddr + 32 * c, x + 32 * c);
+            tc_fence_before_sync();
+            mbar_arrive(&acce[a]);                          // the MMA warp may reuse it
+
+            const long tile = blockIdx.x + (long)k * gridDim.x;
+            const long u = tile * kTcTile + r;
+            if (u >= total)
+                continue;
+            const int b = (int)(u / P.n), i = (int)(u - (long)b * P.n);
+            const int p0 = P.pos[b];
+            if (p0 < 0 || (long)p0 + P.n > P.T_cap) {
+                if (i == 0)
+                    flag(P.dev_err, KVQ_DEVERR_POS_RANGE);
+                continue;
+            }
+            const long long row = cache_row(P.pm, b, h, P.Hkv, P.T_cap, p0 + i);
+            if (row < 0) {
+                flag(P.dev_err, KVQ_DEVERR_PAGE_RANGE);
+                continue;
+            }
+            // per group: float16 (s, z), reciprocal, zero flag
+            float zf[NG], sf[NG], rc[NG];
+            bool zero[NG];
+#pragma unroll
+            for (int gr = 0; gr < NG; ++gr) {
+                const float *xg = x + gr * GS;
+                __half sh, zh;
+                bool finite;
+                if (P.clip == kQuestClip) {
+                    double ss = 0.0;
+#pragma unroll
+                    for (int j = 0; j < GS; ++j)
+                        ss = fma((double)xg[j], (double)xg[j], ss);
+                    const float rms = __double2float_rn(sqrt(ss / (double)GS));
+                    const float s = __fmul_rn(rms, quest_delta(bits));
+                    sh = __float2half_rn(s);
+                    zh = __float2half_rn(__fmul_rn(-0.5f * qmax, __half2float(sh)));
+                    finite = isfinite(s);
+                } else {
+                    float lo, hi;
+                    clip_range<GS>(xg, P.clip, lo, hi);
+                    const float range = __fsub_rn(hi, lo);
+                    const float s = __fdiv_rn(range, qmax);
+                    sh = __float2half_rn(s);
+                    zh = __float2half_rn(lo);
+                    finite = isfinite(range) && isfinite(s);
+                }
+                sf[gr] = __half2float(sh);
+                zf[gr] = __half2float(zh);
+                zero[gr] = !finite || sf[gr] == 0.f;
+                rc[gr] = zero[gr] ? 0.f : __frcp_rn(sf[gr]);
+                if (!finite)
+                    flag(P.dev_err, KVQ_DEVERR_NONFINITE);
+                (which ? P.v_sz : P.k_sz)[row * ng + gr] =
+                    (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
+            }
+            if (!which) {
+                // K row: little-endian bit stream, dim j at bit bits*j; stored as 16-byte pieces
+                uint32_t *dst = reinterpret_cast<uint32_t *>(P.k_codes + row * (D * bits / 8));
+                if (bits == 2) {
+#pragma unroll
+                    for (int w4 = 0; w4 < D / 64; ++w4) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t acc = 0;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const int j = 64 * w4 + 16 * q + e, gr = j / GS;
+                                acc |= code_of(x[j], zf[gr], sf[gr], rc[gr], zero[gr], qmax) << (2 * e);
+                            }
+                            w[q] = acc;
+                        }
+                        reinterpret_cast<uint4 *>(dst)[w4] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int w4 = 0; w4 < D / 32; ++w4) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t acc = 0;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int j = 32 * w4 + 8 * q + e, gr = j / GS;
+                                acc |= code_of(x[j], zf[gr], sf[gr], rc[gr], zero[gr], qmax) << (4 * e);
+                            }
+                            w[q] = acc;
+                        }
+                        reinterpret_cast<uint4 *>(dst)[w4] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            } else {
+                // V tile halves of this token: half (gq, rr) holds dims 8(E rr + s) + gq
+                unsigned char *tile_base =
+                    P.v_codes + (size_t)(row / kTileTokens) * (kTileTokens * D * bits / 8);
+                const int tok = (int)(row % kTileTokens);
+                if (bits == 2) {
+                    constexpr int E = 8, W = D * 2 / 128;
+#pragma unroll
+                    for (int gq = 0; gq < 8; ++gq)
+#pragma unroll
+                        for (int rr = 0; rr < W; ++rr) {
+                            uint32_t hv = 0;
+#pragma unroll
+                            for (int s2 = 0; s2 < E; ++s2) {
+                                const int j = 8 * (E * rr + s2) + gq, gr = j / GS;
+                                hv |= code_of(x[j], zf[gr], sf[gr], rc[gr], zero[gr], qmax) << (2 * s2);
+                            }
+                            *reinterpret_cast<uint16_t *>(tile_base + v_half_offset(D, 2, tok, gq, rr)) =
+                                (uint16_t)hv;
+                        }
+                } else {
+                    constexpr int E = 4, W = D * 4 / 128;
+#pragma unroll
+                    for (int gq = 0; gq < 8; ++gq)
+#pragma unroll
+                        for (int rr = 0; rr < W; ++rr) {
+                            uint32_t hv = 0;
+#pragma unroll
+                            for (int s2 = 0; s2 < E; ++s2) {
+                                const int j = 8 * (E * rr + s2) + gq, gr = j / GS;
+                                hv |= code_of(x[j], zf[gr], sf[gr], rc[gr], zero[gr], qmax) << (4 * s2);
+                            }
+                            *reinterpret_cast<uint16_t *>(tile_base + v_half_offset(D, 4, tok, gq, rr)) =
+                                (uint16_t)hv;
+                        }
+                }
+            }
+        }
+    }
+
+    // ---- teardown: on a timeout, wait (bounded) for what this CTA still has in flight
+    __syncthreads();
+    if (*abort_flag) {
+        if (threadIdx.x == 0)
+            flag(P.dev_err, KVQ_DEVERR_WAIT_TIMEOUT);
+        if (warp == kTcEpiWarps && lane == 0)              // copies never consumed
+            for (int k = consumed; k < issued; ++k)
+                mbar_wait_bounded(&full[k % kTcStages], (k / kTcStages) & 1);
+        if (warp == kTcEpiWarps + 1 && lane == 0 && consumed > 0)   // the last MMAs
+            mbar_wait_bounded(&accf[(consumed - 1) & 1], ((consumed - 1) >> 1) & 1);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// Tensor map over in[tokens][Hkv][D] bf16: dims (D, Hkv, tokens), box (64, 1, 128) with the
+// 128-byte swizzle; rows past the last token read as zeros.
+bool make_input_map(CUtensorMap *m, const void *base, int D, int Hkv, long tokens)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)tokens};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+    cuuint32_t box[3] = {kTcKBlock, 1, kTcTile};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int GS>
+cudaError_t launch_tc_t(const void *k, const void *v, const float *Tk, const float *Tv, int B, int n,
+                        const kvq_cache *c, int clip, const int32_t *pos, int32_t *dev_err,
+                        cudaStream_t st)
+{
+    using Cf = TcCfg<D>;
+    static unsigned long long attr_done = 0;
+    cudaError_t e = ensure_dynamic_smem(append_tc_kernel<D, GS>, Cf::SMEM, attr_done);
+    if (e != cudaSuccess)
+        return e;
+    const long tokens = (long)B * n;
+    CUtensorMap mk, mv;
+    if (!make_input_map(&mk, k, D, c->Hkv, tokens) || !make_input_map(&mv, v, D, c->Hkv, tokens))
+        return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long ntiles = (tokens + kTcTile - 1) / kTcTile;
+    long gx = ((long)sms * Cf::PER_SM) / (2L * c->Hkv);
+    if (gx < 1)
+        gx = 1;
+    if (gx > ntiles)
+        gx = ntiles;
+    TcParams P;
+    P.Tk = Tk;
+    P.Tv = Tv;
+    P.B = B;
+    P.n = n;
+    P.Hkv = c->Hkv;
+    P.T_cap = c->T_cap;
+    P.bits_k = c->qp.bits_k;
+    P.bits_v = c->qp.bits_v;
+    P.clip = clip;
+    P.k_codes = (uint8_t *)c->k_codes;
+    P.k_sz = (uint32_t *)c->k_sz;
+    P.v_codes = (uint8_t *)c->v_codes;
+    P.v_sz = (uint32_t *)c->v_sz;
+    P.pos = pos;
+    P.dev_err = dev_err;
+    P.pm = PageMap{c->block_table, c->page_tokens, c->num_pages};
+    append_tc_kernel<D, GS><<<dim3((unsigned)gx, (unsigned)c->Hkv, 2), kTcThreads, Cf::SMEM, st>>>(
+        mk, mv, P);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// bf16 chunks with both transforms: X . T^T on tcgen05 tensor cores. Needs the inputs
+// 16-byte aligned (tensor-map base) and B * n < 2^31 tokens.
+cudaError_t append_tc(const void *k, const void *v, const float *Tk, const float *Tv, int B, int n,
+                      const kvq_cache *c, int clip, const int32_t *pos, int32_t *dev_err,
+                      cudaStream_t st)
+{
+    const int d = c->d, g = c->qp.group;
+    if (d == 64 && g == 64)
+        return launch_tc_t<64, 64>(k, v, Tk, Tv, B, n, c, clip, pos, dev_err, st);
+    if (d == 64 && g == 32)
+        return launch_tc_t<64, 32>(k, v, Tk, Tv, B, n, c, clip, pos, dev_err, st);
+    if (d == 128 && g == 128)
+        return launch_tc_t<128, 128>(k, v, Tk, Tv, B, n, c, clip, pos, dev_err, st);
+    if (d == 128 && g == 64)
+        return launch_tc_t<128, 64>(k, v, Tk, Tv, B, n, c, clip, pos, dev_err, st);
+    if (d == 128 && g == 32)
+        return launch_tc_t<128, 32>(k, v, Tk, Tv, B, n, c, clip, pos, dev_err, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kvq
