@@ -401,6 +401,7 @@ def run_gpu(args):
     if not args.no_extras:
         line["bf16_comparator"] = bf16_comparator(w, cfg, K, stream, dec_ms)
         line["paged_decode"] = paged_decode(w, cfg, K, stream, dec_ms, dec_bytes)
+        line["window_decode"] = window_decode(w, cfg, stream, dec_ms, peak)
         del w
         torch.cuda.empty_cache()
         line["chunk_append"] = chunk_append(device, stream)
@@ -470,6 +471,34 @@ def decode_config_line(idx, device, stream, peak):
     return res
 
 
+def decode_split_sweep(idx, device, stream, peak, splits):
+    """Decode time of one workload for several split counts (KVQ_DECODE_SPLITS), one cache."""
+    import torch
+    import decode_attention_post_b200 as kvq
+    cfg = synth.CONFIGS[idx]
+    cache, seql, Tit = build_cache(cfg, device)
+    q = torch.from_numpy(synth.queries(cfg)).to(device).to(torch.bfloat16)
+    sd = torch.from_numpy(seql).to(device)
+    out = torch.empty((cfg.B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    nbytes = decode_bytes(cfg, seql)
+    res = []
+    for sp in [0] + list(splits):
+        if sp:
+            os.environ["KVQ_DECODE_SPLITS"] = str(sp)
+        else:
+            os.environ.pop("KVQ_DECODE_SPLITS", None)
+        ws = torch.empty(kvq.decode_workspace_bytes(cache, cfg.Hq, cfg.T_cap), dtype=torch.uint8,
+                         device=device)
+        fn = lambda: kvq.decode_attention(q, Tit, cache, sd, cfg.T_cap, out, ws, dev_err=err)
+        ms = statistics.mean(time_events(fn, 100, stream))
+        res.append({"splits": sp or "default", "ms": round(ms, 5),
+                    "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4)})
+        del ws
+    os.environ.pop("KVQ_DECODE_SPLITS", None)
+    return res
+
+
 def append_config0(device, stream):
     """Prefill append of the tiny float32 workload (1 sequence, 2048 tokens, 1 KV head,
     d 128): float32 CUDA-core transform path."""
@@ -535,6 +564,61 @@ def paged_decode(w, cfg, K, stream, dec_ms, dec_bytes, page_tokens=256):
     return {"page_tokens": page_tokens, "num_pages": num_pages, "ms_per_launch": round(ms, 5),
             "GB_s": round(dec_bytes / (ms * 1e-3) / 1e9, 1),
             "time_vs_contiguous": round(ms / dec_ms, 4), "output_identical": same}
+
+
+def window_decode(w, cfg, stream, dec_ms, peak, S_sink=64, S_keep=256, S_flush=128):
+    """The same sequences with a full-precision window (WUSH-KV section 4.4): the state is
+    built by kvq_window_append (one call per sequence over its whole context), then the
+    windowed decode (q prologue + window kernel + decode of the quantized middle) is timed,
+    and one decode-time step (window append of 1 token per sequence + windowed decode)."""
+    import torch
+    import decode_attention_post_b200 as kvq
+    B, Hkv, d = cfg.B, cfg.Hkv, cfg.d
+    R = S_keep + S_flush
+    z = lambda n: torch.zeros((B, Hkv, n, d), dtype=torch.bfloat16, device=w.dev)
+    ks, vs, kr, vr = z(S_sink), z(S_sink), z(R), z(R)
+    cache = kvq.KVCache.allocate(B, Hkv, cfg.T_cap, d, w.qp, device=w.dev, zero=False)
+    zero = torch.zeros(1, dtype=torch.int32, device=w.dev)
+    for b in range(B):
+        L = int(w.seqlens[b]) - 1                    # the step appends the last token
+        kb = w.kb[b, :, :L].transpose(0, 1).contiguous()[None]
+        vb = w.vb[b, :, :L].transpose(0, 1).contiguous()[None]
+        kvq.window_append(kb, vb, w.Tk, w.Tv, w.qp, cache.view_sequence(b), S_sink, S_keep,
+                          S_flush, ks[b:b + 1], vs[b:b + 1], kr[b:b + 1], vr[b:b + 1], zero,
+                          dev_err=w.err)
+    torch.cuda.synchronize()
+    prev = torch.from_numpy((w.seqlens - 1).astype(np.int32)).to(w.dev)
+    kvq.window_append(w.knew, w.vnew, w.Tk, w.Tv, w.qp, cache, S_sink, S_keep, S_flush, ks, vs,
+                      kr, vr, prev, dev_err=w.err)
+    out = torch.empty_like(w.out)
+    ws = torch.empty(kvq.decode_workspace_bytes(cache, cfg.Hq, cfg.T_cap), dtype=torch.uint8,
+                     device=w.dev)
+    dec = lambda: kvq.decode_attention_window(w.q, w.Tit, cache, S_sink, S_keep, S_flush, ks, vs,
+                                              kr, vr, w.Tv, w.seq_d, cfg.T_cap, out, ws,
+                                              dev_err=w.err)
+    ms = statistics.mean(time_events(dec, 200, stream))
+    # one serving step: re-append the newest token (the state for seqlens - 1 positions
+    # plus that token is the same state) and decode
+    step = lambda: (kvq.window_append(w.knew, w.vnew, w.Tk, w.Tv, w.qp, cache, S_sink, S_keep,
+                                      S_flush, ks, vs, kr, vr, prev, dev_err=w.err), dec())
+    step_ms = statistics.mean(time_events(step, 100, stream))
+    Q = np.array([(max(0, L - S_sink - S_keep) // S_flush) * S_flush for L in w.seqlens])
+    nwin = w.seqlens - Q
+    ng = d // cfg.group
+    per_q = Hkv * (d * (cfg.bits_k + cfg.bits_v) // 8 + 8 * ng)
+    nbytes = int(Q.sum()) * per_q + int(nwin.sum()) * Hkv * 2 * d * 2 + \
+        2 * Hkv * d * d * 4 + 2 * B * cfg.Hq * d * 2
+    torch.cuda.synchronize()
+    res = {"S_sink": S_sink, "S_keep": S_keep, "S_flush": S_flush,
+           "window_positions": int(nwin.sum()), "quantized_positions": int(Q.sum()),
+           "bytes_per_launch": nbytes, "ms_per_launch": round(ms, 5),
+           "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+           "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4),
+           "time_vs_plain_decode": round(ms / dec_ms, 4),
+           "step_ms_append_plus_decode": round(step_ms, 5), "dev_err": int(w.err.item())}
+    del cache, ks, vs, kr, vr, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def chunk_append(device, stream):
@@ -689,7 +773,13 @@ def profile_case(name):
     elif name == "append_config0":
         res = append_config0(device, stream)
     elif name.startswith("decode_config"):
-        res = decode_config_line(int(name[len("decode_config"):]), device, stream, peak)
+        idx = int(name[len("decode_config"):])
+        sweep = os.environ.get("KVQ_BENCH_SPLIT_SWEEP")    # e.g. "2,4,8": splits to time
+        if sweep:
+            res = {"sweep": decode_split_sweep(idx, device, stream, peak,
+                                               [int(x) for x in sweep.split(",")])}
+        else:
+            res = decode_config_line(idx, device, stream, peak)
     elif name == "bf16_config1":
         # the uncompressed comparator at the batch-16 / 16K shape (1.07 GB of bf16 K and V);
         # its time does not depend on the values, so they are drawn on the device

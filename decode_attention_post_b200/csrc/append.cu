@@ -19,6 +19,7 @@
 //      no read-modify-write is needed even for single-token appends. The token slot
 //      comes from the contiguous layout or, for a paged cache, the block table.
 #include "kvq_common.cuh"
+#include "kvq_ptx.cuh"
 
 #include <stdlib.h>
 
@@ -132,6 +133,107 @@ __device__ __forceinline__ TokenSlot token_slot(const TokenMap &tm, const void *
     }
     ts.dst = qo + i;
     return ts;
+}
+
+// Quantize one token held by a warp (lane l holds dims l + 32 r in vals[r]) and store it
+// at cache row `row`: per group the clip range (order statistics, or the RMS for the QuEST
+// INT quantizer, kappa == kQuestClip), the float16 scale and zero-point, IEEE-exact codes,
+// the K row (whole 32-bit words) or the token's halves of its V tile. `codes` is D bytes
+// of this warp's shared memory.
+template <int D>
+__device__ __forceinline__ void quantize_store_token(const float (&vals)[D / 32], int lane,
+                                                     uint8_t *codes, int which, int bits,
+                                                     int group, int kappa, long long row,
+                                                     uint8_t *k_codes, uint32_t *k_sz,
+                                                     uint8_t *v_codes, uint32_t *v_sz,
+                                                     int32_t *dev_err)
+{
+    constexpr int R = D / 32;
+    const int ng = D / group;
+    const int qmax = (1 << bits) - 1;
+    for (int gr = 0; gr < ng; ++gr) {
+        // group gr covers dims [gr*group, (gr+1)*group), i.e. r in [r0, r0+nr);
+        // dims outside the group are padded with +-inf so they are never picked.
+        const int r0 = gr * group / 32, nr = group / 32;
+        __half sh, zh;
+        bool finite;
+        if (kappa == kQuestClip) {
+            // QuEST INT: s = f32(rms * delta_b), z = -(2^b - 1)/2 * s_h; the sum of
+            // squares in float64 (each square exact), reduced over the warp
+            double ss = 0.0;
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                if (r >= r0 && r < r0 + nr)
+                    ss = fma((double)vals[r], (double)vals[r], ss);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            const float rms = __double2float_rn(sqrt(ss / (double)group));
+            const float s = __fmul_rn(rms, quest_delta(bits));
+            sh = __float2half_rn(s);
+            zh = __float2half_rn(__fmul_rn(-0.5f * (float)qmax, __half2float(sh)));
+            finite = isfinite(s);
+        } else {
+            float vmin[R], vmax[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const bool ing = r >= r0 && r < r0 + nr;
+                vmin[r] = ing ? vals[r] : INFINITY;
+                vmax[r] = ing ? vals[r] : -INFINITY;
+            }
+            const float lo = order_stat<R, false>(vmin, kappa, lane);
+            const float hi = order_stat<R, true>(vmax, kappa, lane);
+            const float range = __fsub_rn(hi, lo);
+            const float s = __fdiv_rn(range, (float)qmax);
+            sh = __float2half_rn(s);
+            zh = __float2half_rn(lo);
+            finite = isfinite(range) && isfinite(s);
+        }
+        const float sf = __half2float(sh), zf = __half2float(zh);
+        if (!finite && lane == 0)
+            flag(dev_err, KVQ_DEVERR_NONFINITE);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            if (r < r0 || r >= r0 + nr)
+                continue;
+            int c = 0;
+            if (finite && sf != 0.f) {
+                float y = __fdiv_rn(__fsub_rn(vals[r], zf), sf);
+                float cr = rintf(y);
+                cr = fminf(fmaxf(cr, 0.f), (float)qmax);
+                c = (int)cr;
+            }
+            codes[lane + 32 * r] = (uint8_t)c;
+        }
+        if (lane == 0) {
+            uint32_t pair = (uint32_t)__half_as_ushort(sh) |
+                            ((uint32_t)__half_as_ushort(zh) << 16);
+            (which ? v_sz : k_sz)[row * ng + gr] = pair;
+        }
+    }
+    __syncwarp();
+    if (!which) {
+        const int words = D * bits / 32, cpw = 32 / bits;
+        if (lane < words) {
+            uint32_t w = 0;
+            for (int e = 0; e < cpw; ++e)
+                w |= (uint32_t)codes[lane * cpw + e] << (bits * e);
+            reinterpret_cast<uint32_t *>(k_codes + row * (D * bits / 8))[lane] = w;
+        }
+    } else {
+        const int E = 16 / bits, halves = D / E;
+        if (lane < halves) {
+            const int gq = lane & 7, r = lane >> 3;
+            uint32_t hv = 0;
+            for (int s2 = 0; s2 < E; ++s2)
+                hv |= (uint32_t)codes[8 * (E * r + s2) + gq] << (bits * s2);
+            const size_t tile_base =
+                (size_t)(row / kTileTokens) * (kTileTokens * D * bits / 8);
+            const int off = v_half_offset(D, bits, (int)(row % kTileTokens), gq, r);
+            *reinterpret_cast<uint16_t *>(v_codes + tile_base + off) = (uint16_t)hv;
+        }
+    }
+    __syncwarp();
 }
 
 template <int D, int TPW>
@@ -279,91 +381,204 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
                     flag(dev_err, KVQ_DEVERR_PAGE_RANGE);
                 continue;
             }
-            for (int gr = 0; gr < ng; ++gr) {
-                // group gr covers dims [gr*group, (gr+1)*group), i.e. r in [r0, r0+nr);
-                // dims outside the group are padded with +-inf so they are never picked.
-                const int r0 = gr * group / 32, nr = group / 32;
-                __half sh, zh;
-                bool finite;
-                if (kappa == kQuestClip) {
-                    // QuEST INT: s = f32(rms * delta_b), z = -(2^b - 1)/2 * s_h; the sum of
-                    // squares in float64 (each square exact), reduced over the warp
-                    double ss = 0.0;
-#pragma unroll
-                    for (int r = 0; r < R; ++r)
-                        if (r >= r0 && r < r0 + nr)
-                            ss = fma((double)acc[q][r], (double)acc[q][r], ss);
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1)
-                        ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                    const float rms = __double2float_rn(sqrt(ss / (double)group));
-                    const float s = __fmul_rn(rms, quest_delta(bits));
-                    sh = __float2half_rn(s);
-                    zh = __float2half_rn(__fmul_rn(-0.5f * (float)qmax, __half2float(sh)));
-                    finite = isfinite(s);
-                } else {
-                    float vmin[R], vmax[R];
-#pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        const bool ing = r >= r0 && r < r0 + nr;
-                        vmin[r] = ing ? acc[q][r] : INFINITY;
-                        vmax[r] = ing ? acc[q][r] : -INFINITY;
-                    }
-                    const float lo = order_stat<R, false>(vmin, kappa, lane);
-                    const float hi = order_stat<R, true>(vmax, kappa, lane);
-                    const float range = __fsub_rn(hi, lo);
-                    const float s = __fdiv_rn(range, (float)qmax);
-                    sh = __float2half_rn(s);
-                    zh = __float2half_rn(lo);
-                    finite = isfinite(range) && isfinite(s);
-                }
-                const float sf = __half2float(sh), zf = __half2float(zh);
-                if (!finite && lane == 0)
-                    flag(dev_err, KVQ_DEVERR_NONFINITE);
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    if (r < r0 || r >= r0 + nr)
-                        continue;
-                    int c = 0;
-                    if (finite && sf != 0.f) {
-                        float y = __fdiv_rn(__fsub_rn(acc[q][r], zf), sf);
-                        float cr = rintf(y);
-                        cr = fminf(fmaxf(cr, 0.f), (float)qmax);
-                        c = (int)cr;
-                    }
-                    sm.codes[warp][lane + 32 * r] = (uint8_t)c;
-                }
-                if (lane == 0) {
-                    uint32_t pair = (uint32_t)__half_as_ushort(sh) |
-                                    ((uint32_t)__half_as_ushort(zh) << 16);
-                    (which ? v_sz : k_sz)[row * ng + gr] = pair;
-                }
-            }
-            __syncwarp();
-            if (!which) {
-                const int words = D * bits / 32, cpw = 32 / bits;
-                if (lane < words) {
-                    uint32_t w = 0;
-                    for (int e = 0; e < cpw; ++e)
-                        w |= (uint32_t)sm.codes[warp][lane * cpw + e] << (bits * e);
-                    reinterpret_cast<uint32_t *>(k_codes + row * (D * bits / 8))[lane] = w;
-                }
-            } else {
-                const int E = 16 / bits, halves = D / E;
-                if (lane < halves) {
-                    const int gq = lane & 7, r = lane >> 3;
-                    uint32_t hv = 0;
-                    for (int s2 = 0; s2 < E; ++s2)
-                        hv |= (uint32_t)sm.codes[warp][8 * (E * r + s2) + gq] << (bits * s2);
-                    const size_t tile_base =
-                        (size_t)(row / kTileTokens) * (kTileTokens * D * bits / 8);
-                    const int off = v_half_offset(D, bits, (int)(row % kTileTokens), gq, r);
-                    *reinterpret_cast<uint16_t *>(v_codes + tile_base + off) = (uint16_t)hv;
-                }
-            }
-            __syncwarp();
+            quantize_store_token<D>(acc[q], lane, sm.codes[warp], which, bits, group, kappa, row,
+                                    k_codes, k_sz, v_codes, v_sz, dev_err);
         }
     }
+}
+
+// ---------------------------------------------------------------- short bf16 appends
+
+// Decode-time appends (a few tokens per sequence, bfloat16, both transforms) and window
+// flushes: 16-token tiles, 8 warps. Warp w computes output dims [w D/8, (w+1) D/8) of the
+// tile on mma.sync (bf16, float32 accumulate): its fragments of T = T_hi + T_lo (two
+// bfloat16 pieces, 16 significant bits) come straight from global memory (L2) into
+// registers once per CTA, so no CTA stages the whole transform in shared memory. The
+// tile's inputs are staged in shared memory (ldmatrix A operands), the transformed tile
+// goes back to shared memory, and each warp quantizes and stores two of its tokens.
+constexpr int kSmallWarps = 8;
+constexpr int kSmallTile = 16;
+
+template <int D>
+struct SmallSmem {
+    static constexpr int XS = D + 8;                 // bf16 per staged input row
+    static constexpr int YS = D + 4;                 // float per transformed row
+    __nv_bfloat16 X[kSmallTile * XS];
+    float Y[kSmallTile * YS];
+    uint8_t codes[kSmallWarps][D];
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo_elem, float hi_elem)
+{
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo_elem)) |
+           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi_elem)) << 16);
+}
+
+__device__ __forceinline__ float bf16_rn(float x)
+{
+    return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSmallWarps * 32)
+append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *__restrict__ v_in,
+                    const float *__restrict__ Tk, const float *__restrict__ Tv, int B, int n,
+                    int Hkv, int T_cap, int bits_k, int bits_v, int group, int kappa,
+                    uint8_t *__restrict__ k_codes, uint32_t *__restrict__ k_sz,
+                    uint8_t *__restrict__ v_codes, uint32_t *__restrict__ v_sz,
+                    const int32_t *__restrict__ pos, int32_t *dev_err, PageMap pm, TokenMap tm)
+{
+    constexpr int NTW = D / 64;                      // n-tiles (8 output dims) per warp
+    constexpr int KS = D / 16;
+    using Sm = SmallSmem<D>;
+    __shared__ __align__(16) Sm sm;
+    __shared__ int tile_active;
+
+    const int h = blockIdx.y, which = blockIdx.z;
+    const void *in = which ? (const void *)v_in : (const void *)k_in;
+    const float *T = (which ? Tv : Tk) + (size_t)h * D * D;
+    const int bits = which ? bits_v : bits_k;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const long total = (long)B * n;
+    const long tiles = (total + kSmallTile - 1) / kSmallTile;
+
+    uint32_t bhi[NTW][KS][2], blo[NTW][KS][2];
+    bool have_b = false;
+    auto load_b = [&]() {
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt) {
+            const float *row = T + (size_t)(8 * (warp * NTW + nt) + g) * D;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const float2 f = *reinterpret_cast<const float2 *>(row + 16 * ks + 8 * half + 2 * t);
+                    const float h0 = bf16_rn(f.x), h1 = bf16_rn(f.y);
+                    bhi[nt][ks][half] = pack_bf16x2(f.x, f.y);
+                    blo[nt][ks][half] = pack_bf16x2(f.x - h0, f.y - h1);
+                }
+        }
+        have_b = true;
+    };
+
+    for (long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        const long u0 = tile * kSmallTile;
+        __syncthreads();                             // the previous tile's readers are done
+        if (tm.ring_k) {
+            // window flush: skip tiles without a token to write (most of a decode step)
+            if (threadIdx.x == 0)
+                tile_active = 0;
+            __syncthreads();
+            if (threadIdx.x < kSmallTile && u0 + threadIdx.x < total) {
+                const long u = u0 + threadIdx.x;
+                const TokenSlot ts = token_slot(tm, in, which, pos, (int)(u / n), (int)(u % n), n,
+                                                h, Hkv, D, T_cap);
+                if (ts.active || (ts.bad_range && ts.first))
+                    tile_active = 1;
+            }
+            __syncthreads();
+            if (!tile_active)
+                continue;
+        }
+        if (!have_b)
+            load_b();
+        // ---- stage the tile's inputs (16-byte chunks; inactive rows are zero)
+        for (int c = threadIdx.x; c < kSmallTile * (D / 8); c += kSmallWarps * 32) {
+            const int rr = c / (D / 8), ch = c % (D / 8);
+            const long u = u0 + rr;
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (u < total) {
+                const TokenSlot ts = token_slot(tm, in, which, pos, (int)(u / n), (int)(u % n), n,
+                                                h, Hkv, D, T_cap);
+                if (ts.active)
+                    val = reinterpret_cast<const uint4 *>(
+                        reinterpret_cast<const __nv_bfloat16 *>(ts.base) + ts.src)[ch];
+            }
+            *reinterpret_cast<uint4 *>(sm.X + rr * Sm::XS + 8 * ch) = val;
+        }
+        __syncthreads();
+        // ---- X~ = X . (T_hi + T_lo)^T, this warp's output dims
+        float acc[NTW][4];
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[nt][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            uint32_t a[4];
+            ldmatrix_x4(a, sm.X + (lane & 15) * Sm::XS + 16 * ks + 8 * (lane >> 4));
+#pragma unroll
+            for (int nt = 0; nt < NTW; ++nt) {
+                mma_bf16(acc[nt], a[0], a[1], a[2], a[3], bhi[nt][ks][0], bhi[nt][ks][1]);
+                mma_bf16(acc[nt], a[0], a[1], a[2], a[3], blo[nt][ks][0], blo[nt][ks][1]);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt) {
+            const int col = 8 * (warp * NTW + nt) + 2 * t;
+            *reinterpret_cast<float2 *>(sm.Y + g * Sm::YS + col) = make_float2(acc[nt][0], acc[nt][1]);
+            *reinterpret_cast<float2 *>(sm.Y + (g + 8) * Sm::YS + col) =
+                make_float2(acc[nt][2], acc[nt][3]);
+        }
+        __syncthreads();
+        // ---- quantize and store: warp w takes tokens 2w, 2w+1 of the tile
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int rr = 2 * warp + q;
+            const long u = u0 + rr;
+            if (u >= total)
+                break;
+            const int b = (int)(u / n), i = (int)(u % n);
+            const TokenSlot ts = token_slot(tm, in, which, pos, b, i, n, h, Hkv, D, T_cap);
+            if (ts.bad_range) {
+                if (ts.first && lane == 0)
+                    flag(dev_err, KVQ_DEVERR_POS_RANGE);
+                continue;
+            }
+            if (!ts.active)
+                continue;
+            const long long row = cache_row(pm, b, h, Hkv, T_cap, ts.dst);
+            if (row < 0) {
+                if (lane == 0)
+                    flag(dev_err, KVQ_DEVERR_PAGE_RANGE);
+                continue;
+            }
+            float vals[D / 32];
+#pragma unroll
+            for (int r = 0; r < D / 32; ++r)
+                vals[r] = sm.Y[rr * Sm::YS + lane + 32 * r];
+            quantize_store_token<D>(vals, lane, sm.codes[warp], which, bits, group, kappa, row,
+                                    k_codes, k_sz, v_codes, v_sz, dev_err);
+        }
+    }
+}
+
+template <int D>
+cudaError_t launch_append_small(const void *k, const void *v, const float *Tk, const float *Tv,
+                                int B, int n, const kvq_cache *c, int kappa, const int32_t *pos,
+                                int32_t *dev_err, cudaStream_t st, const TokenMap &tm = TokenMap{})
+{
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long tiles = ((long)B * n + kSmallTile - 1) / kSmallTile;
+    // one tile per CTA while that fills the GPU; a flush (most tiles empty) or a long
+    // chunk walks the tiles grid-stride with about two CTAs per SM
+    long want = (2L * sms + 2L * c->Hkv - 1) / (2L * c->Hkv);
+    long gx = tiles;
+    if (tm.ring_k || tiles > 4 * want)
+        gx = tiles < want ? tiles : want;
+    if (gx < 1)
+        gx = 1;
+    dim3 grid((unsigned)gx, (unsigned)c->Hkv, 2);
+    append_small_kernel<D><<<grid, kSmallWarps * 32, 0, st>>>(
+        (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, Tk, Tv, B, n, c->Hkv, c->T_cap,
+        c->qp.bits_k, c->qp.bits_v, c->qp.group, kappa, (uint8_t *)c->k_codes, (uint32_t *)c->k_sz,
+        (uint8_t *)c->v_codes, (uint32_t *)c->v_sz, pos, dev_err,
+        PageMap{c->block_table, c->page_tokens, c->num_pages}, tm);
+    return cudaGetLastError();
 }
 
 template <int D, int TPW>
@@ -433,6 +648,13 @@ cudaError_t window_flush_launch(const void *k_new, const void *v_new, const floa
     const long nmax = (long)S_flush * ((n_new + S_flush - 1) / S_flush);
     if (nmax > 0x7fffffffL / (B > 0 ? B : 1))
         return cudaErrorInvalidValue;
+    if (Tk && Tv) {                     // bf16 tokens (ring and new) through the tensor cores
+        if (c->d == 64)
+            return launch_append_small<64>(k_new, v_new, Tk, Tv, B, (int)nmax, c, kappa, nullptr,
+                                           dev_err, st, tm);
+        return launch_append_small<128>(k_new, v_new, Tk, Tv, B, (int)nmax, c, kappa, nullptr,
+                                        dev_err, st, tm);
+    }
     if (c->d == 64)
         return launch_append_fp32<64, 4>(k_new, v_new, 1, Tk, Tv, B, (int)nmax, c, kappa, nullptr,
                                          dev_err, st, tm);
@@ -444,10 +666,11 @@ cudaError_t append_tc(const void *k, const void *v, const float *Tk, const float
                       const kvq_cache *c, int clip, const int32_t *pos, int32_t *dev_err,
                       cudaStream_t st);
 
-// Chunks of bfloat16 inputs with both transforms go to the tcgen05 tensor-core kernel
-// (KVQ_APPEND_PATH=mma selects the warp-level mma.sync kernel instead, for comparison);
-// float32 inputs, identity transforms, small (decode-time) appends and unaligned inputs
-// use the float32 CUDA-core kernel.
+// bfloat16 inputs with both transforms: chunks of 256 tokens or more go to the tcgen05
+// tensor-core kernel, shorter (decode-time) appends to the short mma.sync kernel
+// (KVQ_APPEND_PATH=mma / fp32 select the older warp-level chunk kernel or the CUDA-core
+// kernel instead, for comparison); float32 inputs, identity transforms and unaligned
+// inputs use the float32 CUDA-core kernel.
 cudaError_t append_launch(const void *k, const void *v, int in_bf16, const float *Tk,
                           const float *Tv, int B, int n, const kvq_cache *c, int kappa,
                           const int32_t *pos, int32_t *dev_err, cudaStream_t st)
@@ -455,11 +678,17 @@ cudaError_t append_launch(const void *k, const void *v, int in_bf16, const float
     const long tokens = (long)B * n;
     const bool a16 = ((uintptr_t)k % 16 == 0) && ((uintptr_t)v % 16 == 0) &&
                      ((uintptr_t)Tk % 16 == 0) && ((uintptr_t)Tv % 16 == 0);
-    if (in_bf16 && Tk && Tv && a16 && tokens >= 256) {
-        const char *path = getenv("KVQ_APPEND_PATH");
+    const char *path = getenv("KVQ_APPEND_PATH");
+    const bool force_fp32 = path && path[0] == 'f';
+    if (in_bf16 && Tk && Tv && a16 && tokens >= 256 && !force_fp32) {
         if ((path && path[0] == 'm') || tokens > 0x7fffff00L)
             return append_mma(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
         return append_tc(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
+    }
+    if (in_bf16 && Tk && Tv && a16 && !force_fp32) {
+        if (c->d == 64)
+            return launch_append_small<64>(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
+        return launch_append_small<128>(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
     }
     const bool small = tokens <= 2048;
     if (c->d == 64)

@@ -13,16 +13,19 @@
 //                      instruction; two accumulator buffers so that the next tile's MMAs
 //                      overlap this tile's epilogue;
 //   warps 0-3          epilogue: thread r owns token r of the tile; tcgen05.ld brings its
-//                      d transformed values into registers, then per group the clip range
-//                      (order statistics, or the RMS for the QuEST INT quantizer), the
-//                      float16 scale and zero-point, the codes (reciprocal multiply with an
-//                      IEEE-division fallback within 2^-20 of a rounding tie, so the codes
-//                      are those of the definition bit for bit) and the fixed-width stores
-//                      (one K row, or the token's halves of its 16-token V tile).
+//                      transformed values into registers 32 columns at a time, in two
+//                      passes: per group the clip range (order statistics, or the RMS for
+//                      the QuEST INT quantizer) and the float16 scale and zero-point, then
+//                      the codes (reciprocal multiply; a row with a value within 2^-16 of a
+//                      rounding tie is redone with IEEE division, so the codes are those of
+//                      the definition bit for bit) and the fixed-width stores (one K row,
+//                      or the token's halves of its 16-token V tile).
 // T (the B operand, N = d output dims x K = d input dims, K-major) is converted and
 // swizzled into shared memory once per CTA. Every wait is bounded; a wait that gives up
 // flags KVQ_DEVERR_WAIT_TIMEOUT, the CTA waits (bounded) for its copies and MMAs in flight,
 // frees its TMEM and stops.
+// The codes use no conversion unit: rounding by the float addition of 1.5 * 2^23, packing
+// by multiply-adds of the resulting bit patterns.
 #include "kvq_common.cuh"
 #include "kvq_ptx.cuh"
 
@@ -97,77 +100,190 @@ __device__ __forceinline__ void tmem_ld32_f(uint32_t taddr, float *x)
         x[i] = __uint_as_float(r[i]);
 }
 
-// Code of x for the float16 pair (s, z): clamp(rint(f32(f32(x - z) / s)), 0, qmax).
-// The quotient is taken as a reciprocal multiply (within 2 ulp of the IEEE quotient);
-// within 2^-20 of a rounding tie it is recomputed with IEEE division.
-__device__ __forceinline__ uint32_t code_of(float x, float zf, float sf, float rc, bool zero,
-                                            float qmax)
+// Codes of a group: c = clamp(rint(f32(f32(x - z) / s)), 0, qmax) for float16 (s, z).
+// The quotient is taken as a reciprocal multiply (within 2 ulp of the IEEE quotient), the
+// clamp comes first (the same result: rint and the clamp are both monotone and the clamp
+// bounds are integers) and the rounding to nearest even is the float addition of
+// 1.5 * 2^23, whose bit pattern is then 0x4B400000 + c. A value within 2^-16 of a
+// rounding tie sets `tie`; the caller then recomputes the row with IEEE division.
+constexpr float kRoundMagic = 12582912.0f;        // 1.5 * 2^23
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+constexpr float kTieBand = 0.5f - 1.52587890625e-05f;   // 0.5 - 2^-16
+
+// bit pattern 0x4B400000 + c of the rounded value
+__device__ __forceinline__ uint32_t code_bits(float x, float zf, float rc, float qmax, bool &tie)
+{
+    float y = __fmul_rn(__fsub_rn(x, zf), rc);
+    y = fminf(fmaxf(y, 0.f), qmax);
+    const float r = __fadd_rn(y, kRoundMagic);
+    const float t = __fsub_rn(y, __fsub_rn(r, kRoundMagic));
+    tie |= fabsf(t) >= kTieBand;
+    return __float_as_uint(r);
+}
+
+// the same code by IEEE division (ties to even); s_h == 0 or a non-finite range gives 0
+__device__ __forceinline__ uint32_t code_exact(float x, float zf, float sf, bool zero, float qmax)
 {
     if (zero)
         return 0u;
-    const float dlt = __fsub_rn(x, zf);
-    float y = __fmul_rn(dlt, rc);
-    float k = rintf(y);
-    if (fabsf(y - k) >= 0.5f - 9.5367431640625e-07f * fmaxf(fabsf(y), 1.f)) {
-        y = __fdiv_rn(dlt, sf);
-        k = rintf(y);
-    }
+    const float k = rintf(__fdiv_rn(__fsub_rn(x, zf), sf));
     return (uint32_t)fminf(fmaxf(k, 0.f), qmax);
 }
 
-// Clip range (lo, hi) of the GS values x[0..GS) by order statistics kappa and GS-1-kappa.
-template <int GS>
-__device__ __forceinline__ void clip_range(const float *x, int kappa, float &lo, float &hi)
+// sum over e < N of 0x4B400000 * 2^(B*e), modulo 2^32: what packing N magic-rounded codes
+// with multiply-adds leaves above the codes themselves
+__host__ __device__ constexpr uint32_t magic_sum(int B, int N)
 {
-    if (kappa == 0) {
-        lo = x[0];
-        hi = x[0];
+    uint32_t s = 0;
+    for (int e = 0; e < N; ++e)
+        s += kRoundMagicBits << (B * e);
+    return s;
+}
+
+__device__ __forceinline__ float fmin3(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// The K row of one token (little-endian bit stream, dim j at bit bits*j) from its row in
+// TMEM, 32 columns at a time; stored as 16-byte pieces when row >= 0. exact = false: the
+// fast codes (sets `tie` near a rounding tie); exact = true: IEEE division. Warp-wide (the
+// TMEM loads), every lane calls it.
+template <int D, int GS, int NG>
+__device__ __forceinline__ void store_k_row(const TcParams &P, long long row, int bits,
+                                            uint32_t taddr, const float (&zf)[NG],
+                                            const float (&sf)[NG], const float (&rc)[NG],
+                                            const bool (&zero)[NG], float qmax, bool &tie,
+                                            bool exact)
+{
+    float x[32];
+    uint4 *dst = reinterpret_cast<uint4 *>(P.k_codes + row * (D * bits / 8));
 #pragma unroll
-        for (int j = 1; j < GS; ++j) {
-            lo = fminf(lo, x[j]);
-            hi = fmaxf(hi, x[j]);
-        }
-    } else if (kappa == 1) {
-        float m1 = INFINITY, m2 = INFINITY, M1 = -INFINITY, M2 = -INFINITY;
+    for (int c = 0; c < D / 32; ++c) {
+        const int gr = (32 * c) / GS;
+        tmem_ld32_f(taddr + 32 * c, x);
+        if (bits == 2) {
+            uint32_t w[2];
 #pragma unroll
-        for (int j = 0; j < GS; ++j) {
-            const float v = x[j];
-            m2 = fminf(m2, fmaxf(m1, v));
-            m1 = fminf(m1, v);
-            M2 = fmaxf(M2, fminf(M1, v));
-            M1 = fmaxf(M1, v);
+            for (int q = 0; q < 2; ++q) {
+                uint32_t acc = exact ? 0u : 0u - magic_sum(2, 16);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float v = x[16 * q + e];
+                    acc += (exact ? code_exact(v, zf[gr], sf[gr], zero[gr], qmax)
+                                  : code_bits(v, zf[gr], rc[gr], qmax, tie)) << (2 * e);
+                }
+                w[q] = acc;
+            }
+            // two words per 32 columns: a 16-byte piece every other chunk
+            if (row >= 0) {
+                if (c % 2 == 0) {
+                    dst[c / 2].x = w[0];
+                    dst[c / 2].y = w[1];
+                } else {
+                    dst[c / 2].z = w[0];
+                    dst[c / 2].w = w[1];
+                }
+            }
+        } else {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t acc = exact ? 0u : 0u - magic_sum(4, 8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float v = x[8 * q + e];
+                    acc += (exact ? code_exact(v, zf[gr], sf[gr], zero[gr], qmax)
+                                  : code_bits(v, zf[gr], rc[gr], qmax, tie)) << (4 * e);
+                }
+                w[q] = acc;
+            }
+            if (row >= 0)
+                dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        lo = m2;
-        hi = M2;
+    }
+}
+
+// The token's halves of its 16-token V tile: half (gq, rr) holds dims 8(E rr + s) + gq at
+// bits*s, E = 16/bits; a half gathers dims 8 apart, so the halves are built up over the
+// 32-column chunks and stored at the end (row >= 0). Same conventions as store_k_row.
+template <int D, int GS, int NG>
+__device__ __forceinline__ void store_v_token(const TcParams &P, long long row, int bits,
+                                              uint32_t taddr, const float (&zf)[NG],
+                                              const float (&sf)[NG], const float (&rc)[NG],
+                                              const bool (&zero)[NG], float qmax, bool &tie,
+                                              bool exact)
+{
+    float x[32];
+    if (bits == 2) {
+        constexpr int E = 8, W = D * 2 / 128;           // a half spans 64 dims
+        uint32_t hv[8][W];
+#pragma unroll
+        for (int gq = 0; gq < 8; ++gq)
+#pragma unroll
+            for (int rr = 0; rr < W; ++rr)
+                hv[gq][rr] = exact ? 0u : 0u - magic_sum(2, E);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            const int gr = (32 * c) / GS;
+            tmem_ld32_f(taddr + 32 * c, x);
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                const int j = 32 * c + jj, gq = j % 8, n8 = j / 8, rr = n8 / E, s2 = n8 % E;
+                hv[gq][rr] += (exact ? code_exact(x[jj], zf[gr], sf[gr], zero[gr], qmax)
+                                     : code_bits(x[jj], zf[gr], rc[gr], qmax, tie)) << (2 * s2);
+            }
+        }
+        if (row >= 0) {
+            unsigned char *tile_base =
+                P.v_codes + (size_t)(row / kTileTokens) * (kTileTokens * D * 2 / 8);
+            const int tok = (int)(row % kTileTokens);
+#pragma unroll
+            for (int gq = 0; gq < 8; ++gq)
+#pragma unroll
+                for (int rr = 0; rr < W; ++rr)
+                    *reinterpret_cast<uint16_t *>(tile_base + v_half_offset(D, 2, tok, gq, rr)) =
+                        (uint16_t)hv[gq][rr];
+        }
     } else {
-        // kappa <= 8: the 9 smallest and 9 largest by insertion
-        float sm[9], lg[9];
+        constexpr int E = 4, W = D * 4 / 128;           // a half spans 32 dims
+        uint32_t hv[8][W];
 #pragma unroll
-        for (int i = 0; i < 9; ++i) {
-            sm[i] = INFINITY;
-            lg[i] = -INFINITY;
-        }
+        for (int gq = 0; gq < 8; ++gq)
 #pragma unroll
-        for (int j = 0; j < GS; ++j) {
-            float a = x[j], b = x[j];
+            for (int rr = 0; rr < W; ++rr)
+                hv[gq][rr] = exact ? 0u : 0u - magic_sum(4, E);
 #pragma unroll
-            for (int i = 0; i < 9; ++i) {
-                const float s0 = fminf(sm[i], a), s1 = fmaxf(sm[i], a);
-                sm[i] = s0;
-                a = s1;
-                const float l0 = fmaxf(lg[i], b), l1 = fminf(lg[i], b);
-                lg[i] = l0;
-                b = l1;
+        for (int c = 0; c < D / 32; ++c) {
+            const int gr = (32 * c) / GS;
+            tmem_ld32_f(taddr + 32 * c, x);
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                const int j = 32 * c + jj, gq = j % 8, n8 = j / 8, rr = n8 / E, s2 = n8 % E;
+                hv[gq][rr] += (exact ? code_exact(x[jj], zf[gr], sf[gr], zero[gr], qmax)
+                                     : code_bits(x[jj], zf[gr], rc[gr], qmax, tie)) << (4 * s2);
             }
         }
-        lo = sm[0];
-        hi = lg[0];
+        if (row >= 0) {
+            unsigned char *tile_base =
+                P.v_codes + (size_t)(row / kTileTokens) * (kTileTokens * D * 4 / 8);
+            const int tok = (int)(row % kTileTokens);
 #pragma unroll
-        for (int i = 1; i < 9; ++i)
-            if (i == kappa) {
-                lo = sm[i];
-                hi = lg[i];
-            }
+            for (int gq = 0; gq < 8; ++gq)
+#pragma unroll
+                for (int rr = 0; rr < W; ++rr)
+                    *reinterpret_cast<uint16_t *>(tile_base + v_half_offset(D, 4, tok, gq, rr)) =
+                        (uint16_t)hv[gq][rr];
+        }
     }
 }
 
@@ -294,10 +410,13 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Two passes over the token's row in TMEM, 32 columns at a time (registers stay
+        // low): the clip parameters of every group, then the codes. The accumulator buffer
+        // is released after the row is done, so a row near a rounding tie can be reloaded
+        // and recomputed with IEEE division.
         const int r = warp * 32 + lane;                     // token row of the tile
-        const uint32_t qmax_i = (1u << bits) - 1u;
-        const float qmax = (float)qmax_i;
-        const int ng = NG;
+        const float qmax = (float)((1u << bits) - 1u);
+        const bool quest = P.clip == kQuestClip;
         for (int k = 0; k < my_tiles; ++k) {
             const int a = k & 1;
             if (*abort_flag || !mbar_wait_bounded(&accf[a], (k >> 1) & 1)) {
@@ -305,139 +424,142 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 break;
             }
             tc_fence_after_sync();
-            float x[D];
             const uint32_t taddr = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(a * D);
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c)
-                tmem_ld32_f(taddr + 32 * c, x + 32 * c);
-            tc_fence_before_sync();
-            mbar_arrive(&acce[a]);                          // the MMA warp may reuse it
-
             const long tile = blockIdx.x + (long)k * gridDim.x;
             const long u = tile * kTcTile + r;
-            if (u >= total)
-                continue;
-            const int b = (int)(u / P.n), i = (int)(u - (long)b * P.n);
-            const int p0 = P.pos[b];
-            if (p0 < 0 || (long)p0 + P.n > P.T_cap) {
-                if (i == 0)
-                    flag(P.dev_err, KVQ_DEVERR_POS_RANGE);
-                continue;
+            long long row = -1;
+            if (u < total) {
+                const unsigned uu = (unsigned)u;            // the launcher keeps B * n < 2^31
+                const int b = (int)(uu / (unsigned)P.n), i = (int)(uu - (unsigned)b * (unsigned)P.n);
+                const int p0 = P.pos[b];
+                if (p0 < 0 || (long)p0 + P.n > P.T_cap) {
+                    if (i == 0)
+                        flag(P.dev_err, KVQ_DEVERR_POS_RANGE);
+                } else {
+                    row = cache_row(P.pm, b, h, P.Hkv, P.T_cap, p0 + i);
+                    if (row < 0)
+                        flag(P.dev_err, KVQ_DEVERR_PAGE_RANGE);
+                }
             }
-            const long long row = cache_row(P.pm, b, h, P.Hkv, P.T_cap, p0 + i);
-            if (row < 0) {
-                flag(P.dev_err, KVQ_DEVERR_PAGE_RANGE);
-                continue;
-            }
-            // per group: float16 (s, z), reciprocal, zero flag
+            // every lane of the warp takes part in the TMEM loads (warp-wide instructions)
+            // ---- pass 1: clip parameters per group
             float zf[NG], sf[NG], rc[NG];
             bool zero[NG];
+            {
+                float x[32];
+                float lo = 0.f, hi = 0.f;
+                float m1 = INFINITY, m2 = INFINITY, M1 = -INFINITY, M2 = -INFINITY;
+                float sm9[9], lg9[9];
+                double ss = 0.0;
 #pragma unroll
-            for (int gr = 0; gr < NG; ++gr) {
-                const float *xg = x + gr * GS;
-                __half sh, zh;
-                bool finite;
-                if (P.clip == kQuestClip) {
-                    double ss = 0.0;
+                for (int c = 0; c < D / 32; ++c) {
+                    const int gr = (32 * c) / GS;
+                    const bool first = (32 * c) % GS == 0, last = (32 * c + 32) % GS == 0;
+                    tmem_ld32_f(taddr + 32 * c, x);
+                    if (first) {
+                        lo = INFINITY;
+                        hi = -INFINITY;
+                        m1 = m2 = INFINITY;
+                        M1 = M2 = -INFINITY;
+                        ss = 0.0;
 #pragma unroll
-                    for (int j = 0; j < GS; ++j)
-                        ss = fma((double)xg[j], (double)xg[j], ss);
-                    const float rms = __double2float_rn(sqrt(ss / (double)GS));
-                    const float s = __fmul_rn(rms, quest_delta(bits));
-                    sh = __float2half_rn(s);
-                    zh = __float2half_rn(__fmul_rn(-0.5f * qmax, __half2float(sh)));
-                    finite = isfinite(s);
-                } else {
-                    float lo, hi;
-                    clip_range<GS>(xg, P.clip, lo, hi);
-                    const float range = __fsub_rn(hi, lo);
-                    const float s = __fdiv_rn(range, qmax);
-                    sh = __float2half_rn(s);
-                    zh = __float2half_rn(lo);
-                    finite = isfinite(range) && isfinite(s);
-                }
-                sf[gr] = __half2float(sh);
-                zf[gr] = __half2float(zh);
-                zero[gr] = !finite || sf[gr] == 0.f;
-                rc[gr] = zero[gr] ? 0.f : __frcp_rn(sf[gr]);
-                if (!finite)
-                    flag(P.dev_err, KVQ_DEVERR_NONFINITE);
-                (which ? P.v_sz : P.k_sz)[row * ng + gr] =
-                    (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
-            }
-            if (!which) {
-                // K row: little-endian bit stream, dim j at bit bits*j; stored as 16-byte pieces
-                uint32_t *dst = reinterpret_cast<uint32_t *>(P.k_codes + row * (D * bits / 8));
-                if (bits == 2) {
-#pragma unroll
-                    for (int w4 = 0; w4 < D / 64; ++w4) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t acc = 0;
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                const int j = 64 * w4 + 16 * q + e, gr = j / GS;
-                                acc |= code_of(x[j], zf[gr], sf[gr], rc[gr], zero[gr], qmax) << (2 * e);
-                            }
-                            w[q] = acc;
+                        for (int e = 0; e < 9; ++e) {
+                            sm9[e] = INFINITY;
+                            lg9[e] = -INFINITY;
                         }
-                        reinterpret_cast<uint4 *>(dst)[w4] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                } else {
+                    if (quest) {
 #pragma unroll
-                    for (int w4 = 0; w4 < D / 32; ++w4) {
-                        uint32_t w[4];
+                        for (int j = 0; j < 32; ++j)
+                            ss = fma((double)x[j], (double)x[j], ss);
+                    } else if (P.clip == 0) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t acc = 0;
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int j = 32 * w4 + 8 * q + e, gr = j / GS;
-                                acc |= code_of(x[j], zf[gr], sf[gr], rc[gr], zero[gr], qmax) << (4 * e);
-                            }
-                            w[q] = acc;
+                        for (int j = 0; j < 32; j += 2) {
+                            lo = fmin3(lo, x[j], x[j + 1]);
+                            hi = fmax3(hi, x[j], x[j + 1]);
                         }
-                        reinterpret_cast<uint4 *>(dst)[w4] = make_uint4(w[0], w[1], w[2], w[3]);
+                    } else if (P.clip == 1) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float v = x[j];
+                            m2 = fminf(m2, fmaxf(m1, v));
+                            m1 = fminf(m1, v);
+                            M2 = fmaxf(M2, fminf(M1, v));
+                            M1 = fmaxf(M1, v);
+                        }
+                    } else {
+                        // kappa <= 8: the 9 smallest and 9 largest by insertion
+                        for (int j = 0; j < 32; ++j) {
+                            float av = x[j], bv = x[j];
+#pragma unroll
+                            for (int e = 0; e < 9; ++e) {
+                                const float s0 = fminf(sm9[e], av), s1 = fmaxf(sm9[e], av);
+                                sm9[e] = s0;
+                                av = s1;
+                                const float l0 = fmaxf(lg9[e], bv), l1 = fminf(lg9[e], bv);
+                                lg9[e] = l0;
+                                bv = l1;
+                            }
+                        }
                     }
-                }
-            } else {
-                // V tile halves of this token: half (gq, rr) holds dims 8(E rr + s) + gq
-                unsigned char *tile_base =
-                    P.v_codes + (size_t)(row / kTileTokens) * (kTileTokens * D * bits / 8);
-                const int tok = (int)(row % kTileTokens);
-                if (bits == 2) {
-                    constexpr int E = 8, W = D * 2 / 128;
+                    if (last) {
+                        __half sh, zh;
+                        bool finite;
+                        if (quest) {
+                            const float rms = __double2float_rn(sqrt(ss / (double)GS));
+                            const float s = __fmul_rn(rms, quest_delta(bits));
+                            sh = __float2half_rn(s);
+                            zh = __float2half_rn(__fmul_rn(-0.5f * qmax, __half2float(sh)));
+                            finite = isfinite(s);
+                        } else {
+                            if (P.clip == 1) {
+                                lo = m2;
+                                hi = M2;
+                            } else if (P.clip > 1) {
+                                lo = sm9[0];
+                                hi = lg9[0];
 #pragma unroll
-                    for (int gq = 0; gq < 8; ++gq)
-#pragma unroll
-                        for (int rr = 0; rr < W; ++rr) {
-                            uint32_t hv = 0;
-#pragma unroll
-                            for (int s2 = 0; s2 < E; ++s2) {
-                                const int j = 8 * (E * rr + s2) + gq, gr = j / GS;
-                                hv |= code_of(x[j], zf[gr], sf[gr], rc[gr], zero[gr], qmax) << (2 * s2);
+                                for (int e = 1; e < 9; ++e)
+                                    if (e == P.clip) {
+                                        lo = sm9[e];
+                                        hi = lg9[e];
+                                    }
                             }
-                            *reinterpret_cast<uint16_t *>(tile_base + v_half_offset(D, 2, tok, gq, rr)) =
-                                (uint16_t)hv;
+                            const float range = __fsub_rn(hi, lo);
+                            const float s = __fdiv_rn(range, qmax);
+                            sh = __float2half_rn(s);
+                            zh = __float2half_rn(lo);
+                            finite = isfinite(range) && isfinite(s);
                         }
-                } else {
-                    constexpr int E = 4, W = D * 4 / 128;
-#pragma unroll
-                    for (int gq = 0; gq < 8; ++gq)
-#pragma unroll
-                        for (int rr = 0; rr < W; ++rr) {
-                            uint32_t hv = 0;
-#pragma unroll
-                            for (int s2 = 0; s2 < E; ++s2) {
-                                const int j = 8 * (E * rr + s2) + gq, gr = j / GS;
-                                hv |= code_of(x[j], zf[gr], sf[gr], rc[gr], zero[gr], qmax) << (4 * s2);
-                            }
-                            *reinterpret_cast<uint16_t *>(tile_base + v_half_offset(D, 4, tok, gq, rr)) =
-                                (uint16_t)hv;
+                        sf[gr] = __half2float(sh);
+                        zf[gr] = __half2float(zh);
+                        zero[gr] = !finite || sf[gr] == 0.f;
+                        rc[gr] = zero[gr] ? 0.f : __frcp_rn(sf[gr]);
+                        if (row >= 0) {
+                            if (!finite)
+                                flag(P.dev_err, KVQ_DEVERR_NONFINITE);
+                            (which ? P.v_sz : P.k_sz)[row * NG + gr] =
+                                (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
                         }
+                    }
                 }
             }
+            // ---- pass 2: codes; pass 3 (rows near a rounding tie only): the same by division
+            bool tie = false;
+            if (!which)
+                store_k_row<D, GS, NG>(P, row, bits, taddr, zf, sf, rc, zero, qmax, tie, false);
+            else
+                store_v_token<D, GS, NG>(P, row, bits, taddr, zf, sf, rc, zero, qmax, tie, false);
+            if (__any_sync(0xffffffffu, tie)) {
+                if (!which)
+                    store_k_row<D, GS, NG>(P, tie ? row : -1, bits, taddr, zf, sf, rc, zero, qmax,
+                                           tie, true);
+                else
+                    store_v_token<D, GS, NG>(P, tie ? row : -1, bits, taddr, zf, sf, rc, zero, qmax,
+                                             tie, true);
+            }
+            tc_fence_before_sync();
+            mbar_arrive(&acce[a]);                          // the MMA warp may reuse it
         }
     }
 

@@ -15,7 +15,7 @@ import torch
 import decode_attention_post_b200 as kvq
 import oracle
 from tests import synth
-from tests.test_gpu_parity import assert_close, qp_of, t_
+from tests.test_gpu_parity import assert_close, host_cache_from, qp_of, t_, upload_cache
 
 pytestmark = pytest.mark.gpu
 
@@ -133,7 +133,8 @@ def test_window_append_serving_loop(ci, prefill, steps, S_sink, S_keep, S_flush)
             Q = st.Q(st.len[b])
             assert np.array_equal(g[b, :, :Q * w], r[b, :, :Q * w]), b
     assert Qmax > 0
-    # ---- the windowed decode over this state against the oracle's windowed decode
+    # ---- the oracle quantizes every position of the history itself; the GPU's quantized
+    #      middle matches its codes end to end (<= 0.1% of codes off by one, s/z <= 1 ulp)
     Lmax = int(st.len.max())
     Tfull = 64 * ((Lmax + 63) // 64)
     kall = np.zeros((B, Tfull, cfg.Hkv, cfg.d), np.uint16)
@@ -143,17 +144,51 @@ def test_window_append_serving_loop(ci, prefill, steps, S_sink, S_keep, S_flush)
     ofull = oracle.Cache(B, cfg.Hkv, Tfull, cfg.d, cfg.bits_k, cfg.bits_v, cfg.group)
     oracle.quantize_append(kall, vall, st.Tk_h, st.Tv_h, cfg.bits_k, cfg.bits_v, cfg.group,
                            cfg.clip_alpha, ofull, np.zeros(B, np.int32))
+    gh = host_cache_from(st.cache, cfg)
+    diff = total = 0
+    for b in range(B):
+        Q = st.Q(st.len[b])
+        for h in range(cfg.Hkv):
+            if Q == 0:
+                continue
+            gk, gv, gks, gvs = gh.unpack_tokens(b, h, 0, Q)
+            ok_, ov, oks, ovs = ofull.unpack_tokens(b, h, S_sink, Q)
+            for x, y in ((gk, ok_), (gv, ov)):
+                dlt = x.astype(np.int32) - y.astype(np.int32)
+                assert np.abs(dlt).max() <= 1
+                diff += np.count_nonzero(dlt)
+                total += dlt.size
+            for x, y in ((gks, oks), (gvs, ovs)):
+                assert np.abs(x.astype(np.int32) - y.astype(np.int32)).max() <= 1
+    assert diff <= 1e-3 * total, diff / total
+    # ---- decode parity over the same cache: the oracle's quantized middle at cache
+    #      positions [0, Q), the sink and ring as kvq_window_append left them (checked
+    #      above to be the exact tokens), against the oracle's windowed decode
+    Tc = st.cache.T_cap
+    om = oracle.Cache(B, cfg.Hkv, Tc, cfg.d, cfg.bits_k, cfg.bits_v, cfg.group)
+    for b in range(B):
+        Q = st.Q(st.len[b])
+        for h in range(cfg.Hkv):
+            if Q:
+                om.pack_tokens(b, h, 0, *ofull.unpack_tokens(b, h, S_sink, Q))
+    gc = upload_cache(om, cfg)
     q = synth.as_dtype(synth.queries(cfg.with_(B=B)), "bf16")
     want = oracle.window_decode(q, st.Tit_h, st.Tv_h, kall, vall, ofull, st.len, S_sink, S_keep,
                                 S_flush)
     out = torch.empty((B, cfg.Hq, cfg.d), dtype=torch.float32, device=DEV)
-    ws = torch.empty(kvq.decode_workspace_bytes(st.cache, cfg.Hq, st.cache.T_cap),
-                     dtype=torch.uint8, device=DEV)
-    kvq.decode_attention_window(t_(q), st.Tit, st.cache, S_sink, S_keep, S_flush, st.ks, st.vs,
+    ws = torch.empty(kvq.decode_workspace_bytes(gc, cfg.Hq, Tc), dtype=torch.uint8, device=DEV)
+    kvq.decode_attention_window(t_(q), st.Tit, gc, S_sink, S_keep, S_flush, st.ks, st.vs,
                                 st.kr, st.vr, st.Tv, t_(st.len), Lmax, out, ws, dev_err=st.err)
     torch.cuda.synchronize()
     assert st.err.item() == 0
     assert_close(out.cpu().numpy(), want, where=f"window append {S_sink}/{S_keep}/{S_flush}")
+    # ---- and end to end over the GPU's own state: the same attention up to the code
+    #      differences above (relative L2 only)
+    kvq.decode_attention_window(t_(q), st.Tit, st.cache, S_sink, S_keep, S_flush, st.ks, st.vs,
+                                st.kr, st.vr, st.Tv, t_(st.len), Lmax, out, ws, dev_err=st.err)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    assert np.linalg.norm(got - want) <= 1e-3 * np.linalg.norm(want)
 
 
 def test_window_append_out_of_range_is_flagged_and_skipped():
