@@ -68,6 +68,11 @@ def lib():
         L.oracle_window_decode.argtypes = [P, I, I, I, I, I, P, P, P, P, I, I, I, I, I,
                                            P, P, P, P, P, I, I, I, P]
         L.oracle_window_decode.restype = I
+        L.oracle_vq_encode.argtypes = [P, I, P, P, P]
+        L.oracle_vq_append.argtypes = [P, P, I, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, P]
+        L.oracle_vq_append.restype = I
+        L.oracle_vq_decode.argtypes = [P, I, I, I, I, I, P, P, P, I, P, P, P, P, P, P, I, P]
+        L.oracle_vq_decode.restype = I
         L.oracle_set_threads.argtypes = [I]
         L.oracle_get_threads.restype = I
         _lib = L
@@ -406,3 +411,73 @@ def build_cache_from_fields(cfg, fields_per_b, tokens):
         for h in range(cfg.Hkv):
             c.pack_tokens(b, h, 0, kc[h], vc[h], ksz[h], vsz[h])
     return c
+
+
+# ------------------------------------------------------------------ NOVA-KV vector quantization
+
+VQ_DIM, VQ_SIZE = 4, 256
+
+
+def vq_encode(x, cb):
+    """(idx uint8 [d/4], gain float16 bits) of one transformed token x [d] (float32) with
+    codebook cb [256][4] float16 bits."""
+    x = _c(x, np.float32)
+    cb = _c(cb, np.uint16)
+    d = x.shape[0]
+    idx = np.empty(d // VQ_DIM, np.uint8)
+    g = np.zeros(1, np.uint16)
+    lib().oracle_vq_encode(_p(x), d, _p(cb), _p(idx), _p(g))
+    return idx, int(g[0])
+
+
+class VQCache:
+    """Host planes of a vector-quantized cache: indices [B][Hkv][T_cap][d/4] uint8 and
+    gains [B][Hkv][T_cap] float16 bits, for keys and values."""
+
+    def __init__(self, B, Hkv, T_cap, d):
+        self.B, self.Hkv, self.T_cap, self.d = B, Hkv, T_cap, d
+        self.k_idx = np.zeros(B * Hkv * T_cap * (d // VQ_DIM), np.uint8)
+        self.v_idx = np.zeros_like(self.k_idx)
+        self.k_gain = np.zeros(B * Hkv * T_cap, np.uint16)
+        self.v_gain = np.zeros_like(self.k_gain)
+
+    def planes(self):
+        return self.k_idx, self.k_gain, self.v_idx, self.v_gain
+
+
+def vq_append(k, v, T_k, T_v, cb_k, cb_v, cache: VQCache, pos, return_transformed=False):
+    """k, v [B][n][Hkv][d] float32 or bf16 bits; T_k, T_v [Hkv][d][d] float32 or None;
+    codebooks [Hkv][256][4] float16 bits."""
+    dt = _dt(k)
+    k, v = np.ascontiguousarray(k), np.ascontiguousarray(v)
+    B, n, Hkv, d = k.shape
+    Tk = None if T_k is None else _c(T_k, np.float32)
+    Tv = None if T_v is None else _c(T_v, np.float32)
+    ck, cv = _c(cb_k, np.uint16), _c(cb_v, np.uint16)
+    pos = _c(pos, np.int32)
+    kt = np.empty((B, n, Hkv, d), np.float32) if return_transformed else None
+    vt = np.empty((B, n, Hkv, d), np.float32) if return_transformed else None
+    r = lib().oracle_vq_append(_p(k), _p(v), dt, _p(Tk), _p(Tv), _p(ck), _p(cv), B, n, Hkv, d,
+                               cache.T_cap, _p(pos), _p(cache.k_idx), _p(cache.k_gain),
+                               _p(cache.v_idx), _p(cache.v_gain), _p(kt), _p(vt))
+    if r:
+        raise ValueError("oracle_vq_append: bad arguments")
+    return (kt, vt) if return_transformed else None
+
+
+def vq_decode(q, M, cb_k, cb_v, cache: VQCache, seqlens, sel=None) -> np.ndarray:
+    dt = _dt(q)
+    q = np.ascontiguousarray(q)
+    B, Hq, d = q.shape
+    Mc = None if M is None else _c(M, np.float32)
+    ck, cv = _c(cb_k, np.uint16), _c(cb_v, np.uint16)
+    seqlens = _c(seqlens, np.int32)
+    out = np.full((B, Hq, d), np.nan, np.float64)
+    selc = None if sel is None else _c(sel, np.int32).reshape(-1, 2)
+    nsel = 0 if selc is None else selc.shape[0]
+    r = lib().oracle_vq_decode(_p(q), dt, B, Hq, cache.Hkv, d, _p(Mc), _p(ck), _p(cv),
+                               cache.T_cap, _p(cache.k_idx), _p(cache.k_gain), _p(cache.v_idx),
+                               _p(cache.v_gain), _p(seqlens), _p(selc), nsel, _p(out))
+    if r:
+        raise ValueError("oracle_vq_decode: bad arguments")
+    return out

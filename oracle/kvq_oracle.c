@@ -21,6 +21,9 @@
  *   - WUSH-KV page, section 4.4: the full-precision window (first S_sink and newest
  *     S_keep positions kept in full precision, the middle quantized in batches of
  *     S_flush) -- the decode over such a sequence.
+ *   - WUSH-KV page, section 4.3: the QuEST INT quantizer (RMS-based clipped levels).
+ *   - "Spend Bits Where Queries Look" (NOVA-KV project page): the vector-quantized cache
+ *     (codebook lookup plus one multiply on the read path).
  * Every step the pages leave open is stated next to the code that fixes it.
  *
  * Arithmetic: all transform and attention arithmetic is float64. Where the quantizer
@@ -853,6 +856,174 @@ int oracle_window_decode(const void *q, int q_dtype, int B, int Hq, int Hkv, int
             }
             for (int j = 0; j < d; ++j)
                 o[j] += p * val[j];
+        }
+        for (int j = 0; j < d; ++j)
+            out[((size_t)b * Hq + hq) * d + j] = l > 0 ? o[j] / l : 0.0;
+        free(logit);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ NOVA-KV vector quantization */
+
+/*
+ * Vector-quantized cache ("Spend Bits Where Queries Look: KV Cache Vector Quantization with
+ * Attention-Preserving Transforms", NOVA-KV project page: transformed keys and values are
+ * encoded once on the write path into a fixed-width cache; "the read path ... is a
+ * codebook lookup plus one multiply"; equal-size codebooks keep every token the same
+ * width). The page fixes neither the sub-vector size nor the codebook layout. Reading:
+ *   - the d transformed coefficients of a token form d/4 groups of 4 consecutive
+ *     coefficients, each coded by an 8-bit index into a codebook of 256 four-dimensional
+ *     codewords (float16), one codebook per KV head for keys and one for values, shared
+ *     by the groups: 2 bits per coefficient;
+ *   - the "one multiply" is a per-token gain g (float16): x^_group = g * C[idx];
+ *   - encoding: g = f16(f32(sqrt(sum_j x_j^2 / d))) (sum in float64), then per group the
+ *     index of the codeword nearest to the coefficients after scaling by g, in float32 with
+ *     a fixed operation order (this decides an integer, so both sides compute it the same
+ *     way): e_m = f32(x_m - f32(g * c_m)) (the product is exact), dist = f32(e_0 * e_0),
+ *     then dist = fmaf(e_m, e_m, dist) for m = 1, 2, 3; the smallest dist wins, ties to
+ *     the lowest index. g == 0 codes every group as index 0.
+ * Layout: idx planes [B][Hkv][T_cap][d/4] bytes, gain planes [B][Hkv][T_cap] float16,
+ * codebooks [Hkv][256][4] float16.
+ */
+#define VQ_DIM 4
+#define VQ_SIZE 256
+
+void oracle_vq_encode(const float *x, int d, const uint16_t *cb, uint8_t *idx, uint16_t *gain)
+{
+    double ss = 0.0;
+    for (int j = 0; j < d; ++j)
+        ss += (double)x[j] * (double)x[j];
+    float rms = (float)sqrt(ss / (double)d);
+    uint16_t gh = oracle_f32_to_f16(rms);
+    float g = (float)oracle_f16_to_f64(gh);
+    *gain = gh;
+    for (int grp = 0; grp < d / VQ_DIM; ++grp) {
+        int best = 0;
+        if (g != 0.0f) {
+            float bestd = INFINITY;
+            for (int i = 0; i < VQ_SIZE; ++i) {
+                float dist = 0.0f;
+                for (int m = 0; m < VQ_DIM; ++m) {
+                    float c = (float)oracle_f16_to_f64(cb[i * VQ_DIM + m]);
+                    float e = f32((double)x[grp * VQ_DIM + m] - (double)f32((double)g * c));
+                    dist = m == 0 ? f32((double)e * e) : fmaf(e, e, dist);
+                }
+                if (dist < bestd) {
+                    bestd = dist;
+                    best = i;
+                }
+            }
+        }
+        idx[grp] = (uint8_t)best;
+    }
+}
+
+/* Write path: x~ = f32(T x) in float64 (as oracle_quantize_append), then the encoder above;
+ * token i of sequence b goes to position pos[b] + i. cb_k, cb_v: [Hkv][256][4] float16. */
+int oracle_vq_append(const void *k, const void *v, int in_dtype, const float *T_k,
+                     const float *T_v, const uint16_t *cb_k, const uint16_t *cb_v, int B, int n,
+                     int Hkv, int d, int T_cap, const int32_t *pos, uint8_t *k_idx,
+                     uint16_t *k_gain, uint8_t *v_idx, uint16_t *v_gain, float *kt_out,
+                     float *vt_out)
+{
+    if (d <= 0 || d > 1024 || d % VQ_DIM)
+        return -1;
+    for (int b = 0; b < B; ++b)
+        if (pos[b] < 0 || pos[b] + n > T_cap)
+            return -1;
+    long total = (long)B * n * Hkv;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (long u = 0; u < total; ++u) {
+        int h = (int)(u % Hkv);
+        int i = (int)((u / Hkv) % n);
+        int b = (int)(u / ((long)Hkv * n));
+        double xin[1024];
+        float xf[1024];
+        for (int which = 0; which < 2; ++which) {
+            const void *src = which ? v : k;
+            const float *T = which ? T_v : T_k;
+            size_t base = (((size_t)b * n + i) * Hkv + h) * d;
+            for (int j = 0; j < d; ++j)
+                xin[j] = load_in(src, in_dtype, base + j);
+            for (int r = 0; r < d; ++r) {
+                double acc = 0.0;
+                if (T) {
+                    const float *Th = T + (size_t)h * d * d;
+                    for (int j = 0; j < d; ++j)
+                        acc += (double)Th[(size_t)r * d + j] * xin[j];
+                } else {
+                    acc = xin[r];
+                }
+                xf[r] = (float)acc;
+            }
+            float *dump = which ? vt_out : kt_out;
+            if (dump)
+                memcpy(dump + base, xf, sizeof(float) * d);
+            size_t slot = ((size_t)b * Hkv + h) * T_cap + pos[b] + i;
+            const uint16_t *cb = (which ? cb_v : cb_k) + (size_t)h * VQ_SIZE * VQ_DIM;
+            oracle_vq_encode(xf, d, cb, (which ? v_idx : k_idx) + slot * (d / VQ_DIM),
+                             (which ? v_gain : k_gain) + slot);
+        }
+    }
+    return 0;
+}
+
+/* Dequantized token of a VQ cache: x^_j = g * C[idx_{j/4}][j%4] (exact in float64). */
+static void vq_load_token(const uint8_t *idx_plane, const uint16_t *gain_plane, const uint16_t *cb,
+                          int d, size_t slot, double *xhat)
+{
+    double g = oracle_f16_to_f64(gain_plane[slot]);
+    const uint8_t *row = idx_plane + slot * (d / VQ_DIM);
+    for (int j = 0; j < d; ++j)
+        xhat[j] = g * oracle_f16_to_f64(cb[(size_t)row[j / VQ_DIM] * VQ_DIM + j % VQ_DIM]);
+}
+
+/* Decode attention over a VQ cache: softmax_t((1/sqrt(d)) (M q) . k^_t) v^_t over t <
+ * seqlens[b], as oracle_decode with the dequantization above. sel as in oracle_decode. */
+int oracle_vq_decode(const void *q, int q_dtype, int B, int Hq, int Hkv, int d, const float *M,
+                     const uint16_t *cb_k, const uint16_t *cb_v, int T_cap,
+                     const uint8_t *k_idx, const uint16_t *k_gain, const uint8_t *v_idx,
+                     const uint16_t *v_gain, const int32_t *seqlens, const int32_t *sel,
+                     int nsel, double *out)
+{
+    if (Hkv <= 0 || Hq % Hkv || d > 1024 || d % VQ_DIM)
+        return -1;
+    int npairs = sel ? nsel : B * Hq;
+    for (int u = 0; u < npairs; ++u) {
+        int b = sel ? sel[2 * u] : u / Hq, hq = sel ? sel[2 * u + 1] : u % Hq;
+        if (b < 0 || b >= B || hq < 0 || hq >= Hq || seqlens[b] < 0 || seqlens[b] > T_cap)
+            return -1;
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int u = 0; u < npairs; ++u) {
+        int b = sel ? sel[2 * u] : u / Hq, hq = sel ? sel[2 * u + 1] : u % Hq;
+        int G = Hq / Hkv, h = hq / G, L = seqlens[b];
+        double qt[1024], o[1024], xh[1024];
+        double sm = 1.0 / sqrt((double)d);
+        query_transform(q, q_dtype, M, Hq, Hkv, d, b, hq, qt);
+        const uint16_t *ck = cb_k + (size_t)h * VQ_SIZE * VQ_DIM;
+        const uint16_t *cv = cb_v + (size_t)h * VQ_SIZE * VQ_DIM;
+        double *logit = (double *)malloc(sizeof(double) * (L > 0 ? L : 1));
+        double m = -INFINITY;
+        for (int t = 0; t < L; ++t) {
+            vq_load_token(k_idx, k_gain, ck, d, ((size_t)b * Hkv + h) * T_cap + t, xh);
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j)
+                acc += qt[j] * xh[j];
+            logit[t] = sm * acc;
+            if (logit[t] > m)
+                m = logit[t];
+        }
+        double l = 0.0;
+        for (int j = 0; j < d; ++j)
+            o[j] = 0.0;
+        for (int t = 0; t < L; ++t) {
+            double p = exp(logit[t] - m);
+            l += p;
+            vq_load_token(v_idx, v_gain, cv, d, ((size_t)b * Hkv + h) * T_cap + t, xh);
+            for (int j = 0; j < d; ++j)
+                o[j] += p * xh[j];
         }
         for (int j = 0; j < d; ++j)
             out[((size_t)b * Hq + hq) * d + j] = l > 0 ? o[j] / l : 0.0;

@@ -28,6 +28,7 @@ import math
 import numpy as np
 
 STREAM_K, STREAM_V, STREAM_Q, STREAM_TK, STREAM_TV, STREAM_SEQ, STREAM_CACHE = 1, 2, 3, 4, 5, 6, 7
+STREAM_CODEBOOK = 8
 
 
 @dataclasses.dataclass(frozen=True)
@@ -244,3 +245,16 @@ def random_cache_fields(cfg: Config, b: int, tokens: int):
     vs = f16(r.uniform(0.2, 1.5, size=(cfg.Hkv, tokens, ng)))
     vz = f16(r.uniform(-2.5, -0.5, size=(cfg.Hkv, tokens, ng)))
     return kc, vc, ks, kz, vs, vz
+
+
+def codebooks(cfg: Config):
+    """Synthetic vector-quantization codebooks (codebook training is out of scope): for
+    keys and values, per KV head, 256 four-dimensional codewords drawn N(0, 1) and rounded
+    to float16 (the encoder scales tokens to unit RMS first). Returns (cb_k, cb_v) as
+    float16 bit patterns uint16 [Hkv][256][4]."""
+    r = _rng(cfg, STREAM_CODEBOOK)
+    out = []
+    for _ in range(2):
+        c = r.standard_normal((cfg.Hkv, 256, 4)).astype(np.float16)
+        out.append(np.ascontiguousarray(c).view(np.uint16))
+    return out[0], out[1]
