@@ -182,3 +182,32 @@ def test_vq_append_codes_the_transformed_tokens():
             assert c.k_gain[slot] == gk and c.v_gain[slot] == gv
             want = np.float64(Tk[h]).astype(np.float64) @ k[0, i, h].astype(np.float64)
             assert np.array_equal(kt[0, i, h], want.astype(np.float32))
+
+
+def test_vq_encoder_uses_the_float16_gain():
+    """Codewords on a line, c_i = (i / 64, 0, 0, 0); tokens (x0, 0, 0, 0, x1, 0, 0, 0) with
+    random x0, x1. The nearest codeword to x0 / g moves when g changes by its float16
+    rounding (about 1e-3 of a target, a tenth of the spacing), so an encoder that scaled by
+    the unrounded RMS picks other indices for some of these tokens."""
+    c = np.zeros((256, 4), np.float16)
+    c[:, 0] = (np.arange(256) / 64.0).astype(np.float16)
+    cb = c.view(np.uint16)
+    rng = np.random.default_rng(7)
+    flips = 0
+    for _ in range(200):
+        x0, x1 = rng.uniform(0.2, 3.0, size=2)
+        x = np.zeros(8, np.float32)
+        x[0], x[4] = x0, x1
+        idx, gh = oracle.vq_encode(x, cb)
+        g = np.float32(np.array(gh, np.uint16).view(np.float16))
+        want = []
+        for t in (x[0], x[4]):
+            d = [np.float32(np.float32(t - np.float32(g * c[i, 0].astype(np.float32))) ** 2)
+                 for i in range(256)]
+            want.append(int(np.argmin(d)))                 # first minimum: lowest index
+        assert idx.tolist() == want
+        rms = np.float32(np.sqrt(np.sum(x.astype(np.float64) ** 2) / 8))
+        raw = [int(np.argmin([(t - rms * c[i, 0].astype(np.float32)) ** 2 for i in range(256)]))
+               for t in (x[0], x[4])]
+        flips += raw != want
+    assert flips > 0                                   # the test can tell the two gains apart
