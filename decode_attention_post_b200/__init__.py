@@ -17,6 +17,7 @@ from .kvq import (  # noqa: F401
     KvqError,
     KVCache,
     QParams,
+    VQCache,
     bf16_decode,
     bf16_decode_workspace_bytes,
     cache_plane_bytes,
@@ -27,5 +28,8 @@ from .kvq import (  # noqa: F401
     library_path,
     load,
     quantize_append,
+    vq_append,
+    vq_decode_attention,
+    vq_decode_workspace_bytes,
     window_append,
 )

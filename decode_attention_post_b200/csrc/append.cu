@@ -261,8 +261,6 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
     const long total = (long)B * n;
     const long tiles = (total + kTokPerTile - 1) / kTokPerTile;
     constexpr int R = D / 32;                   // dims per lane
-    const int ng = D / group;
-    const int qmax = (1 << bits) - 1;
 
     // T_h staged transposed; a window flush stages it only once the CTA meets a tile with
     // work (most CTAs of a decode-time flush have none)

@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kQprepThreads)
 qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M, int B, int Hq,
              int Hkv, int bb, const int32_t *__restrict__ seqlens, int max_seqlen, void *out,
              int out_bf16, uint32_t *__restrict__ qfrag, float *__restrict__ qscale,
-             float *__restrict__ qw, int *__restrict__ ticket)
+             float *__restrict__ qw, int *__restrict__ ticket, float *__restrict__ qt_out)
 {
     constexpr int CPB = 8 / BK, NT = (2 * G) / 8, WPT = D * BK / 128;
     constexpr int KCH = WPT >= 2 ? WPT / 2 : 1, KS = CPB * KCH;
@@ -235,6 +235,12 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
         __syncthreads();
     }
     const float *qt = pt;                         // [NVMAX][D]
+    if (qt_out) {                                 // q~ itself, for the vector-quantized decode
+        for (int idx = tid; idx < NV * D; idx += kQprepThreads) {
+            const int v = idx / D, j = idx % D;
+            qt_out[((size_t)(b0 + v / G) * Hq + h * G + v % G) * D + j] = qt[idx];
+        }
+    }
     // per sequence: max |q~| over its G heads; per head: sum of q~
     const int warp = tid >> 5, lane = tid & 31;
     const float sm = rsqrtf((float)D);
@@ -754,7 +760,7 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
         qprep_kernel<D, G, BK><<<grid, kQprepThreads, QS::BYTES, st>>>(
             L.q, L.q_bf16, L.M, L.p.B, L.p.Hq, L.p.Hkv, kQprepSeqs, L.p.seqlens, L.p.max_seqlen,
             L.p.out, L.p.out_bf16, const_cast<uint32_t *>(L.p.qfrag),
-            const_cast<float *>(L.p.qscale), const_cast<float *>(L.p.qw), L.p.ticket);
+            const_cast<float *>(L.p.qscale), const_cast<float *>(L.p.qw), L.p.ticket, nullptr);
         e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
@@ -782,9 +788,68 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
     return cudaLaunchKernelEx(&cfg, decode_kernel<D, G, BK, BV>, L.p);
 }
 
+template <int D, int G>
+cudaError_t launch_qprep_qt_t(const DecodeLaunch &L, float *qt_out, cudaStream_t st)
+{
+    using QS = QprepSmem<D, G>;
+    static unsigned long long attr = 0;
+    cudaError_t e = ensure_dynamic_smem(qprep_kernel<D, G, 2>, QS::BYTES, attr);
+    if (e != cudaSuccess)
+        return e;
+    dim3 grid(L.p.Hkv, (L.p.B + kQprepSeqs - 1) / kQprepSeqs);
+    qprep_kernel<D, G, 2><<<grid, kQprepThreads, QS::BYTES, st>>>(
+        L.q, L.q_bf16, L.M, L.p.B, L.p.Hq, L.p.Hkv, kQprepSeqs, L.p.seqlens, L.p.max_seqlen,
+        L.p.out, L.p.out_bf16, const_cast<uint32_t *>(L.p.qfrag), const_cast<float *>(L.p.qscale),
+        const_cast<float *>(L.p.qw), L.p.ticket, qt_out);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t decode_qfrag_words(int d, int G) { return (size_t)((2 * G) / 8) * (d / 16) * 64; }
+
+// Resident decode CTAs per SM of the instantiation for (d, G, bits_k, bits_v) (registers
+// and shared memory), for the host's split count.
+int decode_resident_ctas(int d, int G, int bk, int bv)
+{
+#define KVQ_RES(DD, GG, KK, VV)                                        \
+    if (d == DD && G == GG && bk == KK && bv == VV)                    \
+        return Cfg<DD, GG, KK, VV>::MINB;
+    KVQ_RES(128, 4, 2, 2)
+    KVQ_RES(128, 4, 4, 2)
+    KVQ_RES(128, 4, 2, 4)
+    KVQ_RES(128, 4, 4, 4)
+    KVQ_RES(128, 8, 2, 2)
+    KVQ_RES(128, 8, 4, 2)
+    KVQ_RES(128, 8, 2, 4)
+    KVQ_RES(128, 8, 4, 4)
+    KVQ_RES(64, 4, 2, 2)
+    KVQ_RES(64, 4, 4, 2)
+    KVQ_RES(64, 4, 2, 4)
+    KVQ_RES(64, 4, 4, 4)
+    KVQ_RES(64, 8, 2, 2)
+    KVQ_RES(64, 8, 4, 2)
+    KVQ_RES(64, 8, 2, 4)
+    KVQ_RES(64, 8, 4, 4)
+#undef KVQ_RES
+    return kDecodeMinBlocks;
+}
+
+// The query prologue alone, also writing q~ (float32 [B][Hq][d]) to qt_out: the first
+// kernel of the vector-quantized decode (it also zeroes the merge tickets and writes the
+// zero output of empty sequences).
+cudaError_t launch_qprep_qt(const DecodeLaunch &L, float *qt_out, cudaStream_t st)
+{
+    if (L.d == 128 && L.G == 4)
+        return launch_qprep_qt_t<128, 4>(L, qt_out, st);
+    if (L.d == 128 && L.G == 8)
+        return launch_qprep_qt_t<128, 8>(L, qt_out, st);
+    if (L.d == 64 && L.G == 4)
+        return launch_qprep_qt_t<64, 4>(L, qt_out, st);
+    if (L.d == 64 && L.G == 8)
+        return launch_qprep_qt_t<64, 8>(L, qt_out, st);
+    return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_decode(const DecodeLaunch &L, cudaStream_t st)
 {

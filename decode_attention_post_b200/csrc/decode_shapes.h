@@ -72,12 +72,25 @@ struct DecodeLaunch {
 
 // Byte offsets of the decode workspace sections (each 256-byte aligned).
 struct DecodeWorkspace {
-    size_t qfrag, qscale, qw, part, ticket, total;
+    size_t qfrag, qscale, qw, part, ticket, qt, total;
 };
 
 size_t decode_qfrag_words(int d, int G);
+int decode_resident_ctas(int d, int G, int bk, int bv);
 cudaError_t launch_decode(const DecodeLaunch &L, cudaStream_t st);
 cudaError_t launch_window(const WindowParams &W, cudaStream_t st);
+cudaError_t launch_qprep_qt(const DecodeLaunch &L, float *qt_out, cudaStream_t st);
+
+// Vector-quantized decode: the query prologue (writing q~ to qt) and the VQ decode grid
+// over the same split layout, partials, tickets and output as DecodeLaunch describes.
+struct VqLaunch {
+    DecodeLaunch L;
+    float *qt;
+    const uint8_t *k_idx, *v_idx;
+    const uint16_t *k_gain, *v_gain;
+    const uint16_t *cb_k, *cb_v;
+};
+cudaError_t launch_vq_decode(const VqLaunch &V, cudaStream_t st);
 
 
 }  // namespace kvq

@@ -23,6 +23,11 @@ cudaError_t launch_window_store(const void *k_new, const void *v_new, int B, int
                                 int d, const int32_t *len, int S_sink, int S_keep, int S_flush,
                                 int T_cap, void *k_sink, void *v_sink, void *k_ring, void *v_ring,
                                 cudaStream_t st);
+cudaError_t launch_vq_append(const void *k, const void *v, int in_bf16, const float *Tk,
+                             const float *Tv, const void *cb_k, const void *cb_v, int B, int n,
+                             const kvq_vq_cache *c, const int32_t *pos, int32_t *dev_err,
+                             cudaStream_t st);
+int vq_resident_ctas(int d, int G);
 cudaError_t launch_bf16_decode(const void *q, int Hq, const void *k, const void *v, int B,
                                int Hkv, int T_cap, int d, const int32_t *seqlens, int max_seqlen,
                                void *out, void *ws, int nsplit, int split_tokens,
@@ -131,13 +136,18 @@ static int num_sms()
 }
 
 // Target number of splits per (sequence, KV head), before clamping to the blocks of the
-// sequence: about 4 waves of the resident CTAs per SM over the pairs.
+// sequence. With `resident` CTAs per SM there are slots = SMs * resident places. When
+// there are at least two slots per (sequence, KV head) pair, floor(slots / pairs) splits
+// fill one wave with long CTAs (the per-CTA prologue, ring fill and merge are paid once
+// per split; measured on B200: batch 4 x 128K 0.144 -> 0.096 ms, batch 16 x 16K
+// 0.073 -> 0.055 ms against 4 waves). With fewer, about 4 waves: the short last splits of
+// ragged sequences then fill the tail (batch 64 x U[12K, 16K]: 5 splits best).
 // KVQ_DECODE_SPLITS overrides it (tuning).
-static long target_splits(int B, int Hkv)
+static long target_splits(int B, int Hkv, int resident)
 {
     const long pairs = (long)B * Hkv;
-    const long target = (long)num_sms() * kDecodeMinBlocks * 4;
-    long ns = (target + pairs - 1) / pairs;
+    const long slots = (long)num_sms() * (resident > 0 ? resident : kDecodeMinBlocks);
+    long ns = slots >= 2 * pairs ? slots / pairs : (4 * slots + pairs - 1) / pairs;
     if (const char *e = getenv("KVQ_DECODE_SPLITS"))
         ns = atol(e);
     return ns < 1 ? 1 : ns;
@@ -151,10 +161,10 @@ static int blocks_of(int max_seqlen)
 // Splits along the tokens; each split is a whole number of 64-token blocks. The count
 // is ceil(blocks / ceil(blocks / ns)) with ns = min(target, blocks), which is at most ns;
 // it is not monotonic in max_seqlen (75 blocks over 74 target splits give 38 splits).
-static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens)
+static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens, int resident)
 {
     const int blocks = blocks_of(max_seqlen);
-    long ns = target_splits(B, Hkv);
+    long ns = target_splits(B, Hkv, resident);
     if (ns > blocks)
         ns = blocks;
     const int bps = (int)((blocks + ns - 1) / ns);
@@ -165,9 +175,9 @@ static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens)
 // Split partial slots the workspace holds: min(target, blocks), an upper bound of
 // choose_splits that never decreases as max_seqlen grows, so a workspace sized for a
 // longer max_seqlen always serves a shorter one.
-static int split_slots(int B, int Hkv, int max_seqlen)
+static int split_slots(int B, int Hkv, int max_seqlen, int resident)
 {
-    const long ns = target_splits(B, Hkv);
+    const long ns = target_splits(B, Hkv, resident);
     const int blocks = blocks_of(max_seqlen);
     return (int)(ns < blocks ? ns : blocks);
 }
@@ -289,7 +299,8 @@ size_t kvq_decode_workspace_bytes(const kvq_cache *c, int Hq, int max_seqlen)
 {
     if (check_decode_shape(c, Hq, max_seqlen) != KVQ_OK)
         return 0;
-    return decode_layout(c->B, c->Hkv, Hq, c->d, split_slots(c->B, c->Hkv, max_seqlen)).total;
+    const int res = decode_resident_ctas(c->d, Hq / c->Hkv, c->qp.bits_k, c->qp.bits_v);
+    return decode_layout(c->B, c->Hkv, Hq, c->d, split_slots(c->B, c->Hkv, max_seqlen, res)).total;
 }
 
 // Shared by the plain and the windowed decode: argument checks beyond the cache shape,
@@ -310,8 +321,9 @@ static kvq_status decode_common(const void *q, kvq_dtype q_dtype, int Hq, const 
         (out_dtype != KVQ_F32 && out_dtype != KVQ_BF16))
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "q_dtype/out_dtype must be KVQ_F32 or KVQ_BF16");
     int split_tokens = 0;
-    const int ns = choose_splits(c->B, c->Hkv, qmax, &split_tokens);
-    const int nslots = split_slots(c->B, c->Hkv, qmax);     // >= ns
+    const int res = decode_resident_ctas(c->d, Hq / c->Hkv, c->qp.bits_k, c->qp.bits_v);
+    const int ns = choose_splits(c->B, c->Hkv, qmax, &split_tokens, res);
+    const int nslots = split_slots(c->B, c->Hkv, qmax, res);     // >= ns
     const DecodeWorkspace w = decode_layout(c->B, c->Hkv, Hq, c->d, nslots);
     if (!workspace || !aligned(workspace, 256))
         KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
@@ -482,6 +494,188 @@ kvq_status kvq_decode_attention_window(const void *q, kvq_dtype q_dtype, int Hq,
                          workspace, ws_bytes, dev_err, stream, win);
 }
 
+// ------------------------------------------------------------------ vector-quantized cache
+
+static kvq_status check_vq_cache(const kvq_vq_cache *c)
+{
+    if (!c)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (c->B <= 0 || c->Hkv <= 0 || c->T_cap <= 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "cache B=%d Hkv=%d T_cap=%d must be positive", c->B, c->Hkv,
+                 c->T_cap);
+    if (c->T_cap % kCapAlign)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "T_cap=%d must be a multiple of %d", c->T_cap, kCapAlign);
+    if (c->d != 64 && c->d != 128)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "d=%d: only 64 and 128 are implemented", c->d);
+    if (!c->k_idx || !c->k_gain || !c->v_idx || !c->v_gain)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "a cache plane pointer is NULL");
+    if (!aligned(c->k_idx, 16) || !aligned(c->k_gain, 16) || !aligned(c->v_idx, 16) ||
+        !aligned(c->v_gain, 16))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "cache planes must be 16-byte aligned");
+    return KVQ_OK;
+}
+
+static kvq_status check_codebooks(const void *cb_k, const void *cb_v)
+{
+    if (!cb_k || !cb_v)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "codebooks must not be NULL");
+    if (!aligned(cb_k, 16) || !aligned(cb_v, 16))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "codebooks must be 16-byte aligned");
+    return KVQ_OK;
+}
+
+size_t kvq_vq_plane_bytes(const kvq_vq_cache *c, int which)
+{
+    if (!c || c->B <= 0 || c->Hkv <= 0 || c->T_cap <= 0 || c->d <= 0 || c->d % KVQ_VQ_DIM)
+        return 0;
+    const size_t tok = (size_t)c->B * c->Hkv * c->T_cap;
+    switch (which) {
+    case 0:
+    case 2: return tok * (c->d / KVQ_VQ_DIM);
+    case 1:
+    case 3: return tok * 2;
+    }
+    return 0;
+}
+
+kvq_status kvq_vq_append(const void *k, const void *v, kvq_dtype in_dtype, const float *T_k,
+                         const float *T_v, const void *cb_k, const void *cb_v,
+                         kvq_vq_cache *cache, const int32_t *pos, int n, int32_t *dev_err,
+                         kvq_stream_t stream)
+{
+    g_last_error[0] = 0;
+    kvq_status s = check_vq_cache(cache);
+    if (s != KVQ_OK)
+        return s;
+    s = check_codebooks(cb_k, cb_v);
+    if (s != KVQ_OK)
+        return s;
+    if (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "in_dtype=%d is not KVQ_F32 or KVQ_BF16", (int)in_dtype);
+    if (n < 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "n=%d is negative", n);
+    if (n > cache->T_cap)
+        KVQ_FAIL(KVQ_ERR_CAPACITY, "n=%d exceeds T_cap=%d", n, cache->T_cap);
+    if (n == 0)
+        return KVQ_OK;
+    if (!k || !v || !pos)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "k, v and pos must not be NULL");
+    if ((T_k && !aligned(T_k, 16)) || (T_v && !aligned(T_v, 16)))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "transforms must be 16-byte aligned");
+    cudaError_t e = launch_vq_append(k, v, in_dtype == KVQ_BF16, T_k, T_v, cb_k, cb_v, cache->B,
+                                     n, cache, pos, dev_err, (cudaStream_t)stream);
+    if (e != cudaSuccess)
+        KVQ_FAIL(KVQ_ERR_CUDA, "vq append launch: %s", cudaGetErrorString(e));
+    return KVQ_OK;
+}
+
+// The VQ decode's workspace: the scalar decode's sections (query prologue outputs, split
+// partials, tickets) plus q~ itself (float32 [B][Hq][d]) at the end.
+static kvq_status vq_shape(const kvq_vq_cache *c, int Hq, int max_seqlen)
+{
+    kvq_status s = check_vq_cache(c);
+    if (s != KVQ_OK)
+        return s;
+    if (Hq <= 0 || Hq % c->Hkv)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d", Hq, c->Hkv);
+    const int G = Hq / c->Hkv;
+    if (G != 4 && G != 8)
+        KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "query heads per KV head G=%d: 4 and 8 are implemented", G);
+    if (max_seqlen < 0)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "max_seqlen=%d is negative", max_seqlen);
+    if (max_seqlen > c->T_cap)
+        KVQ_FAIL(KVQ_ERR_CAPACITY, "max_seqlen=%d exceeds T_cap=%d", max_seqlen, c->T_cap);
+    return KVQ_OK;
+}
+
+static size_t vq_workspace(const kvq_vq_cache *c, int Hq, int max_seqlen, size_t *qt_off)
+{
+    const DecodeWorkspace w =
+        decode_layout(c->B, c->Hkv, Hq, c->d,
+                      split_slots(c->B, c->Hkv, max_seqlen, vq_resident_ctas(c->d, Hq / c->Hkv)));
+    *qt_off = w.total;
+    return w.total + up256((size_t)c->B * Hq * c->d * 4);
+}
+
+size_t kvq_vq_decode_workspace_bytes(const kvq_vq_cache *c, int Hq, int max_seqlen)
+{
+    if (vq_shape(c, Hq, max_seqlen) != KVQ_OK)
+        return 0;
+    size_t qt_off;
+    return vq_workspace(c, Hq, max_seqlen, &qt_off);
+}
+
+kvq_status kvq_vq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, const float *Tk_invT,
+                                   const void *cb_k, const void *cb_v, const kvq_vq_cache *c,
+                                   const int32_t *seqlens, int max_seqlen, void *out,
+                                   kvq_dtype out_dtype, void *workspace, size_t ws_bytes,
+                                   int32_t *dev_err, kvq_stream_t stream)
+{
+    g_last_error[0] = 0;
+    kvq_status s = vq_shape(c, Hq, max_seqlen);
+    if (s != KVQ_OK)
+        return s;
+    s = check_codebooks(cb_k, cb_v);
+    if (s != KVQ_OK)
+        return s;
+    if (!q || !seqlens || !out)
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "q, seqlens and out must not be NULL");
+    if ((q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) ||
+        (out_dtype != KVQ_F32 && out_dtype != KVQ_BF16))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG, "q_dtype/out_dtype must be KVQ_F32 or KVQ_BF16");
+    size_t qt_off;
+    const size_t need = vq_workspace(c, Hq, max_seqlen, &qt_off);
+    if (!workspace || !aligned(workspace, 256))
+        KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
+    if (ws_bytes < need)
+        KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
+    int split_tokens = 0;
+    const int res = vq_resident_ctas(c->d, Hq / c->Hkv);
+    const int ns = choose_splits(c->B, c->Hkv, max_seqlen, &split_tokens, res);
+    const int nslots = split_slots(c->B, c->Hkv, max_seqlen, res);
+    const DecodeWorkspace w = decode_layout(c->B, c->Hkv, Hq, c->d, nslots);
+    unsigned char *ws = (unsigned char *)workspace;
+    VqLaunch V;
+    DecodeLaunch &L = V.L;
+    memset(&L.p, 0, sizeof(L.p));
+    L.p.seqlens = seqlens;
+    L.p.B = c->B;
+    L.p.Hkv = c->Hkv;
+    L.p.Hq = Hq;
+    L.p.T_cap = c->T_cap;
+    L.p.max_seqlen = max_seqlen;
+    L.p.nsplit = ns;
+    L.p.split_tokens = split_tokens;
+    L.p.qfrag = (const uint32_t *)(ws + w.qfrag);
+    L.p.qscale = (const float *)(ws + w.qscale);
+    L.p.qw = (const float *)(ws + w.qw);
+    L.p.part = (float *)(ws + w.part);
+    L.p.ticket = (int *)(ws + w.ticket);
+    L.p.out = out;
+    L.p.out_bf16 = out_dtype == KVQ_BF16;
+    L.p.dev_err = dev_err;
+    L.p.part_slots = nslots + 1;
+    L.win = nullptr;
+    L.q = q;
+    L.q_bf16 = q_dtype == KVQ_BF16;
+    L.M = Tk_invT;
+    L.d = c->d;
+    L.G = Hq / c->Hkv;
+    L.bits_k = 2;
+    L.bits_v = 2;
+    V.qt = (float *)(ws + qt_off);
+    V.k_idx = (const uint8_t *)c->k_idx;
+    V.v_idx = (const uint8_t *)c->v_idx;
+    V.k_gain = (const uint16_t *)c->k_gain;
+    V.v_gain = (const uint16_t *)c->v_gain;
+    V.cb_k = (const uint16_t *)cb_k;
+    V.cb_v = (const uint16_t *)cb_v;
+    cudaError_t e = launch_vq_decode(V, (cudaStream_t)stream);
+    if (e != cudaSuccess)
+        KVQ_FAIL(KVQ_ERR_CUDA, "vq decode launch: %s", cudaGetErrorString(e));
+    return KVQ_OK;
+}
+
 size_t kvq_bf16_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seqlen)
 {
     if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv || (d != 64 && d != 128) || max_seqlen < 0)
@@ -490,7 +684,7 @@ size_t kvq_bf16_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_se
     if (G != 4 && G != 8)
         return 0;
     int split_tokens = 0;
-    const int ns = choose_splits(B, Hkv, max_seqlen, &split_tokens);
+    const int ns = choose_splits(B, Hkv, max_seqlen, &split_tokens, kDecodeMinBlocks);
     return up256((size_t)B * Hkv * ns * G * (d + 2) * 4) + up256((size_t)B * Hkv * 4);
 }
 
@@ -522,7 +716,7 @@ kvq_status kvq_bf16_decode(const void *q, int Hq, const void *k, const void *v, 
     if (ws_bytes < need)
         KVQ_FAIL(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
     int split_tokens = 0;
-    const int ns = choose_splits(B, Hkv, max_seqlen, &split_tokens);
+    const int ns = choose_splits(B, Hkv, max_seqlen, &split_tokens, kDecodeMinBlocks);
     cudaError_t e = launch_bf16_decode(q, Hq, k, v, B, Hkv, T_cap, d, seqlens, max_seqlen, out,
                                        workspace, ns, split_tokens, dev_err, (cudaStream_t)stream);
     if (e != cudaSuccess)

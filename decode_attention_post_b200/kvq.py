@@ -45,6 +45,11 @@ class _Window(C.Structure):
                 ("v_sink", _P), ("k_recent", _P), ("v_recent", _P), ("T_v", _P)]
 
 
+class _VQCache(C.Structure):
+    _fields_ = [("B", _I), ("Hkv", _I), ("T_cap", _I), ("d", _I), ("k_idx", _P),
+                ("k_gain", _P), ("v_idx", _P), ("v_gain", _P)]
+
+
 class KvqError(RuntimeError):
     def __init__(self, status: int, func: str, detail: str):
         self.status = status
@@ -85,6 +90,15 @@ def load():
     L.kvq_window_append.argtypes = [_P, _P, _I, _P, _P, C.POINTER(_QParams), C.POINTER(_Cache),
                                     C.POINTER(_Window), _P, _I, _P, _P]
     L.kvq_window_append.restype = _I
+    L.kvq_vq_plane_bytes.restype = _S
+    L.kvq_vq_plane_bytes.argtypes = [C.POINTER(_VQCache), _I]
+    L.kvq_vq_append.restype = _I
+    L.kvq_vq_append.argtypes = [_P, _P, _I, _P, _P, _P, _P, C.POINTER(_VQCache), _P, _I, _P, _P]
+    L.kvq_vq_decode_workspace_bytes.restype = _S
+    L.kvq_vq_decode_workspace_bytes.argtypes = [C.POINTER(_VQCache), _I, _I]
+    L.kvq_vq_decode_attention.restype = _I
+    L.kvq_vq_decode_attention.argtypes = [_P, _I, _I, _P, _P, _P, C.POINTER(_VQCache), _P, _I,
+                                          _P, _I, _P, _S, _P, _P]
     L.kvq_decode_attention_noalloc.argtypes = [_P, _I, _I, _P, C.POINTER(_Cache), _P, _I, _P,
                                                _I, _P, _P]
     L.kvq_bf16_decode_workspace_bytes.restype = _S
@@ -355,3 +369,75 @@ def bf16_decode(q, k, v, seqlens, max_seqlen: int, out, workspace, dev_err=None,
     _check(L.kvq_bf16_decode(_ptr(q), int(Hq), _ptr(k), _ptr(v), int(B), int(Hkv), int(T_cap),
                              int(d), _ptr(seqlens), int(max_seqlen), _ptr(out), _ptr(workspace),
                              workspace.numel(), _ptr(dev_err), _stream(stream)), "kvq_bf16_decode")
+
+
+# ------------------------------------------------------------------ vector-quantized cache
+
+class VQCache:
+    """kvq_vq_cache: index planes [B][Hkv][T_cap][d/4] uint8 and gain planes
+    [B][Hkv][T_cap] float16 (stored as uint8 tensors), caller-owned device memory."""
+
+    def __init__(self, B, Hkv, T_cap, d, planes):
+        self.B, self.Hkv, self.T_cap, self.d = B, Hkv, T_cap, d
+        self.k_idx, self.k_gain, self.v_idx, self.v_gain = planes
+        for name, t in zip(("k_idx", "k_gain", "v_idx", "v_gain"), planes):
+            _cuda(name, t, torch.uint8)
+        self._desc = _VQCache(B, Hkv, T_cap, d, _ptr(self.k_idx), _ptr(self.k_gain),
+                              _ptr(self.v_idx), _ptr(self.v_gain))
+
+    @classmethod
+    def allocate(cls, B, Hkv, T_cap, d, device="cuda", zero=True):
+        desc = _VQCache(B, Hkv, T_cap, d, None, None, None, None)
+        sizes = [int(load().kvq_vq_plane_bytes(C.byref(desc), w)) for w in range(4)]
+        if min(sizes) <= 0:
+            raise ValueError("invalid VQ cache shape")
+        make = torch.zeros if zero else torch.empty
+        return cls(B, Hkv, T_cap, d, [make(n, dtype=torch.uint8, device=device) for n in sizes])
+
+    @property
+    def desc(self):
+        return self._desc
+
+
+def vq_append(k, v, T_k, T_v, cb_k, cb_v, cache: VQCache, pos, n=None, dev_err=None,
+              stream=None):
+    """kvq_vq_append: k, v [B][n][Hkv][d] float32/bfloat16; T_k, T_v [Hkv][d][d] float32 or
+    None; codebooks cb_k, cb_v [Hkv][256][4] float16; pos int32 [B]."""
+    L = load()
+    _cuda("k", k)
+    _cuda("v", v, k.dtype)
+    _cuda("T_k", T_k, torch.float32)
+    _cuda("T_v", T_v, torch.float32)
+    _cuda("cb_k", cb_k, torch.float16)
+    _cuda("cb_v", cb_v, torch.float16)
+    _cuda("pos", pos, torch.int32)
+    _cuda("dev_err", dev_err, torch.int32)
+    if n is None:
+        n = k.shape[1]
+    _check(L.kvq_vq_append(_ptr(k), _ptr(v), _dt(k), _ptr(T_k), _ptr(T_v), _ptr(cb_k),
+                           _ptr(cb_v), C.byref(cache.desc), _ptr(pos), int(n), _ptr(dev_err),
+                           _stream(stream)), "kvq_vq_append")
+
+
+def vq_decode_workspace_bytes(cache: VQCache, Hq: int, max_seqlen: int) -> int:
+    return int(load().kvq_vq_decode_workspace_bytes(C.byref(cache.desc), int(Hq),
+                                                    int(max_seqlen)))
+
+
+def vq_decode_attention(q, Tk_invT, cb_k, cb_v, cache: VQCache, seqlens, max_seqlen: int, out,
+                        workspace, dev_err=None, stream=None):
+    """kvq_vq_decode_attention: q [B][Hq][d] float32/bfloat16, out [B][Hq][d]."""
+    L = load()
+    _cuda("q", q)
+    _cuda("Tk_invT", Tk_invT, torch.float32)
+    _cuda("cb_k", cb_k, torch.float16)
+    _cuda("cb_v", cb_v, torch.float16)
+    _cuda("seqlens", seqlens, torch.int32)
+    _cuda("out", out)
+    _cuda("workspace", workspace, torch.uint8)
+    _cuda("dev_err", dev_err, torch.int32)
+    _check(L.kvq_vq_decode_attention(_ptr(q), _dt(q), int(q.shape[1]), _ptr(Tk_invT),
+                                     _ptr(cb_k), _ptr(cb_v), C.byref(cache.desc), _ptr(seqlens),
+                                     int(max_seqlen), _ptr(out), _dt(out), _ptr(workspace),
+                                     workspace.numel(), _ptr(dev_err), _stream(stream)),
+           "kvq_vq_decode_attention")

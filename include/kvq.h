@@ -285,6 +285,72 @@ KVQ_API kvq_status kvq_window_append(const void *k_new, const void *v_new, kvq_d
                                      kvq_stream_t stream);
 
 /*
+ * Vector-quantized cache ("Spend Bits Where Queries Look", NOVA-KV project page: keys and
+ * values transformed and encoded once on the write path into a fixed-width cache; the
+ * read path is a codebook lookup plus one multiply; equal-size codebooks keep every token
+ * the same width). This library's reading (the page fixes neither the sub-vector size nor
+ * the codebook layout): the d transformed coefficients of a token form d/4 groups of 4
+ * consecutive coefficients, each coded by an 8-bit index into a codebook of 256 float16
+ * codewords of 4 coefficients (one codebook per KV head for keys, one for values, shared
+ * by the groups), and the token carries a float16 gain g, so x^_group = g * C[idx].
+ * 2 bits per coefficient plus 16 bits per token (2.125 bits per element at d = 128).
+ *  k_idx, v_idx   [B][Hkv][T_cap][d/4] uint8
+ *  k_gain, v_gain [B][Hkv][T_cap] float16
+ *  codebooks      cb_k, cb_v: [Hkv][256][4] float16 (device), caller-owned like the transforms
+ * T_cap a multiple of 64; d 64 or 128; planes 16-byte aligned.
+ */
+#define KVQ_VQ_DIM  4
+#define KVQ_VQ_SIZE 256
+typedef struct {
+    int B;
+    int Hkv;
+    int T_cap;
+    int d;
+    void *k_idx;
+    void *k_gain;
+    void *v_idx;
+    void *v_gain;
+} kvq_vq_cache;
+
+/* Size of plane `which` (0 k_idx, 1 k_gain, 2 v_idx, 3 v_gain); 0 if invalid. */
+KVQ_API size_t kvq_vq_plane_bytes(const kvq_vq_cache *cache, int which);
+
+/*
+ * VQ write path: x~ = T x per KV head (float32), then per token the gain
+ * g = f16(f32(sqrt(sum_j x~_j^2 / d))) (sum in float64) and per group of 4 the codeword
+ * nearest to the group after scaling by g, in float32 with a fixed operation order (an
+ * integer decision, reproduced exactly by the reference): e_m = f32(x~_m - f32(g c_m)),
+ * dist = f32(e_0 e_0), dist = fmaf(e_m, e_m, dist) for m = 1..3; the smallest dist wins,
+ * ties to the lowest index; g == 0 codes index 0. k, v: [B][n][Hkv][d] float32 or
+ * bfloat16; T_k, T_v as kvq_quantize_append (NULL = identity); pos: device int32 [B].
+ * Out-of-range sequences are skipped and flagged as in kvq_quantize_append.
+ */
+KVQ_API kvq_status kvq_vq_append(const void *k, const void *v, kvq_dtype in_dtype,
+                                 const float *T_k, const float *T_v, const void *cb_k,
+                                 const void *cb_v, kvq_vq_cache *cache, const int32_t *pos,
+                                 int n, int32_t *dev_err, kvq_stream_t stream);
+
+/* Workspace bytes kvq_vq_decode_attention needs (0 if the arguments are invalid); never
+ * decreases as max_seqlen grows. */
+KVQ_API size_t kvq_vq_decode_workspace_bytes(const kvq_vq_cache *cache, int Hq, int max_seqlen);
+
+/*
+ * VQ read path: softmax_t(q~ . k^_t / sqrt(d)) v^_t with q~ = Tk_invT q and
+ * k^_t = g^K_t C_K[idx], v^_t = g^V_t C_V[idx] (codebook lookup plus one multiply), in the
+ * value-transform domain. Codewords are expanded into float16 tiles in shared memory and
+ * both contractions run on float16 tensor cores (q~ and the softmax weights as float16
+ * hi/lo pairs), float32 online softmax, split-K with the same merge as
+ * kvq_decode_attention. Arguments and errors as kvq_decode_attention; G in {4, 8}.
+ */
+KVQ_API kvq_status kvq_vq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq,
+                                           const float *Tk_invT, const void *cb_k,
+                                           const void *cb_v, const kvq_vq_cache *cache,
+                                           const int32_t *seqlens, int max_seqlen, void *out,
+                                           kvq_dtype out_dtype, void *workspace,
+                                           size_t ws_bytes, int32_t *dev_err,
+                                           kvq_stream_t stream);
+
+/*
  * Allocation-free decode (no counterpart in the paper; an addition for callers that
  * cannot allocate device memory). Same arguments and result as kvq_decode_attention
  * minus the workspace: an inference engine that has reserved nearly all device memory

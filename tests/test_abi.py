@@ -280,3 +280,50 @@ def test_binding_requires_cuda_tensors():
     qp = kvq.QParams()
     with pytest.raises(TypeError):
         kvq.KVCache(1, 1, 64, 128, qp, [torch.zeros(8, dtype=torch.uint8)] * 4)
+
+
+def _vq_desc(B=2, Hkv=2, T_cap=128, d=128, ptr=0x1000):
+    return K._VQCache(B, Hkv, T_cap, d, ptr, ptr, ptr, ptr)
+
+
+def test_vq_plane_bytes_follow_layout():
+    L = kvq.load()
+    desc = _vq_desc(B=3, Hkv=2, T_cap=192, d=128)
+    tok = 3 * 2 * 192
+    assert [L.kvq_vq_plane_bytes(C.byref(desc), w) for w in range(4)] == \
+        [tok * 32, tok * 2, tok * 32, tok * 2]
+    assert L.kvq_vq_plane_bytes(C.byref(desc), 9) == 0
+
+
+def test_vq_argument_errors():
+    L = kvq.load()
+    desc = _vq_desc()
+
+    def append(**kw):
+        a = dict(k=0x5000, v=0x5000, dt=1, ck=0x7000, cv=0x7000, pos=0x6000, n=4)
+        a.update(kw)
+        return L.kvq_vq_append(a["k"], a["v"], a["dt"], None, None, a["ck"], a["cv"],
+                               C.byref(desc), a["pos"], a["n"], None, None)
+    assert append(ck=0) == 1
+    assert append(ck=0x7008) == 1                       # misaligned codebook
+    assert append(dt=3) == 1
+    assert append(n=-1) == 1
+    assert append(n=1000) == 3
+    assert append(k=0) == 1
+    assert append(n=0, k=0) == 0
+
+    def decode(ws_bytes=16, **kw):
+        a = dict(q=0x5000, Hq=8, ck=0x7000, cv=0x7000, seq=0x6000, mx=64, out=0x8000)
+        a.update(kw)
+        return L.kvq_vq_decode_attention(a["q"], 1, a["Hq"], None, a["ck"], a["cv"],
+                                         C.byref(desc), a["seq"], a["mx"], a["out"], 1, 0x9000,
+                                         ws_bytes, None, None)
+    assert decode(Hq=6) == 2                            # G = 3
+    assert decode(mx=200) == 3
+    assert decode(cv=0) == 1
+    assert decode(out=0) == 1
+    assert decode() == 4                                # workspace too small
+    assert 0 < L.kvq_vq_decode_workspace_bytes(C.byref(desc), 8, 64) <= \
+        L.kvq_vq_decode_workspace_bytes(C.byref(desc), 8, 128)
+    bad = _vq_desc(d=96)
+    assert L.kvq_vq_decode_workspace_bytes(C.byref(bad), 8, 64) == 0

@@ -183,12 +183,13 @@ def test_window_append_serving_loop(ci, prefill, steps, S_sink, S_keep, S_flush)
     assert st.err.item() == 0
     assert_close(out.cpu().numpy(), want, where=f"window append {S_sink}/{S_keep}/{S_flush}")
     # ---- and end to end over the GPU's own state: the same attention up to the code
-    #      differences above (relative L2 only)
+    #      differences checked above (a sanity bound: with 2-bit codes one flipped code
+    #      moves its value by a whole step, so this is looser than the parity bar)
     kvq.decode_attention_window(t_(q), st.Tit, st.cache, S_sink, S_keep, S_flush, st.ks, st.vs,
                                 st.kr, st.vr, st.Tv, t_(st.len), Lmax, out, ws, dev_err=st.err)
     torch.cuda.synchronize()
     got = out.cpu().numpy()
-    assert np.linalg.norm(got - want) <= 1e-3 * np.linalg.norm(want)
+    assert np.linalg.norm(got - want) <= 1e-2 * np.linalg.norm(want)
 
 
 def test_window_append_out_of_range_is_flagged_and_skipped():
