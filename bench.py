@@ -402,6 +402,7 @@ def run_gpu(args):
         line["bf16_comparator"] = bf16_comparator(w, cfg, K, stream, dec_ms)
         line["paged_decode"] = paged_decode(w, cfg, K, stream, dec_ms, dec_bytes)
         line["window_decode"] = window_decode(w, cfg, stream, dec_ms, peak)
+        line["vq_decode"] = vq_decode(w, cfg, stream, dec_ms, peak)
         del w
         torch.cuda.empty_cache()
         line["chunk_append"] = chunk_append(device, stream)
@@ -621,6 +622,50 @@ def window_decode(w, cfg, stream, dec_ms, peak, S_sink=64, S_keep=256, S_flush=1
     return res
 
 
+def vq_decode(w, cfg, stream, dec_ms, peak):
+    """The same sequences in the vector-quantized cache (NOVA-KV: codebook lookup plus one
+    multiply; synthetic codebooks): encoded by kvq_vq_append, then the VQ decode timed, and
+    a decode-time step (VQ append of the newest token + decode)."""
+    import torch
+    import decode_attention_post_b200 as kvq
+    cb_k, cb_v = synth.codebooks(cfg)
+    f16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.float16)).to(w.dev)
+    ck, cv = f16(cb_k), f16(cb_v)
+    cache = kvq.VQCache.allocate(cfg.B, cfg.Hkv, cfg.T_cap, cfg.d, device=w.dev, zero=False)
+    for b in range(cfg.B):
+        L = int(w.seqlens[b])
+        kb = w.kb[b, :, :L].transpose(0, 1).contiguous()[None]
+        vb = w.vb[b, :, :L].transpose(0, 1).contiguous()[None]
+        one = kvq.VQCache(1, cfg.Hkv, cfg.T_cap, cfg.d,
+                          [p[b * (p.numel() // cfg.B):(b + 1) * (p.numel() // cfg.B)]
+                           for p in (cache.k_idx, cache.k_gain, cache.v_idx, cache.v_gain)])
+        kvq.vq_append(kb, vb, w.Tk, w.Tv, ck, cv, one, torch.zeros(1, dtype=torch.int32,
+                                                                    device=w.dev))
+    torch.cuda.synchronize()
+    out = torch.empty_like(w.out)
+    ws = torch.empty(kvq.vq_decode_workspace_bytes(cache, cfg.Hq, cfg.T_cap), dtype=torch.uint8,
+                     device=w.dev)
+    dec = lambda: kvq.vq_decode_attention(w.q, w.Tit, ck, cv, cache, w.seq_d, cfg.T_cap, out, ws,
+                                          dev_err=w.err)
+    ms = statistics.mean(time_events(dec, 200, stream))
+    step = lambda: (kvq.vq_append(w.knew, w.vnew, w.Tk, w.Tv, ck, cv, cache, w.pos, n=1,
+                                  dev_err=w.err), dec())
+    step_ms = statistics.mean(time_events(step, 100, stream))
+    per_tok = cfg.Hkv * 2 * (cfg.d // 4 + 2)
+    nbytes = int(np.sum(w.seqlens)) * per_tok + 2 * cfg.B * cfg.Hq * cfg.d * 2 + \
+        2 * cfg.Hkv * 256 * 4 * 2
+    torch.cuda.synchronize()
+    res = {"bits_per_element": round(8 * (cfg.d // 4 + 2) / cfg.d, 4),
+           "bytes_per_launch": nbytes, "ms_per_launch": round(ms, 5),
+           "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+           "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4),
+           "time_vs_scalar_decode": round(ms / dec_ms, 4),
+           "step_ms_append_plus_decode": round(step_ms, 5), "dev_err": int(w.err.item())}
+    del cache, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def chunk_append(device, stream):
     """32768-token chunk append of the GPT-OSS-20B-like shape (batch 8, 8 KV heads, d 64)."""
     import torch
@@ -780,6 +825,13 @@ def profile_case(name):
                                                [int(x) for x in sweep.split(",")])}
         else:
             res = decode_config_line(idx, device, stream, peak)
+    elif name in ("vq_config1", "window_config1"):
+        # a Workload at the batch-16 / 16K shape (bf16 tokens kept), then the VQ or the
+        # windowed decode line on it
+        cfg = synth.CONFIGS[1]
+        w = Workload(cfg, 0, device, with_bf16=True)
+        dec_ms = statistics.mean(time_events(w.decode, 50, stream))
+        res = (vq_decode if name == "vq_config1" else window_decode)(w, cfg, stream, dec_ms, peak)
     elif name == "bf16_config1":
         # the uncompressed comparator at the batch-16 / 16K shape (1.07 GB of bf16 K and V);
         # its time does not depend on the values, so they are drawn on the device
@@ -815,7 +867,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--profile-case", default=None,
                     help="run one kernel's workload alone (chunk_append, append_config0, "
-                         "decode_config1/3/4, bf16_config1) for an ncu capture")
+                         "decode_config1/2/3/4, bf16_config1, vq_config1, window_config1) "
+                         "for an ncu capture")
     args = ap.parse_args()
     if args.profile_case:
         profile_case(args.profile_case)

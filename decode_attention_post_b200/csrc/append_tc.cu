@@ -4,15 +4,16 @@
 //
 // CTA = (KV head, one of {K, V}, slice of the 128-token tiles of the flattened
 // (sequence, new token) list), 6 warps with fixed roles:
-//   warp 4, one lane   TMA: each 128-token input tile [128 x d] bf16 lands in a 3-stage
+//   warp 8, one lane   TMA: each 128-token input tile [128 x d] bf16 lands in a 3-stage
 //                      shared-memory ring in the 128-byte-swizzled K-major layout (3-D
 //                      tensor map over [tokens][Hkv][d], no multicast);
-//   warp 5, one lane   tcgen05.mma: X~[128 x d] = X . T_hi^T + X . T_lo^T into one float32
+//   warp 9, one lane   tcgen05.mma: X~[128 x d] = X . T_hi^T + X . T_lo^T into one float32
 //                      TMEM accumulator (T split into two bfloat16 pieces, 16 significant
 //                      bits; X is bfloat16, hence exact), M = 128, N = d, K = 16 per
 //                      instruction; two accumulator buffers so that the next tile's MMAs
 //                      overlap this tile's epilogue;
-//   warps 0-3          epilogue: thread r owns token r of the tile; tcgen05.ld brings its
+//   warps 0-7          epilogue, two warpgroups taking alternate tiles (one accumulator
+//                      buffer each): thread r owns token r of the tile; tcgen05.ld brings its
 //                      transformed values into registers 32 columns at a time, in two
 //                      passes: per group the clip range (order statistics, or the RMS for
 //                      the QuEST INT quantizer) and the float16 scale and zero-point, then
@@ -37,7 +38,8 @@ namespace kvq {
 namespace {
 
 constexpr int kTcTile = 128;                       // tokens per tile (MMA M)
-constexpr int kTcEpiWarps = 4;
+constexpr int kTcEpiGroups = 2;                    // epilogue warpgroups, one per accumulator
+constexpr int kTcEpiWarps = 4 * kTcEpiGroups;
 constexpr int kTcThreads = (kTcEpiWarps + 2) * 32; // epilogue warps + TMA warp + MMA warp
 constexpr int kTcStages = 3;
 constexpr int kTcKBlock = 64;                      // bf16 per 128-byte swizzled row
@@ -55,7 +57,7 @@ struct TcCfg {
     static constexpr int SMEM = OFF_BAR + 128 + 1024;         // barriers + alignment slack
     static constexpr int TMEM_COLS = 2 * D;                   // two accumulator buffers
     // CTAs per SM: shared memory allows it, TMEM (512 columns) and registers must too
-    static constexpr int PER_SM = D == 64 ? 3 : 1;
+    static constexpr int PER_SM = D == 64 ? 2 : 1;
     static_assert(PER_SM * TMEM_COLS <= 512, "TMEM oversubscribed");
     static_assert(PER_SM * (SMEM + 1024) <= 228 * 1024, "shared memory oversubscribed");
 };
@@ -76,28 +78,6 @@ struct TcParams {
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
-// 32 TMEM columns of this thread's lane as floats (load and wait in one statement, so
-// that nothing reads the registers before the load has completed).
-__device__ __forceinline__ void tmem_ld32_f(uint32_t taddr, float *x)
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        x[i] = __uint_as_float(r[i]);
 }
 
 // Codes of a group: c = clamp(rint(f32(f32(x - z) / s)), 0, qmax) for float16 (s, z).
@@ -154,137 +134,139 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     return r;
 }
 
-// The K row of one token (little-endian bit stream, dim j at bit bits*j) from its row in
-// TMEM, 32 columns at a time; stored as 16-byte pieces when row >= 0. exact = false: the
-// fast codes (sets `tie` near a rounding tie); exact = true: IEEE division. Warp-wide (the
-// TMEM loads), every lane calls it.
-template <int D, int GS, int NG>
-__device__ __forceinline__ void store_k_row(const TcParams &P, long long row, int bits,
-                                            uint32_t taddr, const float (&zf)[NG],
-                                            const float (&sf)[NG], const float (&rc)[NG],
-                                            const bool (&zero)[NG], float qmax, bool &tie,
-                                            bool exact)
+// 32 TMEM columns of this thread's lane into registers; the load completes at the next
+// tmem_wait (the hardware holds readers of the registers until then).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32])
 {
-    float x[32];
-    uint4 *dst = reinterpret_cast<uint4 *>(P.k_codes + row * (D * bits / 8));
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// Per-group quantities selected by a group index known only at run time, without a
+// local-memory array (NG <= 4 compile-time slots).
+template <int NG>
+__device__ __forceinline__ float pick(const float (&a)[NG], int gr)
+{
+    float v = a[0];
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-        const int gr = (32 * c) / GS;
-        tmem_ld32_f(taddr + 32 * c, x);
-        if (bits == 2) {
-            uint32_t w[2];
+    for (int i = 1; i < NG; ++i)
+        v = gr == i ? a[i] : v;
+    return v;
+}
+
+template <int NG>
+__device__ __forceinline__ bool pickb(const bool (&a)[NG], int gr)
+{
+    bool v = a[0];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                uint32_t acc = exact ? 0u : 0u - magic_sum(2, 16);
+    for (int i = 1; i < NG; ++i)
+        v = gr == i ? a[i] : v;
+    return v;
+}
+
+// Codes of 32 consecutive dims (column c0.. of the row) packed as BITS-bit fields of
+// 32-bit words: `words` words, field e of word q = dim c0 + (32/BITS) q + e. exact = false:
+// reciprocal codes (sets tie near a rounding tie); exact = true: IEEE division.
+template <int BITS, bool EXACT>
+__device__ __forceinline__ void pack32(const uint32_t (&x)[32], float zf, float sf, float rc,
+                                       bool zero, float qmax, bool &tie, uint32_t (&w)[BITS])
+{
+    constexpr bool exact = EXACT;
+    constexpr int PER = 32 / BITS;                  // codes per word
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float v = x[16 * q + e];
-                    acc += (exact ? code_exact(v, zf[gr], sf[gr], zero[gr], qmax)
-                                  : code_bits(v, zf[gr], rc[gr], qmax, tie)) << (2 * e);
-                }
-                w[q] = acc;
-            }
-            // two words per 32 columns: a 16-byte piece every other chunk
-            if (row >= 0) {
-                if (c % 2 == 0) {
-                    dst[c / 2].x = w[0];
-                    dst[c / 2].y = w[1];
-                } else {
-                    dst[c / 2].z = w[0];
-                    dst[c / 2].w = w[1];
-                }
-            }
-        } else {
-            uint32_t w[4];
+    for (int q = 0; q < BITS; ++q) {
+        uint32_t acc = exact ? 0u : 0u - magic_sum(BITS, PER);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t acc = exact ? 0u : 0u - magic_sum(4, 8);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float v = x[8 * q + e];
-                    acc += (exact ? code_exact(v, zf[gr], sf[gr], zero[gr], qmax)
-                                  : code_bits(v, zf[gr], rc[gr], qmax, tie)) << (4 * e);
-                }
-                w[q] = acc;
-            }
-            if (row >= 0)
-                dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int e = 0; e < PER; ++e) {
+            const float v = __uint_as_float(x[PER * q + e]);
+            acc += (exact ? code_exact(v, zf, sf, zero, qmax) : code_bits(v, zf, rc, qmax, tie))
+                   << (BITS * e);
         }
+        w[q] = acc;
     }
 }
 
-// The token's halves of its 16-token V tile: half (gq, rr) holds dims 8(E rr + s) + gq at
-// bits*s, E = 16/bits; a half gathers dims 8 apart, so the halves are built up over the
-// 32-column chunks and stored at the end (row >= 0). Same conventions as store_k_row.
-template <int D, int GS, int NG>
-__device__ __forceinline__ void store_v_token(const TcParams &P, long long row, int bits,
-                                              uint32_t taddr, const float (&zf)[NG],
-                                              const float (&sf)[NG], const float (&rc)[NG],
-                                              const bool (&zero)[NG], float qmax, bool &tie,
-                                              bool exact)
+// One token's codes from its TMEM row, 32 columns per iteration (the other warps of the
+// SM hide the load latency), stored as the K row (little-endian bit stream, dim j at
+// bit BITS*j) or as the token's halves of its 16-token V tile (half (gq, rr) holds dims
+// 8(E rr + s) + gq at BITS*s, E = 16/BITS). row < 0: codes not stored (the warp still
+// takes part in the TMEM loads). Returns whether a value was within the tie band.
+template <int D, int GS, int NG, int BITS, bool V, bool EXACT>
+__device__ __forceinline__ bool store_codes(const TcParams &P, long long row, uint32_t taddr,
+                                            const float (&zf)[NG], const float (&sf)[NG],
+                                            const float (&rc)[NG], const bool (&zero)[NG],
+                                            float qmax)
 {
-    float x[32];
-    if (bits == 2) {
-        constexpr int E = 8, W = D * 2 / 128;           // a half spans 64 dims
-        uint32_t hv[8][W];
-#pragma unroll
-        for (int gq = 0; gq < 8; ++gq)
-#pragma unroll
-            for (int rr = 0; rr < W; ++rr)
-                hv[gq][rr] = exact ? 0u : 0u - magic_sum(2, E);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            const int gr = (32 * c) / GS;
-            tmem_ld32_f(taddr + 32 * c, x);
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj) {
-                const int j = 32 * c + jj, gq = j % 8, n8 = j / 8, rr = n8 / E, s2 = n8 % E;
-                hv[gq][rr] += (exact ? code_exact(x[jj], zf[gr], sf[gr], zero[gr], qmax)
-                                     : code_bits(x[jj], zf[gr], rc[gr], qmax, tie)) << (2 * s2);
+    constexpr bool exact = EXACT;
+    constexpr int NCH = D / 32;
+    bool tie = false;
+    uint32_t cur[32];
+    tmem_ld32_async(taddr, cur);
+    tmem_ld_wait();
+    unsigned char *vbase = nullptr;
+    int tok = 0;
+    if (V && row >= 0) {
+        vbase = P.v_codes + (size_t)(row / kTileTokens) * (kTileTokens * D * BITS / 8);
+        tok = (int)(row % kTileTokens);
+    }
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c) {
+        if (c > 0) { tmem_ld32_async(taddr + 32 * c, cur); tmem_ld_wait(); }
+        const int gr = (32 * c) / GS;
+        const float z = pick(zf, gr), s = pick(sf, gr), r = pick(rc, gr);
+        const bool zr = pickb(zero, gr);
+        if (!V) {
+            uint32_t w[BITS];
+            pack32<BITS, EXACT>(cur, z, s, r, zr, qmax, tie, w);
+            if (row >= 0) {
+                uint32_t *dst = reinterpret_cast<uint32_t *>(P.k_codes + row * (D * BITS / 8)) + BITS * c;
+                if (BITS == 2)
+                    *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1 % BITS]);
+                else
+                    *reinterpret_cast<uint4 *>(dst) =
+                        make_uint4(w[0], w[1 % BITS], w[2 % BITS], w[3 % BITS]);
             }
-        }
-        if (row >= 0) {
-            unsigned char *tile_base =
-                P.v_codes + (size_t)(row / kTileTokens) * (kTileTokens * D * 2 / 8);
-            const int tok = (int)(row % kTileTokens);
+        } else {
+            // The chunk's dims are 32c + 8 n8 + gq (n8 < 4, gq < 8). The half (gq, rr) holds
+            // dims 8(E rr + s) + gq at bits BITS*s, E = 16/BITS: with 4-bit codes chunk c is
+            // all of the halves rr = c; with 2-bit codes chunk c is fields 4(c&1) .. +3 of
+            // the halves rr = c/2, i.e. their byte c&1 (each token owns whole bytes).
+            const int base = BITS == 2 ? 4 * (c & 1) : 0;
+            uint32_t hv[8];
 #pragma unroll
-            for (int gq = 0; gq < 8; ++gq)
+            for (int gq = 0; gq < 8; ++gq) {
+                uint32_t acc = exact ? 0u : 0u - (magic_sum(BITS, 4) << (BITS * base));
 #pragma unroll
-                for (int rr = 0; rr < W; ++rr)
-                    *reinterpret_cast<uint16_t *>(tile_base + v_half_offset(D, 2, tok, gq, rr)) =
-                        (uint16_t)hv[gq][rr];
-        }
-    } else {
-        constexpr int E = 4, W = D * 4 / 128;           // a half spans 32 dims
-        uint32_t hv[8][W];
-#pragma unroll
-        for (int gq = 0; gq < 8; ++gq)
-#pragma unroll
-            for (int rr = 0; rr < W; ++rr)
-                hv[gq][rr] = exact ? 0u : 0u - magic_sum(4, E);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            const int gr = (32 * c) / GS;
-            tmem_ld32_f(taddr + 32 * c, x);
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj) {
-                const int j = 32 * c + jj, gq = j % 8, n8 = j / 8, rr = n8 / E, s2 = n8 % E;
-                hv[gq][rr] += (exact ? code_exact(x[jj], zf[gr], sf[gr], zero[gr], qmax)
-                                     : code_bits(x[jj], zf[gr], rc[gr], qmax, tie)) << (4 * s2);
+                for (int n8 = 0; n8 < 4; ++n8) {
+                    const float v = __uint_as_float(cur[8 * n8 + gq]);
+                    acc += (exact ? code_exact(v, z, s, zr, qmax) : code_bits(v, z, r, qmax, tie))
+                           << (BITS * (base + n8));
+                }
+                hv[gq] = acc;
             }
-        }
-        if (row >= 0) {
-            unsigned char *tile_base =
-                P.v_codes + (size_t)(row / kTileTokens) * (kTileTokens * D * 4 / 8);
-            const int tok = (int)(row % kTileTokens);
+            if (row >= 0) {
 #pragma unroll
-            for (int gq = 0; gq < 8; ++gq)
-#pragma unroll
-                for (int rr = 0; rr < W; ++rr)
-                    *reinterpret_cast<uint16_t *>(tile_base + v_half_offset(D, 4, tok, gq, rr)) =
-                        (uint16_t)hv[gq][rr];
+                for (int gq = 0; gq < 8; ++gq) {
+                    if (BITS == 4)
+                        *reinterpret_cast<uint16_t *>(vbase + v_half_offset(D, 4, tok, gq, c)) =
+                            (uint16_t)hv[gq];
+                    else
+                        vbase[v_half_offset(D, 2, tok, gq, c >> 1) + (c & 1)] =
+                            (unsigned char)(hv[gq] >> (8 * (c & 1)));
+                }
+            }
         }
     }
+    return tie;
 }
 
 template <int D, int GS>
@@ -321,7 +303,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&accf[a], 1);
-            mbar_init(&acce[a], kTcEpiWarps * 32);
+            mbar_init(&acce[a], 128);                  // one epilogue warpgroup
         }
         *abort_flag = 0;
         mbar_fence_init();
@@ -410,21 +392,24 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Two passes over the token's row in TMEM, 32 columns at a time (registers stay
-        // low): the clip parameters of every group, then the codes. The accumulator buffer
-        // is released after the row is done, so a row near a rounding tie can be reloaded
-        // and recomputed with IEEE division.
-        const int r = warp * 32 + lane;                     // token row of the tile
+        // Warpgroup wg takes the tiles k = wg, wg + 2, ... (accumulator buffer wg); thread r
+        // of warp quarter q owns TMEM lane (token row) 32 q + r. Two passes over the row,
+        // 32 columns at a time: the clip parameters of every group, then the codes. The
+        // buffer is released after the row is done, so a row near a rounding tie can be
+        // reloaded and recoded with IEEE division.
+        const int wg = warp / 4, quarter = warp % 4;
+        const int r = quarter * 32 + lane;
         const float qmax = (float)((1u << bits) - 1u);
         const bool quest = P.clip == kQuestClip;
-        for (int k = 0; k < my_tiles; ++k) {
+        for (int k = wg; k < my_tiles; k += kTcEpiGroups) {
             const int a = k & 1;
             if (*abort_flag || !mbar_wait_bounded(&accf[a], (k >> 1) & 1)) {
                 *abort_flag = 1;
                 break;
             }
             tc_fence_after_sync();
-            const uint32_t taddr = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(a * D);
+            const uint32_t taddr =
+                tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * D);
             const long tile = blockIdx.x + (long)k * gridDim.x;
             const long u = tile * kTcTile + r;
             long long row = -1;
@@ -441,47 +426,45 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         flag(P.dev_err, KVQ_DEVERR_PAGE_RANGE);
                 }
             }
-            // every lane of the warp takes part in the TMEM loads (warp-wide instructions)
-            // ---- pass 1: clip parameters per group
+            // ---- pass 1: clip parameters per group (every lane takes part in the loads)
             float zf[NG], sf[NG], rc[NG];
             bool zero[NG];
+#pragma unroll
+            for (int gg = 0; gg < NG; ++gg) {
+                zf[gg] = sf[gg] = rc[gg] = 0.f;
+                zero[gg] = true;
+            }
             {
-                float x[32];
-                float lo = 0.f, hi = 0.f;
+                uint32_t cur[32];
+                float lo = INFINITY, hi = -INFINITY;
                 float m1 = INFINITY, m2 = INFINITY, M1 = -INFINITY, M2 = -INFINITY;
                 float sm9[9], lg9[9];
+#pragma unroll
+                for (int e = 0; e < 9; ++e) {
+                    sm9[e] = INFINITY;
+                    lg9[e] = -INFINITY;
+                }
                 double ss = 0.0;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
-                    const int gr = (32 * c) / GS;
-                    const bool first = (32 * c) % GS == 0, last = (32 * c + 32) % GS == 0;
-                    tmem_ld32_f(taddr + 32 * c, x);
-                    if (first) {
-                        lo = INFINITY;
-                        hi = -INFINITY;
-                        m1 = m2 = INFINITY;
-                        M1 = M2 = -INFINITY;
-                        ss = 0.0;
-#pragma unroll
-                        for (int e = 0; e < 9; ++e) {
-                            sm9[e] = INFINITY;
-                            lg9[e] = -INFINITY;
-                        }
-                    }
+                    tmem_ld32_async(taddr + 32 * c, cur);
+                    tmem_ld_wait();
                     if (quest) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            ss = fma((double)x[j], (double)x[j], ss);
+                        for (int j = 0; j < 32; ++j) {
+                            const double v = (double)__uint_as_float(cur[j]);
+                            ss = fma(v, v, ss);
+                        }
                     } else if (P.clip == 0) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 2) {
-                            lo = fmin3(lo, x[j], x[j + 1]);
-                            hi = fmax3(hi, x[j], x[j + 1]);
+                            lo = fmin3(lo, __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+                            hi = fmax3(hi, __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
                         }
                     } else if (P.clip == 1) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            const float v = x[j];
+                            const float v = __uint_as_float(cur[j]);
                             m2 = fminf(m2, fmaxf(m1, v));
                             m1 = fminf(m1, v);
                             M2 = fmaxf(M2, fminf(M1, v));
@@ -489,8 +472,9 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         }
                     } else {
                         // kappa <= 8: the 9 smallest and 9 largest by insertion
+#pragma unroll 4
                         for (int j = 0; j < 32; ++j) {
-                            float av = x[j], bv = x[j];
+                            float av = __uint_as_float(cur[j]), bv = av;
 #pragma unroll
                             for (int e = 0; e < 9; ++e) {
                                 const float s0 = fminf(sm9[e], av), s1 = fmaxf(sm9[e], av);
@@ -502,7 +486,8 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                             }
                         }
                     }
-                    if (last) {
+                    if ((32 * c + 32) % GS == 0) {          // the group ends with this chunk
+                        const int gr = (32 * c) / GS;
                         __half sh, zh;
                         bool finite;
                         if (quest) {
@@ -512,51 +497,78 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                             zh = __float2half_rn(__fmul_rn(-0.5f * qmax, __half2float(sh)));
                             finite = isfinite(s);
                         } else {
+                            float glo = lo, ghi = hi;
                             if (P.clip == 1) {
-                                lo = m2;
-                                hi = M2;
+                                glo = m2;
+                                ghi = M2;
                             } else if (P.clip > 1) {
-                                lo = sm9[0];
-                                hi = lg9[0];
+                                glo = sm9[0];
+                                ghi = lg9[0];
 #pragma unroll
                                 for (int e = 1; e < 9; ++e)
                                     if (e == P.clip) {
-                                        lo = sm9[e];
-                                        hi = lg9[e];
+                                        glo = sm9[e];
+                                        ghi = lg9[e];
                                     }
                             }
-                            const float range = __fsub_rn(hi, lo);
+                            const float range = __fsub_rn(ghi, glo);
                             const float s = __fdiv_rn(range, qmax);
                             sh = __float2half_rn(s);
-                            zh = __float2half_rn(lo);
+                            zh = __float2half_rn(glo);
                             finite = isfinite(range) && isfinite(s);
                         }
-                        sf[gr] = __half2float(sh);
-                        zf[gr] = __half2float(zh);
-                        zero[gr] = !finite || sf[gr] == 0.f;
-                        rc[gr] = zero[gr] ? 0.f : __frcp_rn(sf[gr]);
+                        const float sfv = __half2float(sh), zfv = __half2float(zh);
+                        const bool zr = !finite || sfv == 0.f;
+                        const float rcv = zr ? 0.f : __frcp_rn(sfv);
+#pragma unroll
+                        for (int gg = 0; gg < NG; ++gg)
+                            if (gg == gr) {
+                                sf[gg] = sfv;
+                                zf[gg] = zfv;
+                                zero[gg] = zr;
+                                rc[gg] = rcv;
+                            }
                         if (row >= 0) {
                             if (!finite)
                                 flag(P.dev_err, KVQ_DEVERR_NONFINITE);
                             (which ? P.v_sz : P.k_sz)[row * NG + gr] =
                                 (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
                         }
+                        // the next group starts fresh
+                        lo = INFINITY;
+                        hi = -INFINITY;
+                        m1 = m2 = INFINITY;
+                        M1 = M2 = -INFINITY;
+                        ss = 0.0;
+#pragma unroll
+                        for (int e = 0; e < 9; ++e) {
+                            sm9[e] = INFINITY;
+                            lg9[e] = -INFINITY;
+                        }
                     }
                 }
             }
             // ---- pass 2: codes; pass 3 (rows near a rounding tie only): the same by division
-            bool tie = false;
+            bool tie;
             if (!which)
-                store_k_row<D, GS, NG>(P, row, bits, taddr, zf, sf, rc, zero, qmax, tie, false);
+                tie = bits == 2 ? store_codes<D, GS, NG, 2, false, false>(P, row, taddr, zf, sf, rc, zero, qmax)
+                                : store_codes<D, GS, NG, 4, false, false>(P, row, taddr, zf, sf, rc, zero, qmax);
             else
-                store_v_token<D, GS, NG>(P, row, bits, taddr, zf, sf, rc, zero, qmax, tie, false);
+                tie = bits == 2 ? store_codes<D, GS, NG, 2, true, false>(P, row, taddr, zf, sf, rc, zero, qmax)
+                                : store_codes<D, GS, NG, 4, true, false>(P, row, taddr, zf, sf, rc, zero, qmax);
             if (__any_sync(0xffffffffu, tie)) {
-                if (!which)
-                    store_k_row<D, GS, NG>(P, tie ? row : -1, bits, taddr, zf, sf, rc, zero, qmax,
-                                           tie, true);
-                else
-                    store_v_token<D, GS, NG>(P, tie ? row : -1, bits, taddr, zf, sf, rc, zero, qmax,
-                                             tie, true);
+                const long long rw = tie ? row : -1;
+                if (!which) {
+                    if (bits == 2)
+                        store_codes<D, GS, NG, 2, false, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
+                    else
+                        store_codes<D, GS, NG, 4, false, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
+                } else {
+                    if (bits == 2)
+                        store_codes<D, GS, NG, 2, true, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
+                    else
+                        store_codes<D, GS, NG, 4, true, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
+                }
             }
             tc_fence_before_sync();
             mbar_arrive(&acce[a]);                          // the MMA warp may reuse it
