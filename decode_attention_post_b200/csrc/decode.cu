@@ -42,7 +42,8 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 4.0f;     // rescale the running sums only when the max grows by > 2^4
-constexpr int kQprepSeqs = 2;     // sequences per q-prologue CTA
+constexpr int kQprepSeqs = 8;     // sequences per q-prologue CTA (one T_k^{-T} load serves
+                                  // 8 G query vectors)
 
 template <int D, int G, int BK, int BV>
 struct Cfg {

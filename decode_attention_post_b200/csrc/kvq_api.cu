@@ -487,6 +487,11 @@ kvq_status kvq_decode_attention_window(const void *q, kvq_dtype q_dtype, int Hq,
         return ws;
     if (q_dtype != KVQ_BF16)
         KVQ_FAIL(KVQ_ERR_UNSUPPORTED, "the windowed decode takes bfloat16 queries");
+    if (!aligned(win->k_recent, 16) || !aligned(win->v_recent, 16) ||
+        (win->S_sink > 0 && (!aligned(win->k_sink, 16) || !aligned(win->v_sink, 16))) ||
+        (win->T_v && !aligned(win->T_v, 16)) || !aligned(q, 4))
+        KVQ_FAIL(KVQ_ERR_INVALID_ARG,
+                 "window buffers and T_v must be 16-byte aligned, q 4-byte aligned");
     if (max_seqlen < 0)
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "max_seqlen=%d must be >= 0", max_seqlen);
     const int qmax = window_quantized(max_seqlen, win->S_sink, win->S_keep, win->S_flush);

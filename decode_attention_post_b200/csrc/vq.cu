@@ -206,16 +206,27 @@ struct VqCfg {
 
 // Expand the codewords of 16 tokens (indices idx [16][NGRP], one byte each) into the
 // float16 tile [16][TS]: entry (token, group) -> C[idx] at columns 4 group .. 4 group + 3.
+// Lane work item = 4 consecutive groups of one token: one 32-bit index load, four
+// codeword loads, two 16-byte stores; fully unrolled so that the loads overlap.
 template <int D>
 __device__ __forceinline__ void expand_tile(const uint8_t *idx, const uint2 *cb, __half *tile,
                                             int lane)
 {
-    constexpr int NGRP = D / kVqDim, TS = D + 8;
+    constexpr int NGRP = D / kVqDim, TS = D + 8, QUADS = kVqSub * NGRP / 4;
+    static_assert(QUADS % 32 == 0, "whole warp iterations");
+    uint32_t iw[QUADS / 32];
 #pragma unroll
-    for (int e = lane; e < kVqSub * NGRP; e += 32) {
-        const int tok = e / NGRP, grp = e % NGRP;
-        const uint2 w = cb[idx[e]];
-        *reinterpret_cast<uint2 *>(tile + tok * TS + kVqDim * grp) = w;
+    for (int m = 0; m < QUADS / 32; ++m)
+        iw[m] = reinterpret_cast<const uint32_t *>(idx)[lane + 32 * m];
+#pragma unroll
+    for (int m = 0; m < QUADS / 32; ++m) {
+        const int e4 = lane + 32 * m;                   // quad of groups 4 e4 .. 4 e4 + 3
+        const int tok = (4 * e4) / NGRP, grp = (4 * e4) % NGRP;
+        const uint2 w0 = cb[iw[m] & 0xFF], w1 = cb[(iw[m] >> 8) & 0xFF];
+        const uint2 w2 = cb[(iw[m] >> 16) & 0xFF], w3 = cb[iw[m] >> 24];
+        uint4 *dst = reinterpret_cast<uint4 *>(tile + tok * TS + kVqDim * grp);
+        dst[0] = make_uint4(w0.x, w0.y, w1.x, w1.y);
+        dst[1] = make_uint4(w2.x, w2.y, w3.x, w3.y);
     }
 }
 
@@ -391,8 +402,9 @@ vq_decode_kernel(const uint8_t *__restrict__ k_idx, const uint16_t *__restrict__
             }
             // ---- P' = p g^V as float16 (hi, lo): rows = tokens, columns (hi, lo) of head t;
             //      one 8x8 transpose per row half makes the B operand of the value product
-            const float gva = __half2float(__ushort_as_half(vg[ta]));
-            const float gvb = __half2float(__ushort_as_half(vg[tb]));
+            // masked tokens: gain 0 (cache bytes past the length may hold any bit pattern)
+            const float gva = va ? __half2float(__ushort_as_half(vg[ta])) : 0.f;
+            const float gvb = vb ? __half2float(__ushort_as_half(vg[tb])) : 0.f;
             uint32_t pb[C::NT][2];
 #pragma unroll
             for (int nt = 0; nt < C::NT; ++nt) {

@@ -4,13 +4,16 @@
 // as one more partial (running max, sum of weights, weighted sum of values) next to the
 // splits of the quantized middle, merged by the decode kernel's last split.
 //
-// One CTA per (KV head, sequence), 128 threads, for the G query heads of the KV head:
-//   logit_t = log2(e)/sqrt(d) * q . k_t  (the query as given: q . k = (T_k^{-T} q) . (T_k k)),
-//   m = max_t logit_t, p_t = 2^(logit_t - m), l = sum_t p_t, o = T_v sum_t p_t v_t,
-// in float32 on CUDA cores (the window is a few hundred positions at most), T_v applied
-// so that o is in the value-transform domain like the quantized values. The logits are in
-// log2 units, as the decode kernel's partials. When nothing of the sequence is quantized
-// the partial is the whole attention and o / l is written as the output.
+// One CTA per (KV head, sequence), 4 warps, for the G query heads of the KV head. The
+// window is the sink rows present plus every slot of the recent ring, each slot masked by
+// the position it holds (the softmax does not depend on the order). Each warp takes
+// 16-row tiles: key and value rows staged in shared memory by 16-byte asynchronous
+// copies, S = K q on bf16 tensor cores (the query as given, bf16, exact: q . k =
+// (T_k^{-T} q) . (T_k k)), logits in log2 units, float32 online softmax, O^T += V^T P^T
+// with P as bf16 (hi, lo) pairs; the warps merge in shared memory, T_v is applied once to
+// the merged sum so that o is in the value-transform domain like the quantized values.
+// When nothing of the sequence is quantized the partial is the whole attention and o / l
+// is written as the output.
 //
 // Ordering with the decode grid that follows: that grid is a programmatic dependent of
 // this kernel and its last split reads this partial and counts this kernel's ticket
@@ -27,111 +30,273 @@ namespace kvq {
 
 namespace {
 
-constexpr int kWinThreads = 128;
+constexpr int kWinWarps = 4;
+constexpr int kWinThreads = kWinWarps * 32;
 constexpr float kWinLog2e = 1.4426950408889634f;
+constexpr int kWinSub = 16;                     // window rows per MMA tile
+constexpr float kWinLazy = 4.0f;
+
+template <int D, int G>
+struct WinCfg {
+    static constexpr int TS = D + 8;            // bf16 per staged row (ldmatrix conflict-free)
+    static constexpr int TILE = kWinSub * TS;   // bf16 of one staged 16-row tile
+    static constexpr int NT = (2 * G) / 8;      // n-tiles of the value product ((hi, lo) x G)
+    static constexpr int NTK = 1;               // n-tiles of the key product (G <= 8 columns)
+    static constexpr int KS = D / 16;
+    static constexpr int MT = D / 16;
+    // per warp: K and V tiles; after the loop the same space holds the warps' partials
+    static constexpr int TILES = kWinWarps * 2 * TILE * 2;
+    static constexpr int MERGE = kWinWarps * G * (D + 2) * 4;
+    static constexpr int SMEM = (TILES > MERGE ? TILES : MERGE) + G * D * 4 + 2 * G * 4;
+};
+
+// Row w of the window: w < nsink is sink row w; otherwise ring slot w - nsink, valid when
+// the position it holds is in [rec0, L) (slot s holds the position t in [L - R, L) with
+// t = s mod R; the others are flushed or not yet written).
+struct WinRows {
+    const __nv_bfloat16 *sink, *ring;           // [S_sink][D] and [R][D] of this (seq, head)
+    int nsink, R, L, rec0;
+};
+
+__device__ __forceinline__ bool win_row(const WinRows &wr, int w, int D, const __nv_bfloat16 **row)
+{
+    if (w < wr.nsink) {
+        *row = wr.sink + (size_t)w * D;
+        return true;
+    }
+    const int s = w - wr.nsink;
+    int t = wr.L - wr.R + (((s - (wr.L - wr.R)) % wr.R) + wr.R) % wr.R;
+    *row = wr.ring + (size_t)s * D;
+    return t >= wr.rec0 && t < wr.L;
+}
 
 template <int D, int G>
 __global__ void __launch_bounds__(kWinThreads) window_kernel(WindowParams W)
 {
-    extern __shared__ __align__(16) float wsm[];
+    using C = WinCfg<D, G>;
+    extern __shared__ __align__(16) unsigned char wsm_raw[];
+    __nv_bfloat16 *tiles = reinterpret_cast<__nv_bfloat16 *>(wsm_raw);
+    float *ofin = reinterpret_cast<float *>(wsm_raw + (C::TILES > C::MERGE ? C::TILES : C::MERGE));
     const int h = blockIdx.x, b = blockIdx.y;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int R = W.S_keep + W.S_flush;                 // recent ring slots
-    const int WMAX = W.S_sink + R;                      // window positions at most
-    float *qf = wsm;                                    // [G][D]
-    float *of = qf + G * D;                             // [G][D]
-    float *stat = of + G * D;                           // [G][2]: m, l
-    float *lg = stat + 2 * G;                           // [G][WMAX]: logits, then weights
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int R = W.S_keep + W.S_flush;
 
     int L = W.seqlens[b];
     L = L < 0 ? 0 : (L > W.max_seqlen ? W.max_seqlen : L);
     if (L == 0)
         return;                                         // the q prologue wrote zeros
     const int Q = window_quantized(L, W.S_sink, W.S_keep, W.S_flush);
-    const int nsink = min(W.S_sink, L);
-    const int rec0 = W.S_sink + Q;                      // first recent position
-    const int nrec = L > rec0 ? L - rec0 : 0;
-    const int nw = nsink + nrec;
     const size_t pair = (size_t)b * W.Hkv + h;
+    WinRows kr, vr;
+    kr.nsink = vr.nsink = min(W.S_sink, L);
+    kr.R = vr.R = R;
+    kr.L = vr.L = L;
+    kr.rec0 = vr.rec0 = W.S_sink + Q;
+    kr.sink = reinterpret_cast<const __nv_bfloat16 *>(W.k_sink) + pair * W.S_sink * D;
+    vr.sink = reinterpret_cast<const __nv_bfloat16 *>(W.v_sink) + pair * W.S_sink * D;
+    kr.ring = reinterpret_cast<const __nv_bfloat16 *>(W.k_recent) + pair * R * D;
+    vr.ring = reinterpret_cast<const __nv_bfloat16 *>(W.v_recent) + pair * R * D;
+    // rows to scan: the sink rows present, then every ring slot (masked by position)
+    const int nrows = kr.nsink + (L > kr.rec0 ? R : 0);
+    const int ntiles = (nrows + kWinSub - 1) / kWinSub;
     const float sc = kWinLog2e * rsqrtf((float)D);
+    __nv_bfloat16 *ktile = tiles + (size_t)warp * 2 * C::TILE;
+    __nv_bfloat16 *vtile = ktile + C::TILE;
 
-    // row of window position w (w < nsink: sink, else recent ring slot)
-    auto k_row = [&](int w) -> const __nv_bfloat16 * {
-        if (w < nsink)
-            return reinterpret_cast<const __nv_bfloat16 *>(W.k_sink) +
-                   (pair * W.S_sink + w) * D;
-        const int t = rec0 + (w - nsink);
-        return reinterpret_cast<const __nv_bfloat16 *>(W.k_recent) + (pair * R + t % R) * D;
-    };
-    auto v_row = [&](int w) -> const __nv_bfloat16 * {
-        if (w < nsink)
-            return reinterpret_cast<const __nv_bfloat16 *>(W.v_sink) +
-                   (pair * W.S_sink + w) * D;
-        const int t = rec0 + (w - nsink);
-        return reinterpret_cast<const __nv_bfloat16 *>(W.v_recent) + (pair * R + t % R) * D;
-    };
-
-    for (int idx = tid; idx < G * D; idx += kWinThreads)
-        qf[idx] = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(
-            W.q)[((size_t)b * W.Hq + h * G + idx / D) * D + idx % D]);
-    __syncthreads();
-    // ---- logits: thread per (head, position)
-    for (int idx = tid; idx < G * nw; idx += kWinThreads) {
-        const int head = idx / nw, w = idx % nw;
-        const __nv_bfloat16 *kr = k_row(w);
-        const float *qh = qf + head * D;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < D; ++j)
-            acc = fmaf(qh[j], __bfloat162float(kr[j]), acc);
-        lg[head * WMAX + w] = sc * acc;
-    }
-    __syncthreads();
-    // ---- per head: max, weights 2^(logit - m), their sum
-    for (int head = warp; head < G; head += kWinThreads / 32) {
-        float m = -INFINITY;
-        for (int w = lane; w < nw; w += 32)
-            m = fmaxf(m, lg[head * WMAX + w]);
+    // q of the G heads (bf16, exact) as the B operand of S = K . q: column n = head n
+    uint32_t qB[C::NTK][C::KS][2];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        float l = 0.f;
-        for (int w = lane; w < nw; w += 32) {
-            const float p = ex2(lg[head * WMAX + w] - m);
-            lg[head * WMAX + w] = p;
-            l += p;
+    for (int nt = 0; nt < C::NTK; ++nt) {
+        const int head = 8 * nt + g;
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t v = 0;
+                if (head < G)
+                    v = *reinterpret_cast<const uint32_t *>(
+                        reinterpret_cast<const __nv_bfloat16 *>(W.q) +
+                        ((size_t)b * W.Hq + h * G + head) * D + 16 * ks + 8 * hh + 2 * t);
+                qB[nt][ks][hh] = v;
+            }
+    }
+
+    float m_run[C::NT], l_run[C::NT];
+    float O[C::MT][C::NT][4];
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt) {
+        m_run[nt] = -INFINITY;
+        l_run[nt] = 0.f;
+#pragma unroll
+        for (int m = 0; m < C::MT; ++m)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                O[m][nt][i] = 0.f;
+    }
+
+    for (int tt = warp; tt < ntiles; tt += kWinWarps) {
+        const int w0 = tt * kWinSub;
+        // ---- stage the tile's key and value rows (16-byte copies). Rows past the end and
+        //      ring slots not holding a window position are zero-filled: their weight is 0,
+        //      and a never-written slot may hold any bit pattern (0 * NaN would not be 0).
+        for (int c = lane; c < 2 * kWinSub * (D / 8); c += 32) {
+            const int which = c / (kWinSub * (D / 8)), cc = c % (kWinSub * (D / 8));
+            const int rr = cc / (D / 8), ch = cc % (D / 8);
+            const __nv_bfloat16 *row = nullptr;
+            bool ok = false;
+            if (w0 + rr < nrows)
+                ok = win_row(which ? vr : kr, w0 + rr, D, &row);
+            __nv_bfloat16 *dst = (which ? vtile : ktile) + rr * C::TS + 8 * ch;
+            cp_async16(dst, ok ? row + 8 * ch : kr.ring, ok ? 16 : 0);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
+        // validity of this lane's two rows (g and g + 8 of the tile)
+        const __nv_bfloat16 *dummy;
+        const bool va = w0 + g < nrows && win_row(kr, w0 + g, D, &dummy);
+        const bool vb = w0 + g + 8 < nrows && win_row(kr, w0 + g + 8, D, &dummy);
+        // ---- S[16 x G] = Ktile . q
+        float S[C::NTK][4];
+#pragma unroll
+        for (int nt = 0; nt < C::NTK; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                S[nt][i] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+            uint32_t a[4];
+            ldmatrix_x4(a, ktile + (lane & 15) * C::TS + 16 * ks + 8 * (lane >> 4));
+#pragma unroll
+            for (int nt = 0; nt < C::NTK; ++nt)
+                mma_bf16(S[nt], a[0], a[1], a[2], a[3], qB[nt][ks][0], qB[nt][ks][1]);
+        }
+        // The key product's accumulator has row g, columns 2t, 2t+1 = heads 2t, 2t+1 (G <= 8:
+        // one n-tile); the value product wants head 4 nt + t on this lane. Its logits come
+        // from the quad lane holding that head.
+        float la[C::NT], lb[C::NT];
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt) {
+            const int head = 4 * nt + t;
+            const int src = (lane & ~3) | ((head & 7) >> 1);
+            const float sa0 = __shfl_sync(0xffffffffu, S[0][0], src);
+            const float sa1 = __shfl_sync(0xffffffffu, S[0][1], src);
+            const float sb0 = __shfl_sync(0xffffffffu, S[0][2], src);
+            const float sb1 = __shfl_sync(0xffffffffu, S[0][3], src);
+            la[nt] = va ? sc * ((head & 1) ? sa1 : sa0) : -INFINITY;
+            lb[nt] = vb ? sc * ((head & 1) ? sb1 : sb0) : -INFINITY;
+            float bm = fmaxf(la[nt], lb[nt]);
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+            if (bm > m_run[nt] + kWinLazy) {
+                const float alpha = ex2(m_run[nt] - bm);
+                l_run[nt] *= alpha;
+#pragma unroll
+                for (int m = 0; m < C::MT; ++m)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        O[m][nt][i] *= alpha;
+                m_run[nt] = bm;
+            }
+        }
+        // ---- P as bf16 (hi, lo) pairs, rows = window rows, columns (hi, lo) of head
+        //      4nt + t; 8x8 transposes make the B operand of the value product
+        uint32_t pb[C::NT][2];
+#pragma unroll
+        for (int nt = 0; nt < C::NT; ++nt) {
+            // no valid row seen yet: every logit so far is -inf and every weight 0
+            const float mr = m_run[nt] == -INFINITY ? 0.f : m_run[nt];
+            const float pa = ex2(la[nt] - mr), pbv = ex2(lb[nt] - mr);
+            l_run[nt] += pa + pbv;
+            const __nv_bfloat16 ha = __float2bfloat16_rn(pa), hb = __float2bfloat16_rn(pbv);
+            const __nv_bfloat162 ra2 =
+                __halves2bfloat162(ha, __float2bfloat16_rn(pa - __bfloat162float(ha)));
+            const __nv_bfloat162 rb2 =
+                __halves2bfloat162(hb, __float2bfloat16_rn(pbv - __bfloat162float(hb)));
+            pb[nt][0] = movmatrix_trans(*reinterpret_cast<const uint32_t *>(&ra2));
+            pb[nt][1] = movmatrix_trans(*reinterpret_cast<const uint32_t *>(&rb2));
+        }
+        // ---- O^T[D x 2G] += Vtile^T . P^T
+#pragma unroll
+        for (int m = 0; m < C::MT; ++m) {
+            const int q = lane >> 3;
+            uint32_t a[4];
+            ldmatrix_x4_trans(a, vtile + (8 * (q >> 1) + (lane & 7)) * C::TS + 16 * m + 8 * (q & 1));
+#pragma unroll
+            for (int nt = 0; nt < C::NT; ++nt)
+                mma_bf16(O[m][nt], a[0], a[1], a[2], a[3], pb[nt][0], pb[nt][1]);
+        }
+        __syncwarp();                                   // the tiles are refilled next
+    }
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt)
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1)
+            l_run[nt] += __shfl_xor_sync(0xffffffffu, l_run[nt], off);
+
+    // ---- merge the warps (log2-scaled (m, l, o) in shared memory)
+    __syncthreads();
+    float *mw = reinterpret_cast<float *>(wsm_raw);
+    float *lw = mw + kWinWarps * G;
+    float *ow = lw + kWinWarps * G;
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt) {
+        const int head = 4 * nt + t;
+        if (g == 0) {
+            mw[warp * G + head] = m_run[nt];
+            lw[warp * G + head] = l_run[nt];
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            l += __shfl_xor_sync(0xffffffffu, l, off);
-        if (lane == 0) {
-            stat[2 * head] = m;
-            stat[2 * head + 1] = l;
+        for (int m = 0; m < C::MT; ++m) {
+            ow[(warp * G + head) * D + 16 * m + g] = O[m][nt][0] + O[m][nt][1];
+            ow[(warp * G + head) * D + 16 * m + g + 8] = O[m][nt][2] + O[m][nt][3];
         }
     }
     __syncthreads();
-    // ---- sum_t p_t v_t (untransformed values): thread per (head, dim)
-    for (int idx = tid; idx < G * D; idx += kWinThreads) {
-        const int head = idx / D, j = idx % D;
-        float acc = 0.f;
-        for (int w = 0; w < nw; ++w)
-            acc = fmaf(lg[head * WMAX + w], __bfloat162float(v_row(w)[j]), acc);
-        of[idx] = acc;
+    float *stat = ofin + G * D;                         // [G][2]
+    for (int idx = threadIdx.x; idx < G * D; idx += kWinThreads) {
+        const int head = idx / D, dim = idx % D;
+        float Mx = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWinWarps; ++w)
+            Mx = fmaxf(Mx, mw[w * G + head]);
+        float Lsum = 0.f, o = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWinWarps; ++w) {
+            const float mwv = mw[w * G + head];
+            if (mwv == -INFINITY)
+                continue;
+            const float wt = ex2(mwv - Mx);
+            Lsum = fmaf(wt, lw[w * G + head], Lsum);
+            o = fmaf(wt, ow[(w * G + head) * D + dim], o);
+        }
+        ofin[idx] = o;
+        if (dim == 0) {
+            stat[2 * head] = Mx;
+            stat[2 * head + 1] = Lsum;
+        }
     }
     __syncthreads();
-    // ---- o = T_v (sum p v), then the partial (or the output)
+    // ---- o = T_v (sum p v), then the partial (or the output); thread per (head, dim i)
     const float *Tv = W.T_v ? W.T_v + (size_t)h * D * D : nullptr;
     float *part = W.part + (pair * W.part_slots + W.slot) * (size_t)(G * (D + 2));
-    for (int idx = tid; idx < G * D; idx += kWinThreads) {
+    for (int idx = threadIdx.x; idx < G * D; idx += kWinThreads) {
         const int head = idx / D, i = idx % D;
-        float o = of[idx];
+        float o = ofin[idx];
         if (Tv) {
-            const float *row = Tv + (size_t)i * D;
-            const float *oh = of + head * D;
+            const float4 *row = reinterpret_cast<const float4 *>(Tv + (size_t)i * D);
+            const float4 *oh = reinterpret_cast<const float4 *>(ofin + head * D);
             float acc = 0.f;
 #pragma unroll 8
-            for (int j = 0; j < D; ++j)
-                acc = fmaf(row[j], oh[j], acc);
+            for (int j4 = 0; j4 < D / 4; ++j4) {
+                const float4 tr = row[j4], ov = oh[j4];
+                acc = fmaf(tr.x, ov.x, acc);
+                acc = fmaf(tr.y, ov.y, acc);
+                acc = fmaf(tr.z, ov.z, acc);
+                acc = fmaf(tr.w, ov.w, acc);
+            }
             o = acc;
         }
         if (Q == 0) {
@@ -152,32 +317,21 @@ __global__ void __launch_bounds__(kWinThreads) window_kernel(WindowParams W)
     if (Q > 0) {
         // count this partial in the pair's ticket: the decode kernel's last split merges it
         __syncthreads();
-        if (tid == 0) {
+        if (threadIdx.x == 0) {
             __threadfence();
             atomicAdd(&W.ticket[pair], 1);
         }
     }
 }
 
-constexpr int kWinMaxPositions = 2048;       // S_sink + S_keep + S_flush limit (host-checked)
-
-template <int D, int G>
-constexpr size_t window_smem_bytes(int positions)
-{
-    return (size_t)(2 * G * D + 2 * G + G * positions) * sizeof(float);
-}
-
 template <int D, int G>
 cudaError_t launch_window_t(const WindowParams &W, cudaStream_t st)
 {
-    const int WMAX = W.S_sink + W.S_keep + W.S_flush;
-    // the attribute is set once per device for the largest window, so every call fits
     static unsigned long long attr_done = 0;
-    cudaError_t e = ensure_dynamic_smem(window_kernel<D, G>,
-                                        (int)window_smem_bytes<D, G>(kWinMaxPositions), attr_done);
+    cudaError_t e = ensure_dynamic_smem(window_kernel<D, G>, WinCfg<D, G>::SMEM, attr_done);
     if (e != cudaSuccess)
         return e;
-    window_kernel<D, G><<<dim3(W.Hkv, W.B), kWinThreads, window_smem_bytes<D, G>(WMAX), st>>>(W);
+    window_kernel<D, G><<<dim3(W.Hkv, W.B), kWinThreads, WinCfg<D, G>::SMEM, st>>>(W);
     return cudaGetLastError();
 }
 

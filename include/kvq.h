@@ -242,8 +242,11 @@ typedef struct {
  * Decode with a full-precision window: seqlens[b] = L (all positions of sequence b,
  * L <= max_seqlen); full-precision positions attend with the query as given (q . k,
  * = (T_k^{-T} q) . (T_k k)), quantized ones as in kvq_decode_attention; one softmax over
- * all L positions. q must be bfloat16. The quantized middle of max_seqlen positions must
- * fit the cache (Q(max_seqlen) <= T_cap); S_sink + S_keep + S_flush <= 2048. Workspace:
+ * all L positions. q must be bfloat16. The window buffers and T_v must be 16-byte aligned
+ * and q 4-byte aligned (KVQ_ERR_INVALID_ARG otherwise). The quantized middle of max_seqlen
+ * positions must fit the cache (Q(max_seqlen) <= T_cap); S_sink + S_keep + S_flush <= 2048.
+ * Ring slots that hold no window position are never read into the result, whatever their
+ * contents. Workspace:
  * kvq_decode_workspace_bytes(cache, Hq, m) for any m >= Q(max_seqlen) (m = T_cap always
  * suffices, as that size never decreases with m). Other arguments and errors as in
  * kvq_decode_attention.

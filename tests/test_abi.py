@@ -171,6 +171,12 @@ def test_window_decode_argument_errors():
     # the quantized middle of max_seqlen must fit the cache: 4 + 32 + 128 fits, + 64 not
     assert _window_decode(desc, _win(), max_seqlen=4 + 32 + 192 + 63) == 3
     assert _window_decode(desc, _win(), ws_bytes=16) == 4
+    # 16-byte copies of window rows and float4 reads of T_v: misaligned buffers refused
+    assert _window_decode(desc, _win(kr=0xA008)) == 1
+    assert _window_decode(desc, _win(vs=0x9004)) == 1
+    w = _win()
+    w.T_v = 0xB004
+    assert _window_decode(desc, w) == 1
     assert kvq.load().kvq_last_error()
 
 
