@@ -32,6 +32,7 @@
 #include "kvq_common.cuh"
 #include "kvq_ptx.cuh"
 #include "decode_shapes.h"
+#include "window_attn.cuh"
 
 #include <math.h>
 #include <type_traits>
@@ -42,7 +43,7 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 4.0f;     // rescale the running sums only when the max grows by > 2^4
-constexpr int kQprepSeqs = 8;     // sequences per q-prologue CTA (one T_k^{-T} load serves
+constexpr int kQprepSeqs = 2;     // sequences per q-prologue CTA (one T_k^{-T} load serves
                                   // 8 G query vectors)
 
 template <int D, int G, int BK, int BV>
@@ -66,9 +67,12 @@ struct Cfg {
     static constexpr int QFRAG = NT * KS * 32 * 2;
     static constexpr int RING = kDecodeWarps * kDecodeStages * STAGE;
     static constexpr int MERGE = kDecodeWarps * G * (D + 2) * 4;
-    // ring (or merge area), stage barriers, one test-hook barrier per warp, merge flag
-    static constexpr int SMEM =
-        (RING > MERGE ? RING : MERGE) + kDecodeWarps * (kDecodeStages + 1) * 8 + 16;
+    // the ring, the merge area after it, or the window split's tiles and sums
+    static constexpr int AREA0 = RING > MERGE ? RING : MERGE;
+    static constexpr int WIN = win::Smem<D, G>::BYTES;
+    static constexpr int AREA = ((AREA0 > WIN ? AREA0 : WIN) + 15) / 16 * 16;
+    // area, stage barriers, one test-hook barrier per warp, merge flag
+    static constexpr int SMEM = AREA + kDecodeWarps * (kDecodeStages + 1) * 8 + 16;
     // resident CTAs per SM the register budget targets: kDecodeMinBlocks, or fewer when
     // shared memory (227 KB per SM, 1 KB reserved per CTA) holds fewer
     static constexpr int SMEM_FIT = (227 * 1024) / (SMEM + 1024);
@@ -314,14 +318,62 @@ qprep_kernel(const void *__restrict__ q, int q_bf16, const float *__restrict__ M
 
 // ---------------------------------------------------------------- main decode
 
-template <int D, int G, int BK, int BV>
+// The last CTA of a (sequence, KV head) to finish -- a split or the window split --
+// merges every partial of the pair: slots 0 .. nsplit_b - 1 hold the splits, the last slot
+// the window's. The barrier orders every thread's partial stores before thread 0's
+// device-scope fence and ticket; the merging CTA's thread 0 fences after its ticket and
+// the barrier orders that before every thread's loads.
+template <int D, int G>
+__device__ __forceinline__ void merge_if_last(const DecodeParams &P, size_t pair, int b, int h,
+                                              int nmerge, int nsplit_b, int *flag_smem)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int last = (atomicAdd(&P.ticket[pair], 1) == nmerge - 1);
+        __threadfence();
+        *flag_smem = last;
+    }
+    __syncthreads();
+    if (!*flag_smem)
+        return;
+    const float *pall = P.part + pair * P.part_slots * (size_t)(G * (D + 2));
+    for (int idx = threadIdx.x; idx < G * D; idx += kDecodeWarps * 32) {
+        const int head = idx / D, dim = idx % D;
+        float Mx = -INFINITY;
+        for (int i = 0; i < nmerge; ++i) {
+            const int sg = i < nsplit_b ? i : P.part_slots - 1;
+            Mx = fmaxf(Mx, __ldcg(pall + (size_t)sg * G * (D + 2) + head * (D + 2)));
+        }
+        float L = 0.f, o = 0.f;
+        for (int i = 0; i < nmerge; ++i) {
+            const int sg = i < nsplit_b ? i : P.part_slots - 1;
+            const float *pp = pall + (size_t)sg * G * (D + 2) + head * (D + 2);
+            const float m = __ldcg(pp);
+            if (m == -INFINITY)
+                continue;                       // a partial that saw no position
+            const float wt = ex2(m - Mx);
+            L = fmaf(wt, __ldcg(pp + 1), L);
+            o = fmaf(wt, __ldcg(pp + 2 + dim), o);
+        }
+        const size_t oi = ((size_t)b * P.Hq + h * G + head) * D + dim;
+        const float r = o / L;
+        if (P.out_bf16)
+            reinterpret_cast<__nv_bfloat16 *>(P.out)[oi] = __float2bfloat16_rn(r);
+        else
+            reinterpret_cast<float *>(P.out)[oi] = r;
+    }
+}
+
+// WIN: the grid has one more split per pair, the full-precision window's (split nsplit);
+// a separate instantiation, so that the plain decode carries none of its code.
+template <int D, int G, int BK, int BV, bool WIN>
 __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) decode_kernel(DecodeParams P)
 {
     using C = Cfg<D, G, BK, BV>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *ring = smem_raw;
-    uint64_t *bars_all =
-        reinterpret_cast<uint64_t *>(smem_raw + (C::RING > C::MERGE ? C::RING : C::MERGE));
+    uint64_t *bars_all = reinterpret_cast<uint64_t *>(smem_raw + C::AREA);
     uint64_t *stall_bars = bars_all + kDecodeWarps * kDecodeStages;
     int *flag_smem = reinterpret_cast<int *>(stall_bars + kDecodeWarps);
 
@@ -345,15 +397,47 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
             flag(P.dev_err, KVQ_DEVERR_SEQLEN_CLAMPED);
         seqlen = seqlen < 0 ? 0 : P.max_seqlen;
     }
-    const bool windowed = P.win_flush > 0;
+    constexpr bool windowed = WIN;
+    const int L_all = seqlen;
     if (windowed)                               // the cache holds the quantized middle only
         seqlen = window_quantized(seqlen, P.win_sink, P.win_keep, P.win_flush);
+    const int nsplit_b = (seqlen + P.split_tokens - 1) / P.split_tokens;
+    const int nmerge = nsplit_b + (windowed ? 1 : 0);   // partials merged for the pair
+    if (WIN && sigma == P.nsplit) {
+        // ---- the window split: its partial in the last slot, or the output when nothing
+        //      of the sequence is quantized
+        if (L_all == 0)
+            return;                             // the prologue wrote zeros
+        const float *o, *stat;
+        win::attend<D, G>(P, b, h, L_all, seqlen, smem_raw, &o, &stat);
+        float *part = P.part + (pair * P.part_slots + P.part_slots - 1) * (size_t)(G * (D + 2));
+        for (int idx = threadIdx.x; idx < G * D; idx += kDecodeWarps * 32) {
+            const int head = idx / D, dim = idx % D;
+            if (nmerge == 1) {
+                const size_t oi = ((size_t)b * P.Hq + h * G + head) * D + dim;
+                const float r = o[idx] / stat[2 * head + 1];
+                if (P.out_bf16)
+                    reinterpret_cast<__nv_bfloat16 *>(P.out)[oi] = __float2bfloat16_rn(r);
+                else
+                    reinterpret_cast<float *>(P.out)[oi] = r;
+            } else {
+                part[head * (D + 2) + 2 + dim] = o[idx];
+                if (dim == 0) {
+                    part[head * (D + 2)] = stat[2 * head];
+                    part[head * (D + 2) + 1] = stat[2 * head + 1];
+                }
+            }
+        }
+        if (nmerge == 1)
+            return;
+        asm volatile("griddepcontrol.wait;" ::: "memory");   // the prologue zeroed the ticket
+        merge_if_last<D, G>(P, pair, b, h, nmerge, nsplit_b, flag_smem);
+        return;
+    }
     const int t_begin = sigma * P.split_tokens;
     if (t_begin >= seqlen)
         return;                                 // nothing here (the prologue zeroes empty ones)
     const int t_end = min(t_begin + P.split_tokens, seqlen);
-    const int nsplit_b = (seqlen + P.split_tokens - 1) / P.split_tokens;
-    const int nmerge = nsplit_b + (windowed ? 1 : 0);   // partials merged for the pair
     const int nblk = (t_end - t_begin + kDecodeBlock - 1) / kDecodeBlock;
     const int my_nblk = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
 
@@ -702,45 +786,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     }
     if (nmerge == 1)
         return;
-    // ---- the last split of the pair to finish merges all splits (and the window's
-    //      partial, counted in the ticket before this kernel started). The barrier orders
-    //      every thread's partial stores before thread 0's device-scope fence and ticket;
-    //      the merging CTA's thread 0 fences after its ticket and the barrier orders that
-    //      before every thread's loads.
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const int last = (atomicAdd(&P.ticket[pair], 1) == nmerge - 1);
-        __threadfence();
-        *flag_smem = last;
-    }
-    __syncthreads();
-    if (!*flag_smem)
-        return;
-    const float *pall = P.part + pair * P.part_slots * (size_t)(G * (D + 2));
-    // slots 0 .. nsplit_b-1 hold the splits; the window's partial is in the last slot
-    for (int idx = threadIdx.x; idx < G * D; idx += kDecodeWarps * 32) {
-        const int head = idx / D, dim = idx % D;
-        float Mx = -INFINITY;
-        for (int i = 0; i < nmerge; ++i) {
-            const int sg = i < nsplit_b ? i : P.part_slots - 1;
-            Mx = fmaxf(Mx, __ldcg(pall + (size_t)sg * G * (D + 2) + head * (D + 2)));
-        }
-        float L = 0.f, o = 0.f;
-        for (int i = 0; i < nmerge; ++i) {
-            const int sg = i < nsplit_b ? i : P.part_slots - 1;
-            const float *pp = pall + (size_t)sg * G * (D + 2) + head * (D + 2);
-            const float wt = ex2(__ldcg(pp) - Mx);
-            L = fmaf(wt, __ldcg(pp + 1), L);
-            o = fmaf(wt, __ldcg(pp + 2 + dim), o);
-        }
-        const size_t oi = ((size_t)b * P.Hq + h * G + head) * D + dim;
-        const float r = o / L;
-        if (P.out_bf16)
-            reinterpret_cast<__nv_bfloat16 *>(P.out)[oi] = __float2bfloat16_rn(r);
-        else
-            reinterpret_cast<float *>(P.out)[oi] = r;
-    }
+    merge_if_last<D, G>(P, pair, b, h, nmerge, nsplit_b, flag_smem);
 }
 
 template <int D, int G, int BK, int BV>
@@ -748,11 +794,13 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
 {
     using C = Cfg<D, G, BK, BV>;
     using QS = QprepSmem<D, G>;
-    static unsigned long long qprep_attr = 0, decode_attr = 0;
+    static unsigned long long qprep_attr = 0, decode_attr = 0, decode_win_attr = 0;
     cudaError_t e = ensure_dynamic_smem(qprep_kernel<D, G, BK>, QS::BYTES, qprep_attr);
     if (e != cudaSuccess)
         return e;
-    e = ensure_dynamic_smem(decode_kernel<D, G, BK, BV>, C::SMEM, decode_attr);
+    const bool win = L.p.win_flush > 0;
+    e = win ? ensure_dynamic_smem(decode_kernel<D, G, BK, BV, true>, C::SMEM, decode_win_attr)
+            : ensure_dynamic_smem(decode_kernel<D, G, BK, BV, false>, C::SMEM, decode_attr);
     if (e != cudaSuccess)
         return e;
     // q prologue
@@ -766,18 +814,11 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
         if (e != cudaSuccess)
             return e;
     }
-    // full-precision window: its partial and ticket count before the decode's merges
-    if (L.win) {
-        e = launch_window(*L.win, st);
-        if (e != cudaSuccess)
-            return e;
-    }
     // decode: CTA (KV head, sequence, split), splits slowest so that the short last
-    // splits of the sequences run last; a programmatic dependent of the kernel launched
-    // just before it (qprep, or the window kernel, which never triggers its dependents
-    // early, so its partial and ticket are complete before this grid's wait returns)
+    // splits of the sequences run last, then the window splits (split nsplit) when there is
+    // a full-precision window; a programmatic dependent of qprep
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(L.p.Hkv, L.p.B, L.p.nsplit);
+    cfg.gridDim = dim3(L.p.Hkv, L.p.B, L.p.nsplit + (win ? 1 : 0));
     cfg.blockDim = dim3(kDecodeWarps * 32);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
@@ -786,7 +827,8 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<D, G, BK, BV>, L.p);
+    return win ? cudaLaunchKernelEx(&cfg, decode_kernel<D, G, BK, BV, true>, L.p)
+               : cudaLaunchKernelEx(&cfg, decode_kernel<D, G, BK, BV, false>, L.p);
 }
 
 template <int D, int G>

@@ -35,35 +35,19 @@ struct DecodeParams {
     int part_slots;             // partial slots per (sequence, KV head): split slots
                                 // (>= nsplit) + 1, the last one for the window's partial
     // full-precision window (win_flush = 0: none): the cache holds the quantized middle,
-    // seqlens are whole lengths, the last slot holds the window's partial
+    // seqlens are whole lengths; split nsplit of every pair attends over the window and
+    // its partial goes to the last slot
     int win_sink, win_keep, win_flush;
+    const void *win_q;                                  // bfloat16 [B][Hq][d], as given
+    const void *k_sink, *v_sink, *k_recent, *v_recent;  // bfloat16 window rows
+    const float *win_Tv;                                // [Hkv][d][d] or nullptr
     // > 0: failure-path test hook, each warp first waits this long on a barrier that
     // nothing arrives at, then takes the timeout path (KVQ_TEST_STALL_NS in kvq.h)
     long long stall_test_ns;
 };
 
-// The window's attention: one CTA per (KV head, sequence) over the full-precision
-// positions, written as the extra partial of the pair (or as the output when nothing of
-// the sequence is quantized).
-struct WindowParams {
-    const void *q;              // bfloat16 [B][Hq][d]
-    const void *k_sink, *v_sink, *k_recent, *v_recent;
-    const float *T_v;
-    const int32_t *seqlens;
-    int B, Hkv, Hq, d, max_seqlen;
-    int S_sink, S_keep, S_flush;
-    float *part;
-    int part_slots, slot;
-    int *ticket;
-    void *out;
-    int out_bf16;
-};
-
-struct WindowParams;
-
 struct DecodeLaunch {
     DecodeParams p;
-    const WindowParams *win;    // full-precision window, launched between qprep and decode
     const void *q;
     int q_bf16;
     const float *M;
@@ -78,7 +62,6 @@ struct DecodeWorkspace {
 size_t decode_qfrag_words(int d, int G);
 int decode_resident_ctas(int d, int G, int bk, int bv);
 cudaError_t launch_decode(const DecodeLaunch &L, cudaStream_t st);
-cudaError_t launch_window(const WindowParams &W, cudaStream_t st);
 cudaError_t launch_qprep_qt(const DecodeLaunch &L, float *qt_out, cudaStream_t st);
 
 // Vector-quantized decode: the query prologue (writing q~ to qt) and the VQ decode grid

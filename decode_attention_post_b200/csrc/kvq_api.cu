@@ -143,11 +143,15 @@ static int num_sms()
 // 0.073 -> 0.055 ms against 4 waves). With fewer, about 4 waves: the short last splits of
 // ragged sequences then fill the tail (batch 64 x U[12K, 16K]: 5 splits best).
 // KVQ_DECODE_SPLITS overrides it (tuning).
-static long target_splits(int B, int Hkv, int resident)
+static long target_splits(int B, int Hkv, int resident, bool window = false)
 {
     const long pairs = (long)B * Hkv;
     const long slots = (long)num_sms() * (resident > 0 ? resident : kDecodeMinBlocks);
     long ns = slots >= 2 * pairs ? slots / pairs : (4 * slots + pairs - 1) / pairs;
+    // a windowed decode adds one window split per pair: when the splits fill one wave,
+    // leave room in it for the window splits (never more splits than without a window)
+    if (window && slots >= 2 * pairs)
+        ns = (slots - pairs) / pairs;
     if (const char *e = getenv("KVQ_DECODE_SPLITS"))
         ns = atol(e);
     return ns < 1 ? 1 : ns;
@@ -161,10 +165,11 @@ static int blocks_of(int max_seqlen)
 // Splits along the tokens; each split is a whole number of 64-token blocks. The count
 // is ceil(blocks / ceil(blocks / ns)) with ns = min(target, blocks), which is at most ns;
 // it is not monotonic in max_seqlen (75 blocks over 74 target splits give 38 splits).
-static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens, int resident)
+static int choose_splits(int B, int Hkv, int max_seqlen, int *split_tokens, int resident,
+                         bool window = false)
 {
     const int blocks = blocks_of(max_seqlen);
-    long ns = target_splits(B, Hkv, resident);
+    long ns = target_splits(B, Hkv, resident, window);
     if (ns > blocks)
         ns = blocks;
     const int bps = (int)((blocks + ns - 1) / ns);
@@ -322,7 +327,7 @@ static kvq_status decode_common(const void *q, kvq_dtype q_dtype, int Hq, const 
         KVQ_FAIL(KVQ_ERR_INVALID_ARG, "q_dtype/out_dtype must be KVQ_F32 or KVQ_BF16");
     int split_tokens = 0;
     const int res = decode_resident_ctas(c->d, Hq / c->Hkv, c->qp.bits_k, c->qp.bits_v);
-    const int ns = choose_splits(c->B, c->Hkv, qmax, &split_tokens, res);
+    const int ns = choose_splits(c->B, c->Hkv, qmax, &split_tokens, res, win != nullptr);
     const int nslots = split_slots(c->B, c->Hkv, qmax, res);     // >= ns
     const DecodeWorkspace w = decode_layout(c->B, c->Hkv, Hq, c->d, nslots);
     if (!workspace || !aligned(workspace, 256))
@@ -368,32 +373,12 @@ static kvq_status decode_common(const void *q, kvq_dtype q_dtype, int Hq, const 
     L.G = Hq / c->Hkv;
     L.bits_k = c->qp.bits_k;
     L.bits_v = c->qp.bits_v;
-    WindowParams W;
-    L.win = nullptr;
-    if (win) {
-        W.q = q;
-        W.k_sink = win->k_sink;
-        W.v_sink = win->v_sink;
-        W.k_recent = win->k_recent;
-        W.v_recent = win->v_recent;
-        W.T_v = win->T_v;
-        W.seqlens = seqlens;
-        W.B = c->B;
-        W.Hkv = c->Hkv;
-        W.Hq = Hq;
-        W.d = c->d;
-        W.max_seqlen = max_seqlen;
-        W.S_sink = win->S_sink;
-        W.S_keep = win->S_keep;
-        W.S_flush = win->S_flush;
-        W.part = L.p.part;
-        W.part_slots = L.p.part_slots;
-        W.slot = nslots;
-        W.ticket = L.p.ticket;
-        W.out = out;
-        W.out_bf16 = L.p.out_bf16;
-        L.win = &W;
-    }
+    L.p.win_q = win ? q : nullptr;
+    L.p.k_sink = win ? win->k_sink : nullptr;
+    L.p.v_sink = win ? win->v_sink : nullptr;
+    L.p.k_recent = win ? win->k_recent : nullptr;
+    L.p.v_recent = win ? win->v_recent : nullptr;
+    L.p.win_Tv = win ? win->T_v : nullptr;
     cudaError_t e = launch_decode(L, (cudaStream_t)stream);
     if (e != cudaSuccess)
         KVQ_FAIL(KVQ_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
@@ -660,7 +645,6 @@ kvq_status kvq_vq_decode_attention(const void *q, kvq_dtype q_dtype, int Hq, con
     L.p.out_bf16 = out_dtype == KVQ_BF16;
     L.p.dev_err = dev_err;
     L.p.part_slots = nslots + 1;
-    L.win = nullptr;
     L.q = q;
     L.q_bf16 = q_dtype == KVQ_BF16;
     L.M = Tk_invT;

@@ -620,19 +620,28 @@ def _round64(x):
     return max(64, (x + 63) // 64 * 64)
 
 
-@pytest.mark.parametrize("ci,S_sink,S_keep,S_flush,seql", [
-    (2, 4, 32, 64, [300, 20, 97]),        # quantized middles; one sequence entirely in the window
-    (2, 0, 0, 64, [256, 128, 64]),        # no window: every position quantized
-    (2, 64, 128, 128, [700, 300, 0]),     # an empty sequence
-    (4, 8, 64, 64, [500, 71]),            # GQA 8, d 64
+@pytest.mark.parametrize("ci,S_sink,S_keep,S_flush,seql,variant", [
+    (2, 4, 32, 64, [300, 20, 97], ""),    # quantized middles; one sequence entirely in the window
+    (2, 0, 0, 64, [256, 128, 64], ""),    # no window: every position quantized
+    (2, 64, 128, 128, [700, 300, 0], ""), # an empty sequence
+    (4, 8, 64, 64, [500, 71], ""),        # GQA 8, d 64
+    # ring slots and sink rows that hold no window position filled with NaN bit patterns:
+    # they must not reach the result
+    (2, 16, 48, 64, [40, 250, 129], "nan"),
+    (3, 16, 64, 64, [400, 150], "nan"),   # 4-bit keys, 2-bit values
+    # identity transforms with no T_v for the window (the window's values are used as given)
+    (2, 4, 32, 64, [300, 97], "ident"),
 ])
-def test_window_decode_matches_oracle(ci, S_sink, S_keep, S_flush, seql):
+def test_window_decode_matches_oracle(ci, S_sink, S_keep, S_flush, seql, variant):
     cfg = synth.CONFIGS[ci]
     B, T = len(seql), _round64(max(seql))
     c = cfg.with_(B=B, T_cap=T)
     k, v = synth.kv_batch(c, 0, T)                       # [B][T][Hkv][d] float32
     kb, vb = synth.as_dtype(k, "bf16"), synth.as_dtype(v, "bf16")
     Tk, Tv, Tit = synth.transforms(cfg)
+    if variant == "ident":
+        Tk = np.broadcast_to(np.eye(cfg.d, dtype=Tk.dtype), Tk.shape).copy()
+        Tv, Tit = Tk.copy(), Tk.copy()
     q = synth.as_dtype(synth.queries(c), "bf16")
     # oracle: every position quantized at its own position; the window decode reads the
     # middle from there and the rest in full precision
@@ -658,10 +667,11 @@ def test_window_decode_matches_oracle(ci, S_sink, S_keep, S_flush, seql):
             dst[b * n:(b + 1) * n] = src
     gc = upload_cache(oc, cfg)
     R = S_keep + S_flush
-    ks = np.zeros((B, cfg.Hkv, max(S_sink, 1), cfg.d), np.uint16)
-    vs = np.zeros_like(ks)
-    kr = np.zeros((B, cfg.Hkv, R, cfg.d), np.uint16)
-    vr = np.zeros_like(kr)
+    fill = 0x7FC1 if variant == "nan" else 0             # a bfloat16 NaN
+    ks = np.full((B, cfg.Hkv, max(S_sink, 1), cfg.d), fill, np.uint16)
+    vs = np.full_like(ks, fill)
+    kr = np.full((B, cfg.Hkv, R, cfg.d), fill, np.uint16)
+    vr = np.full_like(kr, fill)
     for b, L in enumerate(seql):
         for t in range(min(S_sink, L)):
             ks[b, :, t], vs[b, :, t] = kb[b, t], vb[b, t]
@@ -672,11 +682,12 @@ def test_window_decode_matches_oracle(ci, S_sink, S_keep, S_flush, seql):
     ws = torch.empty(kvq.decode_workspace_bytes(gc, cfg.Hq, Tc), dtype=torch.uint8, device=DEV)
     kvq.decode_attention_window(t_(q), t_(Tit), gc, S_sink, S_keep, S_flush,
                                 t_(ks) if S_sink else None, t_(vs) if S_sink else None,
-                                t_(kr), t_(vr), t_(Tv), t_(np.array(seql, np.int32)),
-                                max(seql), out, ws, dev_err=err)
+                                t_(kr), t_(vr), None if variant == "ident" else t_(Tv),
+                                t_(np.array(seql, np.int32)), max(seql), out, ws, dev_err=err)
     torch.cuda.synchronize()
     assert err.item() == 0
     got = out.cpu().numpy()
+    assert np.isfinite(got).all()
     for b, L in enumerate(seql):
         if L == 0:
             assert not got[b].any()
