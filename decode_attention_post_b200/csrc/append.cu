@@ -388,14 +388,21 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
 // ---------------------------------------------------------------- short bf16 appends
 
 // Decode-time appends (a few tokens per sequence, bfloat16, both transforms) and window
-// flushes: 16-token tiles, 8 warps. Warp w computes output dims [w D/8, (w+1) D/8) of the
-// tile on mma.sync (bf16, float32 accumulate): its fragments of T = T_hi + T_lo (two
-// bfloat16 pieces, 16 significant bits) come straight from global memory (L2) into
-// registers once per CTA, so no CTA stages the whole transform in shared memory. The
-// tile's inputs are staged in shared memory (ldmatrix A operands), the transformed tile
-// goes back to shared memory, and each warp quantizes and stores two of its tokens.
-constexpr int kSmallWarps = 8;
+// flushes: 16-token tiles, one warp per 8 output dims (D / 8 warps). Warp w computes output
+// dims [8w, 8w + 8) of the tile on mma.sync (bf16, float32 accumulate): its fragments of
+// T = T_hi + T_lo (two bfloat16 pieces, 16 significant bits) come straight from global
+// memory (L2) into registers once per CTA, so no CTA stages the whole transform in shared
+// memory. The tile's inputs are staged in shared memory by asynchronous copies issued
+// before the transform loads (ldmatrix A operands), the transformed tile goes back to
+// shared memory, and each warp quantizes and stores 16 / (D / 8) of its tokens.
 constexpr int kSmallTile = 16;
+
+template <int D>
+struct SmallCfg {
+    static constexpr int WARPS = D / 8;              // 16 at d = 128, 8 at d = 64
+    static constexpr int TPW = kSmallTile / WARPS;   // tokens each warp quantizes
+    static_assert(kSmallTile % WARPS == 0, "whole tokens per warp");
+};
 
 template <int D>
 struct SmallSmem {
@@ -403,7 +410,7 @@ struct SmallSmem {
     static constexpr int YS = D + 4;                 // float per transformed row
     __nv_bfloat16 X[kSmallTile * XS];
     float Y[kSmallTile * YS];
-    uint8_t codes[kSmallWarps][D];
+    uint8_t codes[SmallCfg<D>::WARPS][D];
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo_elem, float hi_elem)
@@ -418,7 +425,7 @@ __device__ __forceinline__ float bf16_rn(float x)
 }
 
 template <int D>
-__global__ void __launch_bounds__(kSmallWarps * 32)
+__global__ void __launch_bounds__(SmallCfg<D>::WARPS * 32)
 append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 *__restrict__ v_in,
                     const float *__restrict__ Tk, const float *__restrict__ Tv, int B, int n,
                     int Hkv, int T_cap, int bits_k, int bits_v, int group, int kappa,
@@ -426,7 +433,7 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
                     uint8_t *__restrict__ v_codes, uint32_t *__restrict__ v_sz,
                     const int32_t *__restrict__ pos, int32_t *dev_err, PageMap pm, TokenMap tm)
 {
-    constexpr int NTW = D / 64;                      // n-tiles (8 output dims) per warp
+    constexpr int NW = SmallCfg<D>::WARPS, NTW = 1;  // one n-tile (8 output dims) per warp
     constexpr int KS = D / 16;
     using Sm = SmallSmem<D>;
     __shared__ __align__(16) Sm sm;
@@ -479,22 +486,24 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
             if (!tile_active)
                 continue;
         }
-        if (!have_b)
-            load_b();
-        // ---- stage the tile's inputs (16-byte chunks; inactive rows are zero)
-        for (int c = threadIdx.x; c < kSmallTile * (D / 8); c += kSmallWarps * 32) {
+        // ---- stage the tile's inputs (16-byte asynchronous copies; inactive rows are zero),
+        //      issued before the transform fragments so that both loads are in flight
+        for (int c = threadIdx.x; c < kSmallTile * (D / 8); c += NW * 32) {
             const int rr = c / (D / 8), ch = c % (D / 8);
             const long u = u0 + rr;
-            uint4 val = make_uint4(0, 0, 0, 0);
+            const __nv_bfloat16 *src = nullptr;
             if (u < total) {
                 const TokenSlot ts = token_slot(tm, in, which, pos, (int)(u / n), (int)(u % n), n,
                                                 h, Hkv, D, T_cap);
                 if (ts.active)
-                    val = reinterpret_cast<const uint4 *>(
-                        reinterpret_cast<const __nv_bfloat16 *>(ts.base) + ts.src)[ch];
+                    src = reinterpret_cast<const __nv_bfloat16 *>(ts.base) + ts.src + 8 * ch;
             }
-            *reinterpret_cast<uint4 *>(sm.X + rr * Sm::XS + 8 * ch) = val;
+            cp_async16(sm.X + rr * Sm::XS + 8 * ch, src ? (const void *)src : in, src ? 16 : 0);
         }
+        cp_async_commit();
+        if (!have_b)
+            load_b();
+        cp_async_wait<0>();
         __syncthreads();
         // ---- X~ = X . (T_hi + T_lo)^T, this warp's output dims
         float acc[NTW][4];
@@ -521,10 +530,10 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
                 make_float2(acc[nt][2], acc[nt][3]);
         }
         __syncthreads();
-        // ---- quantize and store: warp w takes tokens 2w, 2w+1 of the tile
+        // ---- quantize and store: warp w takes tokens TPW w .. TPW w + TPW - 1 of the tile
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int rr = 2 * warp + q;
+        for (int q = 0; q < SmallCfg<D>::TPW; ++q) {
+            const int rr = SmallCfg<D>::TPW * warp + q;
             const long u = u0 + rr;
             if (u >= total)
                 break;
@@ -571,7 +580,7 @@ cudaError_t launch_append_small(const void *k, const void *v, const float *Tk, c
     if (gx < 1)
         gx = 1;
     dim3 grid((unsigned)gx, (unsigned)c->Hkv, 2);
-    append_small_kernel<D><<<grid, kSmallWarps * 32, 0, st>>>(
+    append_small_kernel<D><<<grid, SmallCfg<D>::WARPS * 32, 0, st>>>(
         (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, Tk, Tv, B, n, c->Hkv, c->T_cap,
         c->qp.bits_k, c->qp.bits_v, c->qp.group, kappa, (uint8_t *)c->k_codes, (uint32_t *)c->k_sz,
         (uint8_t *)c->v_codes, (uint32_t *)c->v_sz, pos, dev_err,
