@@ -12,12 +12,13 @@
 //   3. Per group, the order statistics x_(kappa) and x_(g-1-kappa) come from kappa+1
 //      rounds of a warp-wide min (max) with removal of one instance (exact, ties safe);
 //      for the QuEST INT quantizer, the group RMS from a float64 sum of squares.
-//   4. Scale, zero-point and codes use IEEE float32 division (__fdiv_rn) and rintf
-//      (ties to even), so they match the float64 definition bit for bit.
-//   5. Codes are gathered through shared memory and written as whole 32-bit words
-//      (K rows) or whole 16-bit halves (V tiles); every token owns whole bytes, so
-//      no read-modify-write is needed even for single-token appends. The token slot
-//      comes from the contiguous layout or, for a paged cache, the block table.
+//   4. Scale and zero-point use IEEE float32 division (__fdiv_rn); codes use the
+//      reciprocal with the IEEE quotient near rounding ties, ties to even, so they
+//      match the definition bit for bit.
+//   5. Codes are packed in registers by OR-reductions over lanes and written as whole
+//      32-bit words (K rows) or whole 16-bit halves (V tiles); every token owns whole
+//      bytes, so no read-modify-write is needed even for single-token appends. The
+//      token slot comes from the contiguous layout or, for a paged cache, the block table.
 #include "kvq_common.cuh"
 #include "kvq_ptx.cuh"
 
@@ -37,7 +38,6 @@ struct AppendSmem {
     static constexpr int kTokPerTile = kAppendWarps * TPW;
     float Tt[D * (D + 1)];          // Tt[j*(D+1) + i] = T[i][j]
     float X[kTokPerTile][D];
-    uint8_t codes[kAppendWarps][D];
 };
 
 // kappa+1 rounds of "take the warp-wide extreme and remove one instance".
@@ -137,20 +137,29 @@ __device__ __forceinline__ TokenSlot token_slot(const TokenMap &tm, const void *
 
 // Quantize one token held by a warp (lane l holds dims l + 32 r in vals[r]) and store it
 // at cache row `row`: per group the clip range (order statistics, or the RMS for the QuEST
-// INT quantizer, kappa == kQuestClip), the float16 scale and zero-point, IEEE-exact codes,
-// the K row (whole 32-bit words) or the token's halves of its V tile. `codes` is D bytes
-// of this warp's shared memory.
+// INT quantizer, kappa == kQuestClip), the float16 scale and zero-point, and the codes
+// c = clamp(rint((x - z) / s), 0, qmax) computed as (x - z) * rcp_rn(s), which is within
+// 2 ulp of the IEEE quotient; a value within 2^-20 of a rounding tie takes the IEEE
+// quotient, so the codes are those of the definition bit for bit (rint as a float32 add
+// and subtract of 1.5 * 2^23 on y clamped to [-1, qmax + 1], ties to even). The K row
+// (whole 32-bit words) or the token's halves of its V tile are packed in registers by
+// OR-reductions over the lanes that share a word or half. bits is 2 or 4.
+constexpr float kRoundMagic = 12582912.0f;      // 1.5 * 2^23
+
 template <int D>
 __device__ __forceinline__ void quantize_store_token(const float (&vals)[D / 32], int lane,
-                                                     uint8_t *codes, int which, int bits,
-                                                     int group, int kappa, long long row,
-                                                     uint8_t *k_codes, uint32_t *k_sz,
-                                                     uint8_t *v_codes, uint32_t *v_sz,
-                                                     int32_t *dev_err)
+                                                     int which, int bits, int group, int kappa,
+                                                     long long row, uint8_t *k_codes,
+                                                     uint32_t *k_sz, uint8_t *v_codes,
+                                                     uint32_t *v_sz, int32_t *dev_err)
 {
     constexpr int R = D / 32;
     const int ng = D / group;
     const int qmax = (1 << bits) - 1;
+    uint32_t cq[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+        cq[r] = 0;
     for (int gr = 0; gr < ng; ++gr) {
         // group gr covers dims [gr*group, (gr+1)*group), i.e. r in [r0, r0+nr);
         // dims outside the group are padded with +-inf so they are never picked.
@@ -192,18 +201,22 @@ __device__ __forceinline__ void quantize_store_token(const float (&vals)[D / 32]
         const float sf = __half2float(sh), zf = __half2float(zh);
         if (!finite && lane == 0)
             flag(dev_err, KVQ_DEVERR_NONFINITE);
+        const bool zero = !finite || sf == 0.f;
+        const float rc = zero ? 0.f : __frcp_rn(sf);
+        const float ymax = (float)(qmax + 1);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            if (r < r0 || r >= r0 + nr)
+            if (r < r0 || r >= r0 + nr || zero)
                 continue;
-            int c = 0;
-            if (finite && sf != 0.f) {
-                float y = __fdiv_rn(__fsub_rn(vals[r], zf), sf);
-                float cr = rintf(y);
-                cr = fminf(fmaxf(cr, 0.f), (float)qmax);
-                c = (int)cr;
+            const float dlt = __fsub_rn(vals[r], zf);
+            float y = fminf(fmaxf(__fmul_rn(dlt, rc), -1.f), ymax);
+            float k = __fsub_rn(__fadd_rn(y, kRoundMagic), kRoundMagic);
+            if (fabsf(y - k) >= 0.5f - 9.5367431640625e-07f * fmaxf(fabsf(y), 1.f)) {
+                y = fminf(fmaxf(__fdiv_rn(dlt, sf), -1.f), ymax);
+                k = __fsub_rn(__fadd_rn(y, kRoundMagic), kRoundMagic);
             }
-            codes[lane + 32 * r] = (uint8_t)c;
+            k = fminf(fmaxf(k, 0.f), (float)qmax);
+            cq[r] = (uint32_t)(__float_as_int(__fadd_rn(k, kRoundMagic)) - 0x4B400000);
         }
         if (lane == 0) {
             uint32_t pair = (uint32_t)__half_as_ushort(sh) |
@@ -211,29 +224,58 @@ __device__ __forceinline__ void quantize_store_token(const float (&vals)[D / 32]
             (which ? v_sz : k_sz)[row * ng + gr] = pair;
         }
     }
-    __syncwarp();
     if (!which) {
-        const int words = D * bits / 32, cpw = 32 / bits;
-        if (lane < words) {
-            uint32_t w = 0;
-            for (int e = 0; e < cpw; ++e)
-                w |= (uint32_t)codes[lane * cpw + e] << (bits * e);
-            reinterpret_cast<uint32_t *>(k_codes + row * (D * bits / 8))[lane] = w;
+        // K row: word (32 r + l) / cpw holds lane l's code r at bit bits * (l % cpw)
+        const int cpw = 32 / bits;
+        uint32_t w[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            w[r] = cq[r] << (bits * (lane & (cpw - 1)));
+        for (int off = 1; off < cpw; off <<= 1)
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                w[r] |= __shfl_xor_sync(0xffffffffu, w[r], off);
+        if ((lane & (cpw - 1)) == 0) {
+            uint32_t *dst = reinterpret_cast<uint32_t *>(k_codes + row * (D * bits / 8));
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                dst[r * (32 / cpw) + lane / cpw] = w[r];
         }
     } else {
-        const int E = 16 / bits, halves = D / E;
-        if (lane < halves) {
-            const int gq = lane & 7, r = lane >> 3;
-            uint32_t hv = 0;
-            for (int s2 = 0; s2 < E; ++s2)
-                hv |= (uint32_t)codes[8 * (E * r + s2) + gq] << (bits * s2);
-            const size_t tile_base =
-                (size_t)(row / kTileTokens) * (kTileTokens * D * bits / 8);
-            const int off = v_half_offset(D, bits, (int)(row % kTileTokens), gq, r);
-            *reinterpret_cast<uint16_t *>(v_codes + tile_base + off) = (uint16_t)hv;
+        // V tile half (gq, rr) holds dims gq + 8 (E rr + s2), s2 < E = 16 / bits: lane l's
+        // code r is dim l + 32 r, i.e. gq = l % 8, E rr + s2 = 4 r + l / 8, so rr = r / 2
+        // (2-bit) or r (4-bit); OR-reduced over the lanes with the same gq
+        uint32_t hv[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            hv[r] = 0;
+        if (bits == 2) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                hv[r >> 1] |= cq[r] << (2 * (4 * (r & 1) + (lane >> 3)));
+        } else {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                hv[r] = cq[r] << (4 * (lane >> 3));
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            hv[r] |= __shfl_xor_sync(0xffffffffu, hv[r], 8);
+            hv[r] |= __shfl_xor_sync(0xffffffffu, hv[r], 16);
+        }
+        if (lane < 8) {
+            const int W = D * bits / 128;                // halves per gq: D / (8 E)
+            unsigned char *tile_base =
+                v_codes + (size_t)(row / kTileTokens) * (kTileTokens * D * bits / 8);
+            const int tok = (int)(row % kTileTokens);
+#pragma unroll
+            for (int rr = 0; rr < R; ++rr)
+                if (rr < W)
+                    *reinterpret_cast<uint16_t *>(tile_base +
+                                                  v_half_offset(D, bits, tok, lane, rr)) =
+                        (uint16_t)hv[rr];
         }
     }
-    __syncwarp();
 }
 
 template <int D, int TPW>
@@ -379,7 +421,7 @@ append_fp32_kernel(const void *__restrict__ k_in, const void *__restrict__ v_in,
                     flag(dev_err, KVQ_DEVERR_PAGE_RANGE);
                 continue;
             }
-            quantize_store_token<D>(acc[q], lane, sm.codes[warp], which, bits, group, kappa, row,
+            quantize_store_token<D>(acc[q], lane, which, bits, group, kappa, row,
                                     k_codes, k_sz, v_codes, v_sz, dev_err);
         }
     }
@@ -410,19 +452,7 @@ struct SmallSmem {
     static constexpr int YS = D + 4;                 // float per transformed row
     __nv_bfloat16 X[kSmallTile * XS];
     float Y[kSmallTile * YS];
-    uint8_t codes[SmallCfg<D>::WARPS][D];
 };
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo_elem, float hi_elem)
-{
-    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo_elem)) |
-           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi_elem)) << 16);
-}
-
-__device__ __forceinline__ float bf16_rn(float x)
-{
-    return __bfloat162float(__float2bfloat16_rn(x));
-}
 
 template <int D>
 __global__ void __launch_bounds__(SmallCfg<D>::WARPS * 32)
@@ -459,9 +489,11 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     const float2 f = *reinterpret_cast<const float2 *>(row + 16 * ks + 8 * half + 2 * t);
-                    const float h0 = bf16_rn(f.x), h1 = bf16_rn(f.y);
-                    bhi[nt][ks][half] = pack_bf16x2(f.x, f.y);
-                    blo[nt][ks][half] = pack_bf16x2(f.x - h0, f.y - h1);
+                    const __nv_bfloat162 hi2 = __floats2bfloat162_rn(f.x, f.y);
+                    const float2 hf = __bfloat1622float2(hi2);
+                    const __nv_bfloat162 lo2 = __floats2bfloat162_rn(f.x - hf.x, f.y - hf.y);
+                    bhi[nt][ks][half] = *reinterpret_cast<const uint32_t *>(&hi2);
+                    blo[nt][ks][half] = *reinterpret_cast<const uint32_t *>(&lo2);
                 }
         }
         have_b = true;
@@ -556,7 +588,7 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
 #pragma unroll
             for (int r = 0; r < D / 32; ++r)
                 vals[r] = sm.Y[rr * Sm::YS + lane + 32 * r];
-            quantize_store_token<D>(vals, lane, sm.codes[warp], which, bits, group, kappa, row,
+            quantize_store_token<D>(vals, lane, which, bits, group, kappa, row,
                                     k_codes, k_sz, v_codes, v_sz, dev_err);
         }
     }
