@@ -36,7 +36,7 @@ METRIC = "2-bit KV decode attention: achieved HBM GB/s and % of B200 peak; appen
 CONFIG_IDX = 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one decode_kernel launch on this workload
 # (ncu --set full --clock-control none, profiles directory); None once the kernel changes.
-DECODE_TRAFFIC_BYTES = None
+DECODE_TRAFFIC_BYTES = 546806272
 DECODE_TRAFFIC_KERNEL = "decode_kernel<128,4,2,2>"
 APPEND_CONFIG_IDX = 4
 DECODE_CONFIGS = (1, 3, 4)       # further decode shapes timed as extras
@@ -258,14 +258,26 @@ class E2EStep:
                              dev_err=w.err)
         self.out_h.copy_(w.out, non_blocking=True)
 
-    def time(self, iters, stream, barrier):
+    def copies(self):
+        """The step's host<->device copies alone, in the same streams and order."""
         import torch
+        main = torch.cuda.current_stream()
+        self.app_d.copy_(self.app_h, non_blocking=True)
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            self.dec_d.copy_(self.dec_h, non_blocking=True)
+        main.wait_stream(self.side)
+        self.out_h.copy_(self.w.out, non_blocking=True)
+
+    def time(self, iters, stream, barrier, fn=None):
+        import torch
+        fn = fn or self.step
         for _ in range(3):
-            self.step()
+            fn()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            self.step()
+            fn()
         for _ in range(3):
             g.replay()
         torch.cuda.synchronize()
@@ -379,6 +391,7 @@ def run_gpu(args):
     #      the whole sequence is replayed as a CUDA graph
     e2e = E2EStep(w)
     e2e_ms = max_over_ranks(e2e.time(min(K, 500), stream, barrier))
+    copies_ms = max_over_ranks(e2e.time(min(K, 500), stream, barrier, fn=e2e.copies))
     e2e_value = weak_scaling_gbs(dec_bytes + app_bytes, e2e_ms, world)
     h2d, d2h = e2e.h2d_bytes, e2e.d2h_bytes
 
@@ -404,6 +417,7 @@ def run_gpu(args):
                                "append_tok_per_s": round(cfg.B / (app_ms * 1e-3), 1)},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "copies_only_ms": round(copies_ms, 5),
                 "how": "pinned staging buffers: H2D of the append inputs, then append while "
                        "q and seqlens copy on a second stream, decode, D2H of the output; "
                        "replayed as a CUDA graph"},

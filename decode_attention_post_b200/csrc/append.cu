@@ -475,8 +475,10 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
     const int bits = which ? bits_v : bits_k;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const long total = (long)B * n;
-    const long tiles = (total + kSmallTile - 1) / kSmallTile;
+    // B * n < 2^29 on every path here (short appends, bounded window flushes): 32-bit
+    // token indices, so the divisions by n stay 32-bit
+    const int total = B * n;
+    const int tiles = (total + kSmallTile - 1) / kSmallTile;
 
     uint32_t bhi[NTW][KS][2], blo[NTW][KS][2];
     bool have_b = false;
@@ -499,8 +501,8 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
         have_b = true;
     };
 
-    for (long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-        const long u0 = tile * kSmallTile;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        const int u0 = tile * kSmallTile;
         __syncthreads();                             // the previous tile's readers are done
         if (tm.ring_k) {
             // window flush: skip tiles without a token to write (most of a decode step)
@@ -508,8 +510,8 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
                 tile_active = 0;
             __syncthreads();
             if (threadIdx.x < kSmallTile && u0 + threadIdx.x < total) {
-                const long u = u0 + threadIdx.x;
-                const TokenSlot ts = token_slot(tm, in, which, pos, (int)(u / n), (int)(u % n), n,
+                const int u = u0 + (int)threadIdx.x;
+                const TokenSlot ts = token_slot(tm, in, which, pos, u / n, u % n, n,
                                                 h, Hkv, D, T_cap);
                 if (ts.active || (ts.bad_range && ts.first))
                     tile_active = 1;
@@ -522,10 +524,10 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
         //      issued before the transform fragments so that both loads are in flight
         for (int c = threadIdx.x; c < kSmallTile * (D / 8); c += NW * 32) {
             const int rr = c / (D / 8), ch = c % (D / 8);
-            const long u = u0 + rr;
+            const int u = u0 + rr;
             const __nv_bfloat16 *src = nullptr;
             if (u < total) {
-                const TokenSlot ts = token_slot(tm, in, which, pos, (int)(u / n), (int)(u % n), n,
+                const TokenSlot ts = token_slot(tm, in, which, pos, u / n, u % n, n,
                                                 h, Hkv, D, T_cap);
                 if (ts.active)
                     src = reinterpret_cast<const __nv_bfloat16 *>(ts.base) + ts.src + 8 * ch;
@@ -566,10 +568,10 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ k_in, const __nv_bfloat16 
 #pragma unroll
         for (int q = 0; q < SmallCfg<D>::TPW; ++q) {
             const int rr = SmallCfg<D>::TPW * warp + q;
-            const long u = u0 + rr;
+            const int u = u0 + rr;
             if (u >= total)
                 break;
-            const int b = (int)(u / n), i = (int)(u % n);
+            const int b = u / n, i = u % n;
             const TokenSlot ts = token_slot(tm, in, which, pos, b, i, n, h, Hkv, D, T_cap);
             if (ts.bad_range) {
                 if (ts.first && lane == 0)
