@@ -38,27 +38,32 @@ namespace kvq {
 namespace {
 
 constexpr int kTcTile = 128;                       // tokens per tile (MMA M)
-constexpr int kTcEpiGroups = 2;                    // epilogue warpgroups, one per accumulator
-constexpr int kTcEpiWarps = 4 * kTcEpiGroups;
-constexpr int kTcThreads = (kTcEpiWarps + 2) * 32; // epilogue warps + TMA warp + MMA warp
-constexpr int kTcStages = 3;
 constexpr int kTcKBlock = 64;                      // bf16 per 128-byte swizzled row
 
 template <int D>
 struct TcCfg {
+    // epilogue warpgroups, one TMEM accumulator buffer each: at d = 64 four, so that one
+    // CTA per SM keeps 16 epilogue warps with the register budget to hold a whole row
+    static constexpr int EPI = D == 64 ? 4 : 2;
+    static constexpr int EPI_WARPS = 4 * EPI;
+    static constexpr int THREADS = (EPI_WARPS + 2) * 32;      // + TMA warp + MMA warp
+    static constexpr int STAGES = D == 64 ? 4 : 3;            // input tile ring
     static constexpr int KB = D / kTcKBlock;                  // 128-byte K blocks
     static constexpr int A_BLOCK = kTcTile * kTcKBlock * 2;   // 16 KB: one K block of a tile
     static constexpr int A_BYTES = KB * A_BLOCK;              // one input stage
     static constexpr int B_BLOCK = D * kTcKBlock * 2;         // one K block of T_hi or T_lo
     static constexpr int B_BYTES = KB * B_BLOCK;
-    static constexpr int OFF_B_HI = kTcStages * A_BYTES;
+    static constexpr int OFF_B_HI = STAGES * A_BYTES;
     static constexpr int OFF_B_LO = OFF_B_HI + B_BYTES;
     static constexpr int OFF_BAR = OFF_B_LO + B_BYTES;
-    static constexpr int SMEM = OFF_BAR + 128 + 1024;         // barriers + alignment slack
-    static constexpr int TMEM_COLS = 2 * D;                   // two accumulator buffers
-    // CTAs per SM: shared memory allows it, TMEM (512 columns) and registers must too
-    static constexpr int PER_SM = D == 64 ? 2 : 1;
-    static_assert(PER_SM * TMEM_COLS <= 512, "TMEM oversubscribed");
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;         // barriers + alignment slack
+    static constexpr int TMEM_COLS = EPI * D;                 // the accumulator buffers
+    static constexpr int PER_SM = 1;
+    // registers per thread: the most that THREADS threads get from the SM's 64K in
+    // whole 8-register steps (d = 64: 576 threads, 112 registers)
+    static constexpr int MAXREG = ((65536 / THREADS) / 8) * 8 > 255 ? 255 : ((65536 / THREADS) / 8) * 8;
+    static_assert(TMEM_COLS == 256, "TMEM allocation: a power of two of at most 512 columns");
+    static_assert((2 * STAGES + 2 * EPI) * 8 + 8 <= 256, "barrier area");
     static_assert(PER_SM * (SMEM + 1024) <= 228 * 1024, "shared memory oversubscribed");
 };
 
@@ -90,14 +95,14 @@ constexpr float kRoundMagic = 12582912.0f;        // 1.5 * 2^23
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 constexpr float kTieBand = 0.5f - 1.52587890625e-05f;   // 0.5 - 2^-16
 
-// bit pattern 0x4B400000 + c of the rounded value
-__device__ __forceinline__ uint32_t code_bits(float x, float zf, float rc, float qmax, bool &tie)
+// bit pattern 0x4B400000 + c of the rounded value; tmax keeps the largest distance of a
+// quotient from its rounded value (a row with tmax >= kTieBand is near a rounding tie)
+__device__ __forceinline__ uint32_t code_bits(float x, float zf, float rc, float qmax, float &tmax)
 {
     float y = __fmul_rn(__fsub_rn(x, zf), rc);
     y = fminf(fmaxf(y, 0.f), qmax);
     const float r = __fadd_rn(y, kRoundMagic);
-    const float t = __fsub_rn(y, __fsub_rn(r, kRoundMagic));
-    tie |= fabsf(t) >= kTieBand;
+    tmax = fmaxf(tmax, fabsf(__fsub_rn(y, __fsub_rn(r, kRoundMagic))));
     return __float_as_uint(r);
 }
 
@@ -108,6 +113,17 @@ __device__ __forceinline__ uint32_t code_exact(float x, float zf, float sf, bool
         return 0u;
     const float k = rintf(__fdiv_rn(__fsub_rn(x, zf), sf));
     return (uint32_t)fminf(fmaxf(k, 0.f), qmax);
+}
+
+// code of one value: magic-rounded bits (EXACT = false) or the IEEE-division code
+template <bool EXACT>
+__device__ __forceinline__ uint32_t code_of(uint32_t xb, float zf, float sf, float rc, bool zero,
+                                            float qmax, float &tmax)
+{
+    if constexpr (EXACT)
+        return code_exact(__uint_as_float(xb), zf, sf, zero, qmax);
+    else
+        return code_bits(__uint_as_float(xb), zf, rc, qmax, tmax);
 }
 
 // sum over e < N of 0x4B400000 * 2^(B*e), modulo 2^32: what packing N magic-rounded codes
@@ -178,7 +194,7 @@ __device__ __forceinline__ bool pickb(const bool (&a)[NG], int gr)
 // reciprocal codes (sets tie near a rounding tie); exact = true: IEEE division.
 template <int BITS, bool EXACT>
 __device__ __forceinline__ void pack32(const uint32_t (&x)[32], float zf, float sf, float rc,
-                                       bool zero, float qmax, bool &tie, uint32_t (&w)[BITS])
+                                       bool zero, float qmax, float &tie, uint32_t (&w)[BITS])
 {
     constexpr bool exact = EXACT;
     constexpr int PER = 32 / BITS;                  // codes per word
@@ -188,8 +204,7 @@ __device__ __forceinline__ void pack32(const uint32_t (&x)[32], float zf, float 
 #pragma unroll
         for (int e = 0; e < PER; ++e) {
             const float v = __uint_as_float(x[PER * q + e]);
-            acc += (exact ? code_exact(v, zf, sf, zero, qmax) : code_bits(v, zf, rc, qmax, tie))
-                   << (BITS * e);
+            acc += code_of<EXACT>(__float_as_uint(v), zf, sf, rc, zero, qmax, tie) << (BITS * e);
         }
         w[q] = acc;
     }
@@ -208,7 +223,7 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
 {
     constexpr bool exact = EXACT;
     constexpr int NCH = D / 32;
-    bool tie = false;
+    float tie = 0.f;
     uint32_t cur[32];
     tmem_ld32_async(taddr, cur);
     tmem_ld_wait();
@@ -248,7 +263,7 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
 #pragma unroll
                 for (int n8 = 0; n8 < 4; ++n8) {
                     const float v = __uint_as_float(cur[8 * n8 + gq]);
-                    acc += (exact ? code_exact(v, z, s, zr, qmax) : code_bits(v, z, r, qmax, tie))
+                    acc += code_of<EXACT>(__float_as_uint(v), z, s, r, zr, qmax, tie)
                            << (BITS * (base + n8));
                 }
                 hv[gq] = acc;
@@ -266,11 +281,160 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
             }
         }
     }
-    return tie;
+    return tie >= kTieBand;
 }
 
+// d = 64: the token's whole row x0 (dims 0-31), x1 (dims 32-63) is in registers. Codes
+// with the group parameters of each half (p0: dims 0-31, p1: dims 32-63), stored as the
+// K row (one or two 16-byte stores) or as the token's halves of its V tile (whole 16-bit
+// halves: half (gq, rr) holds dims 8(E rr + s) + gq at BITS*s, E = 16/BITS). row < 0:
+// nothing stored. Returns whether a value was within the tie band.
+template <int BITS, bool EXACT>
+__device__ __forceinline__ bool store_row64(const TcParams &P, int which, long long row,
+                                            const uint32_t (&x0)[32], const uint32_t (&x1)[32],
+                                            const float (&z)[2], const float (&sc)[2],
+                                            const float (&rc)[2], const bool (&zr)[2], float qmax)
+{
+    float tmax = 0.f;
+    if (!which) {
+        uint32_t w0[BITS], w1[BITS];
+        pack32<BITS, EXACT>(x0, z[0], sc[0], rc[0], zr[0], qmax, tmax, w0);
+        pack32<BITS, EXACT>(x1, z[1], sc[1], rc[1], zr[1], qmax, tmax, w1);
+        if (row >= 0) {
+            uint4 *dst = reinterpret_cast<uint4 *>(P.k_codes + row * (64 * BITS / 8));
+            if constexpr (BITS == 2) {
+                dst[0] = make_uint4(w0[0], w0[1 % BITS], w1[0], w1[1 % BITS]);
+            } else {
+                dst[0] = make_uint4(w0[0], w0[1 % BITS], w0[2 % BITS], w0[3 % BITS]);
+                dst[1] = make_uint4(w1[0], w1[1 % BITS], w1[2 % BITS], w1[3 % BITS]);
+            }
+        }
+    } else {
+        unsigned char *vbase = nullptr;
+        int tok = 0;
+        if (row >= 0) {
+            vbase = P.v_codes + (size_t)(row / kTileTokens) * (kTileTokens * 64 * BITS / 8);
+            tok = (int)(row % kTileTokens);
+        }
+#pragma unroll
+        for (int gq = 0; gq < 8; ++gq) {
+            if constexpr (BITS == 2) {
+                // one half per gq: s < 4 from x0 (dim gq + 8 s), s >= 4 from x1
+                uint32_t acc = EXACT ? 0u : 0u - magic_sum(2, 8);
+#pragma unroll
+                for (int s2 = 0; s2 < 4; ++s2) {
+                    acc += code_of<EXACT>(x0[8 * s2 + gq], z[0], sc[0], rc[0], zr[0], qmax, tmax)
+                           << (2 * s2);
+                    acc += code_of<EXACT>(x1[8 * s2 + gq], z[1], sc[1], rc[1], zr[1], qmax, tmax)
+                           << (2 * (4 + s2));
+                }
+                if (row >= 0)
+                    *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 2, tok, gq, 0)) =
+                        (uint16_t)acc;
+            } else {
+                // halves rr = 0 (x0) and rr = 1 (x1), s < 4: dim gq + 8 (4 rr + s)
+                uint32_t a0 = EXACT ? 0u : 0u - magic_sum(4, 4), a1 = a0;
+#pragma unroll
+                for (int s2 = 0; s2 < 4; ++s2) {
+                    a0 += code_of<EXACT>(x0[8 * s2 + gq], z[0], sc[0], rc[0], zr[0], qmax, tmax)
+                          << (4 * s2);
+                    a1 += code_of<EXACT>(x1[8 * s2 + gq], z[1], sc[1], rc[1], zr[1], qmax, tmax)
+                          << (4 * s2);
+                }
+                if (row >= 0) {
+                    *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 4, tok, gq, 0)) =
+                        (uint16_t)a0;
+                    *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 4, tok, gq, 1)) =
+                        (uint16_t)a1;
+                }
+            }
+        }
+    }
+    return tmax >= kTieBand;
+}
+
+// Running clip statistics of one group of a row: kappa = 0 (min, max), kappa = 1 (second
+// smallest and largest), kappa <= 8 (the 9 smallest and largest by insertion), or the
+// QuEST INT sum of squares (float64, each square exact).
+struct ClipStats {
+    float lo, hi, m1, m2, M1, M2, sm9[9], lg9[9];
+    double ss;
+
+    __device__ __forceinline__ void reset()
+    {
+        lo = m1 = m2 = INFINITY;
+        hi = M1 = M2 = -INFINITY;
+        ss = 0.0;
+#pragma unroll
+        for (int e = 0; e < 9; ++e) {
+            sm9[e] = INFINITY;
+            lg9[e] = -INFINITY;
+        }
+    }
+
+    __device__ __forceinline__ void add32(const uint32_t (&cur)[32], int clip, bool quest)
+    {
+        if (quest) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const double v = (double)__uint_as_float(cur[j]);
+                ss = fma(v, v, ss);
+            }
+        } else if (clip == 0) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                lo = fmin3(lo, __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+                hi = fmax3(hi, __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+            }
+        } else if (clip == 1) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float v = __uint_as_float(cur[j]);
+                m2 = fminf(m2, fmaxf(m1, v));
+                m1 = fminf(m1, v);
+                M2 = fmaxf(M2, fminf(M1, v));
+                M1 = fmaxf(M1, v);
+            }
+        } else {
+#pragma unroll 4
+            for (int j = 0; j < 32; ++j) {
+                float av = __uint_as_float(cur[j]), bv = av;
+#pragma unroll
+                for (int e = 0; e < 9; ++e) {
+                    const float s0 = fminf(sm9[e], av), s1 = fmaxf(sm9[e], av);
+                    sm9[e] = s0;
+                    av = s1;
+                    const float l0 = fmaxf(lg9[e], bv), l1 = fminf(lg9[e], bv);
+                    lg9[e] = l0;
+                    bv = l1;
+                }
+            }
+        }
+    }
+
+    // the clip range [x_(kappa), x_(g-1-kappa)] of the values added
+    __device__ __forceinline__ void range(int clip, float &glo, float &ghi) const
+    {
+        glo = lo;
+        ghi = hi;
+        if (clip == 1) {
+            glo = m2;
+            ghi = M2;
+        } else if (clip > 1) {
+            glo = sm9[0];
+            ghi = lg9[0];
+#pragma unroll
+            for (int e = 1; e < 9; ++e)
+                if (e == clip) {
+                    glo = sm9[e];
+                    ghi = lg9[e];
+                }
+        }
+    }
+};
+
 template <int D, int GS>
-__global__ void __launch_bounds__(kTcThreads, TcCfg<D>::PER_SM)
+__global__ void __launch_bounds__(TcCfg<D>::THREADS) __maxnreg__(TcCfg<D>::MAXREG)
 append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  TcParams P)
 {
@@ -280,10 +444,10 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *empty = full + kTcStages;
-    uint64_t *accf = empty + kTcStages;
-    uint64_t *acce = accf + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *accf = empty + C::STAGES;
+    uint64_t *acce = accf + C::EPI;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + C::EPI);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int h = blockIdx.y, which = blockIdx.z;
@@ -297,11 +461,11 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTcStages; ++s) {
+        for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < C::EPI; ++a) {
             mbar_init(&accf[a], 1);
             mbar_init(&acce[a], 128);                  // one epilogue warpgroup
         }
@@ -314,7 +478,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // ---- T_h -> bf16 (hi, lo) in the K-major 128-byte-swizzled layout: row i (output dim)
     //      of K block kb at kb*B_BLOCK + (i/8)*1024 + (i%8)*128, 16-byte chunk c of the row
     //      at position c ^ (i % 8)
-    for (int c = threadIdx.x; c < D * D / 8; c += kTcThreads) {
+    for (int c = threadIdx.x; c < D * D / 8; c += C::THREADS) {
         const int i = c / (D / 8), j0 = 8 * (c % (D / 8));
         const float4 *src = reinterpret_cast<const float4 *>(T + ((size_t)h * D + i) * D + j0);
         const float4 f0 = src[0], f1 = src[1];
@@ -341,13 +505,13 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const uint32_t tmem_base = *tmem_slot;
 
     int issued = 0, consumed = 0;       // TMA lane: tiles loaded; MMA lane: tiles multiplied
-    if (warp == kTcEpiWarps) {
+    if (warp == C::EPI_WARPS) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(tmap);
             for (int k = 0; k < my_tiles && !*abort_flag; ++k) {
-                const int s = k % kTcStages;
-                if (!mbar_wait_bounded(&empty[s], ((k / kTcStages) & 1) ^ 1)) {
+                const int s = k % C::STAGES;
+                if (!mbar_wait_bounded(&empty[s], ((k / C::STAGES) & 1) ^ 1)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -360,14 +524,14 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 issued = k + 1;
             }
         }
-    } else if (warp == kTcEpiWarps + 1) {
+    } else if (warp == C::EPI_WARPS + 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_bf16_f32(kTcTile, D);
             for (int k = 0; k < my_tiles && !*abort_flag; ++k) {
-                const int s = k % kTcStages, a = k & 1;
-                if (!mbar_wait_bounded(&acce[a], ((k >> 1) & 1) ^ 1) ||
-                    !mbar_wait_bounded(&full[s], (k / kTcStages) & 1)) {
+                const int s = k % C::STAGES, a = k % C::EPI;
+                if (!mbar_wait_bounded(&acce[a], ((k / C::EPI) & 1) ^ 1) ||
+                    !mbar_wait_bounded(&full[s], (k / C::STAGES) & 1)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -392,18 +556,18 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Warpgroup wg takes the tiles k = wg, wg + 2, ... (accumulator buffer wg); thread r
-        // of warp quarter q owns TMEM lane (token row) 32 q + r. Two passes over the row,
-        // 32 columns at a time: the clip parameters of every group, then the codes. The
-        // buffer is released after the row is done, so a row near a rounding tie can be
-        // reloaded and recoded with IEEE division.
+        // Warpgroup wg takes the tiles k = wg, wg + EPI, ... (accumulator buffer wg); thread
+        // r of warp quarter q owns TMEM lane (token row) 32 q + r. Two passes over the row:
+        // the clip parameters of every group, then the codes (d = 64: the whole row held in
+        // registers; d = 128: 32 columns at a time from TMEM). The buffer is released after
+        // the row is done, so a row near a rounding tie can be recoded with IEEE division.
         const int wg = warp / 4, quarter = warp % 4;
         const int r = quarter * 32 + lane;
         const float qmax = (float)((1u << bits) - 1u);
         const bool quest = P.clip == kQuestClip;
-        for (int k = wg; k < my_tiles; k += kTcEpiGroups) {
-            const int a = k & 1;
-            if (*abort_flag || !mbar_wait_bounded(&accf[a], (k >> 1) & 1)) {
+        for (int k = wg; k < my_tiles; k += C::EPI) {
+            const int a = k % C::EPI;
+            if (*abort_flag || !mbar_wait_bounded(&accf[a], (k / C::EPI) & 1)) {
                 *abort_flag = 1;
                 break;
             }
@@ -434,140 +598,102 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 zf[gg] = sf[gg] = rc[gg] = 0.f;
                 zero[gg] = true;
             }
-            {
-                uint32_t cur[32];
-                float lo = INFINITY, hi = -INFINITY;
-                float m1 = INFINITY, m2 = INFINITY, M1 = -INFINITY, M2 = -INFINITY;
-                float sm9[9], lg9[9];
-#pragma unroll
-                for (int e = 0; e < 9; ++e) {
-                    sm9[e] = INFINITY;
-                    lg9[e] = -INFINITY;
+            ClipStats cs;
+            cs.reset();
+            // group gr is complete: its scale and zero-point, stored with the row
+            auto finish = [&](int gr) {
+                __half sh, zh;
+                bool finite;
+                if (quest) {
+                    const float rms = __double2float_rn(sqrt(cs.ss / (double)GS));
+                    const float sv = __fmul_rn(rms, quest_delta(bits));
+                    sh = __float2half_rn(sv);
+                    zh = __float2half_rn(__fmul_rn(-0.5f * qmax, __half2float(sh)));
+                    finite = isfinite(sv);
+                } else {
+                    float glo, ghi;
+                    cs.range(P.clip, glo, ghi);
+                    const float range = __fsub_rn(ghi, glo);
+                    const float sv = __fdiv_rn(range, qmax);
+                    sh = __float2half_rn(sv);
+                    zh = __float2half_rn(glo);
+                    finite = isfinite(range) && isfinite(sv);
                 }
-                double ss = 0.0;
+                const float sfv = __half2float(sh), zfv = __half2float(zh);
+                const bool zr = !finite || sfv == 0.f;
+                const float rcv = zr ? 0.f : __frcp_rn(sfv);
+#pragma unroll
+                for (int gg = 0; gg < NG; ++gg)
+                    if (gg == gr) {
+                        sf[gg] = sfv;
+                        zf[gg] = zfv;
+                        zero[gg] = zr;
+                        rc[gg] = rcv;
+                    }
+                if (row >= 0) {
+                    if (!finite)
+                        flag(P.dev_err, KVQ_DEVERR_NONFINITE);
+                    (which ? P.v_sz : P.k_sz)[row * NG + gr] =
+                        (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
+                }
+                cs.reset();                                 // the next group starts fresh
+            };
+            if constexpr (D == 64) {
+                // the whole row in registers: one TMEM round trip, both passes (and the
+                // exact redo of a row near a tie) from registers
+                uint32_t x0[32], x1[32];
+                tmem_ld32_async(taddr, x0);
+                tmem_ld32_async(taddr + 32, x1);
+                tmem_ld_wait();
+                cs.add32(x0, P.clip, quest);
+                if (GS == 32)
+                    finish(0);
+                cs.add32(x1, P.clip, quest);
+                finish(NG - 1);
+                const float z2[2] = {zf[0], zf[NG - 1]}, s2[2] = {sf[0], sf[NG - 1]};
+                const float r2[2] = {rc[0], rc[NG - 1]};
+                const bool zr2[2] = {zero[0], zero[NG - 1]};
+                bool tie = bits == 2
+                               ? store_row64<2, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax)
+                               : store_row64<4, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                if (tie && row >= 0) {
+                    if (bits == 2)
+                        store_row64<2, true>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                    else
+                        store_row64<4, true>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                }
+            } else {
+                uint32_t cur[32];
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     tmem_ld32_async(taddr + 32 * c, cur);
                     tmem_ld_wait();
-                    if (quest) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const double v = (double)__uint_as_float(cur[j]);
-                            ss = fma(v, v, ss);
-                        }
-                    } else if (P.clip == 0) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            lo = fmin3(lo, __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
-                            hi = fmax3(hi, __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
-                        }
-                    } else if (P.clip == 1) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float v = __uint_as_float(cur[j]);
-                            m2 = fminf(m2, fmaxf(m1, v));
-                            m1 = fminf(m1, v);
-                            M2 = fmaxf(M2, fminf(M1, v));
-                            M1 = fmaxf(M1, v);
-                        }
-                    } else {
-                        // kappa <= 8: the 9 smallest and 9 largest by insertion
-#pragma unroll 4
-                        for (int j = 0; j < 32; ++j) {
-                            float av = __uint_as_float(cur[j]), bv = av;
-#pragma unroll
-                            for (int e = 0; e < 9; ++e) {
-                                const float s0 = fminf(sm9[e], av), s1 = fmaxf(sm9[e], av);
-                                sm9[e] = s0;
-                                av = s1;
-                                const float l0 = fmaxf(lg9[e], bv), l1 = fminf(lg9[e], bv);
-                                lg9[e] = l0;
-                                bv = l1;
-                            }
-                        }
-                    }
-                    if ((32 * c + 32) % GS == 0) {          // the group ends with this chunk
-                        const int gr = (32 * c) / GS;
-                        __half sh, zh;
-                        bool finite;
-                        if (quest) {
-                            const float rms = __double2float_rn(sqrt(ss / (double)GS));
-                            const float s = __fmul_rn(rms, quest_delta(bits));
-                            sh = __float2half_rn(s);
-                            zh = __float2half_rn(__fmul_rn(-0.5f * qmax, __half2float(sh)));
-                            finite = isfinite(s);
-                        } else {
-                            float glo = lo, ghi = hi;
-                            if (P.clip == 1) {
-                                glo = m2;
-                                ghi = M2;
-                            } else if (P.clip > 1) {
-                                glo = sm9[0];
-                                ghi = lg9[0];
-#pragma unroll
-                                for (int e = 1; e < 9; ++e)
-                                    if (e == P.clip) {
-                                        glo = sm9[e];
-                                        ghi = lg9[e];
-                                    }
-                            }
-                            const float range = __fsub_rn(ghi, glo);
-                            const float s = __fdiv_rn(range, qmax);
-                            sh = __float2half_rn(s);
-                            zh = __float2half_rn(glo);
-                            finite = isfinite(range) && isfinite(s);
-                        }
-                        const float sfv = __half2float(sh), zfv = __half2float(zh);
-                        const bool zr = !finite || sfv == 0.f;
-                        const float rcv = zr ? 0.f : __frcp_rn(sfv);
-#pragma unroll
-                        for (int gg = 0; gg < NG; ++gg)
-                            if (gg == gr) {
-                                sf[gg] = sfv;
-                                zf[gg] = zfv;
-                                zero[gg] = zr;
-                                rc[gg] = rcv;
-                            }
-                        if (row >= 0) {
-                            if (!finite)
-                                flag(P.dev_err, KVQ_DEVERR_NONFINITE);
-                            (which ? P.v_sz : P.k_sz)[row * NG + gr] =
-                                (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
-                        }
-                        // the next group starts fresh
-                        lo = INFINITY;
-                        hi = -INFINITY;
-                        m1 = m2 = INFINITY;
-                        M1 = M2 = -INFINITY;
-                        ss = 0.0;
-#pragma unroll
-                        for (int e = 0; e < 9; ++e) {
-                            sm9[e] = INFINITY;
-                            lg9[e] = -INFINITY;
-                        }
-                    }
+                    cs.add32(cur, P.clip, quest);
+                    if ((32 * c + 32) % GS == 0)          // the group ends with this chunk
+                        finish((32 * c) / GS);
                 }
-            }
-            // ---- pass 2: codes; pass 3 (rows near a rounding tie only): the same by division
-            bool tie;
-            if (!which)
-                tie = bits == 2 ? store_codes<D, GS, NG, 2, false, false>(P, row, taddr, zf, sf, rc, zero, qmax)
-                                : store_codes<D, GS, NG, 4, false, false>(P, row, taddr, zf, sf, rc, zero, qmax);
-            else
-                tie = bits == 2 ? store_codes<D, GS, NG, 2, true, false>(P, row, taddr, zf, sf, rc, zero, qmax)
-                                : store_codes<D, GS, NG, 4, true, false>(P, row, taddr, zf, sf, rc, zero, qmax);
-            if (__any_sync(0xffffffffu, tie)) {
-                const long long rw = tie ? row : -1;
-                if (!which) {
-                    if (bits == 2)
-                        store_codes<D, GS, NG, 2, false, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
-                    else
-                        store_codes<D, GS, NG, 4, false, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
-                } else {
-                    if (bits == 2)
-                        store_codes<D, GS, NG, 2, true, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
-                    else
-                        store_codes<D, GS, NG, 4, true, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
+                // ---- pass 2: codes; pass 3 (rows near a rounding tie only): the same by
+                //      division
+                bool tie;
+                if (!which)
+                    tie = bits == 2 ? store_codes<D, GS, NG, 2, false, false>(P, row, taddr, zf, sf, rc, zero, qmax)
+                                    : store_codes<D, GS, NG, 4, false, false>(P, row, taddr, zf, sf, rc, zero, qmax);
+                else
+                    tie = bits == 2 ? store_codes<D, GS, NG, 2, true, false>(P, row, taddr, zf, sf, rc, zero, qmax)
+                                    : store_codes<D, GS, NG, 4, true, false>(P, row, taddr, zf, sf, rc, zero, qmax);
+                if (__any_sync(0xffffffffu, tie)) {
+                    const long long rw = tie ? row : -1;
+                    if (!which) {
+                        if (bits == 2)
+                            store_codes<D, GS, NG, 2, false, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
+                        else
+                            store_codes<D, GS, NG, 4, false, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
+                    } else {
+                        if (bits == 2)
+                            store_codes<D, GS, NG, 2, true, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
+                        else
+                            store_codes<D, GS, NG, 4, true, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
+                    }
                 }
             }
             tc_fence_before_sync();
@@ -580,11 +706,11 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (*abort_flag) {
         if (threadIdx.x == 0)
             flag(P.dev_err, KVQ_DEVERR_WAIT_TIMEOUT);
-        if (warp == kTcEpiWarps && lane == 0)              // copies never consumed
+        if (warp == C::EPI_WARPS && lane == 0)             // copies never consumed
             for (int k = consumed; k < issued; ++k)
-                mbar_wait_bounded(&full[k % kTcStages], (k / kTcStages) & 1);
-        if (warp == kTcEpiWarps + 1 && lane == 0 && consumed > 0)   // the last MMAs
-            mbar_wait_bounded(&accf[(consumed - 1) & 1], ((consumed - 1) >> 1) & 1);
+                mbar_wait_bounded(&full[k % C::STAGES], (k / C::STAGES) & 1);
+        if (warp == C::EPI_WARPS + 1 && lane == 0 && consumed > 0)   // the last MMAs
+            mbar_wait_bounded(&accf[(consumed - 1) % C::EPI], ((consumed - 1) / C::EPI) & 1);
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -664,7 +790,7 @@ cudaError_t launch_tc_t(const void *k, const void *v, const float *Tk, const flo
     P.pos = pos;
     P.dev_err = dev_err;
     P.pm = PageMap{c->block_table, c->page_tokens, c->num_pages};
-    append_tc_kernel<D, GS><<<dim3((unsigned)gx, (unsigned)c->Hkv, 2), kTcThreads, Cf::SMEM, st>>>(
+    append_tc_kernel<D, GS><<<dim3((unsigned)gx, (unsigned)c->Hkv, 2), Cf::THREADS, Cf::SMEM, st>>>(
         mk, mv, P);
     return cudaGetLastError();
 }

@@ -197,6 +197,8 @@ MMA_APPEND_CASES = [
     (128, 4, 2, 128, 0.005, 1, 512, [0]),
     (128, 4, 4, 32, 0.1, 2, 140, [5, 300]),
     (64, 2, 4, 64, 0.05, 2, 160, [96, 0]),
+    (64, 4, 2, 32, 0.05, 2, 200, [0, 64]),     # d 64, group 32, kappa 1, 4-bit keys
+    (64, 2, 2, 32, 0.01, 1, 300, [0]),          # d 64, group 32, kappa 0
 ]
 
 
