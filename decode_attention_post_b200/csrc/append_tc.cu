@@ -42,9 +42,9 @@ constexpr int kTcKBlock = 64;                      // bf16 per 128-byte swizzled
 
 template <int D>
 struct TcCfg {
-    // epilogue warpgroups, one TMEM accumulator buffer each: at d = 64 four, so that one
-    // CTA per SM keeps 16 epilogue warps with the register budget to hold a whole row
-    static constexpr int EPI = D == 64 ? 4 : 2;
+    // epilogue warpgroups, one TMEM accumulator buffer each: at d = 64 three, so that one
+    // CTA per SM keeps 12 epilogue warps with the register budget to hold a whole row
+    static constexpr int EPI = D == 64 ? 3 : 2;
     static constexpr int EPI_WARPS = 4 * EPI;
     static constexpr int THREADS = (EPI_WARPS + 2) * 32;      // + TMA warp + MMA warp
     static constexpr int STAGES = D == 64 ? 4 : 3;            // input tile ring
@@ -57,12 +57,15 @@ struct TcCfg {
     static constexpr int OFF_B_LO = OFF_B_HI + B_BYTES;
     static constexpr int OFF_BAR = OFF_B_LO + B_BYTES;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;         // barriers + alignment slack
-    static constexpr int TMEM_COLS = EPI * D;                 // the accumulator buffers
+    static constexpr int TMEM_COLS = 256;                     // EPI accumulators of D columns
     static constexpr int PER_SM = 1;
-    // registers per thread: the most that THREADS threads get from the SM's 64K in
-    // whole 8-register steps (d = 64: 576 threads, 112 registers)
-    static constexpr int MAXREG = ((65536 / THREADS) / 8) * 8 > 255 ? 255 : ((65536 / THREADS) / 8) * 8;
-    static_assert(TMEM_COLS == 256, "TMEM allocation: a power of two of at most 512 columns");
+    // registers per thread: each of the SM's 4 schedulers holds 16K registers for its
+    // ceil(warps / 4) warps, in whole 8-register steps (d = 64: 14 warps, 128 registers;
+    // d = 128: 10 warps, 168)
+    static constexpr int WARPS_PER_SMSP = (THREADS / 32 + 3) / 4;
+    static constexpr int MAXREG_RAW = (16384 / (32 * WARPS_PER_SMSP)) / 8 * 8;
+    static constexpr int MAXREG = MAXREG_RAW > 255 ? 248 : MAXREG_RAW;
+    static_assert(EPI * D <= TMEM_COLS, "TMEM accumulators");
     static_assert((2 * STAGES + 2 * EPI) * 8 + 8 <= 256, "barrier area");
     static_assert(PER_SM * (SMEM + 1024) <= 228 * 1024, "shared memory oversubscribed");
 };
