@@ -88,6 +88,16 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// An arrive that orders nothing but itself: the epilogue's release of an accumulator
+// buffer. Its TMEM loads are complete (tcgen05.wait::ld) and fenced before the arrive;
+// its global stores need no ordering with the next MMA, and a releasing arrive would
+// hold the warp until they drain.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
 // Codes of a group: c = clamp(rint(f32(f32(x - z) / s)), 0, qmax) for float16 (s, z).
 // The quotient is taken as a reciprocal multiply (within 2 ulp of the IEEE quotient), the
 // clamp comes first (the same result: rint and the clamp are both monotone and the clamp
@@ -127,6 +137,20 @@ __device__ __forceinline__ uint32_t code_of(uint32_t xb, float zf, float sf, flo
         return code_exact(__uint_as_float(xb), zf, sf, zero, qmax);
     else
         return code_bits(__uint_as_float(xb), zf, rc, qmax, tmax);
+}
+
+// magic-rounded bits 0x4B400000 + c of one value; a quotient within the tie band is
+// redone with IEEE division on the spot (rare: the branch is taken by a few lanes)
+__device__ __forceinline__ uint32_t code_fix(uint32_t xb, float zf, float sf, float rc, bool zero,
+                                             float qmax)
+{
+    const float x = __uint_as_float(xb);
+    float y = __fmul_rn(__fsub_rn(x, zf), rc);
+    y = fminf(fmaxf(y, 0.f), qmax);
+    const float r = __fadd_rn(y, kRoundMagic);
+    if (__builtin_expect(fabsf(__fsub_rn(y, __fsub_rn(r, kRoundMagic))) >= kTieBand, 0))
+        return kRoundMagicBits + code_exact(x, zf, sf, zero, qmax);
+    return __float_as_uint(r);
 }
 
 // sum over e < N of 0x4B400000 * 2^(B*e), modulo 2^32: what packing N magic-rounded codes
@@ -288,28 +312,39 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
 }
 
 // d = 64: the token's whole row x0 (dims 0-31), x1 (dims 32-63) is in registers. Codes
-// with the group parameters of each half (p0: dims 0-31, p1: dims 32-63), stored as the
-// K row (one or two 16-byte stores) or as the token's halves of its V tile (whole 16-bit
-// halves: half (gq, rr) holds dims 8(E rr + s) + gq at BITS*s, E = 16/BITS). row < 0:
-// nothing stored. Returns whether a value was within the tie band.
-template <int BITS, bool EXACT>
-__device__ __forceinline__ bool store_row64(const TcParams &P, int which, long long row,
+// with the group parameters of each half (p0: dims 0-31, p1: dims 32-63), each value near
+// a rounding tie redone by IEEE division, stored as the K row (one or two 16-byte stores)
+// or as the token's halves of its V tile (whole 16-bit halves: half (gq, rr) holds dims
+// 8(E rr + s) + gq at BITS*s, E = 16/BITS). row < 0: nothing stored.
+template <int BITS>
+__device__ __forceinline__ void store_row64(const TcParams &P, int which, long long row,
                                             const uint32_t (&x0)[32], const uint32_t (&x1)[32],
                                             const float (&z)[2], const float (&sc)[2],
                                             const float (&rc)[2], const bool (&zr)[2], float qmax)
 {
-    float tmax = 0.f;
     if (!which) {
-        uint32_t w0[BITS], w1[BITS];
-        pack32<BITS, EXACT>(x0, z[0], sc[0], rc[0], zr[0], qmax, tmax, w0);
-        pack32<BITS, EXACT>(x1, z[1], sc[1], rc[1], zr[1], qmax, tmax, w1);
+        // word q of a 32-dim half: dims (32/BITS) q + e at BITS*e
+        constexpr int PER = 32 / BITS;
+        uint32_t w[2][BITS];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int q = 0; q < BITS; ++q) {
+                uint32_t acc = 0u - magic_sum(BITS, PER);
+#pragma unroll
+                for (int e = 0; e < PER; ++e)
+                    acc += code_fix(hf ? x1[PER * q + e] : x0[PER * q + e], z[hf], sc[hf], rc[hf],
+                                    zr[hf], qmax)
+                           << (BITS * e);
+                w[hf][q] = acc;
+            }
         if (row >= 0) {
             uint4 *dst = reinterpret_cast<uint4 *>(P.k_codes + row * (64 * BITS / 8));
             if constexpr (BITS == 2) {
-                dst[0] = make_uint4(w0[0], w0[1 % BITS], w1[0], w1[1 % BITS]);
+                dst[0] = make_uint4(w[0][0], w[0][1 % BITS], w[1][0], w[1][1 % BITS]);
             } else {
-                dst[0] = make_uint4(w0[0], w0[1 % BITS], w0[2 % BITS], w0[3 % BITS]);
-                dst[1] = make_uint4(w1[0], w1[1 % BITS], w1[2 % BITS], w1[3 % BITS]);
+                dst[0] = make_uint4(w[0][0], w[0][1 % BITS], w[0][2 % BITS], w[0][3 % BITS]);
+                dst[1] = make_uint4(w[1][0], w[1][1 % BITS], w[1][2 % BITS], w[1][3 % BITS]);
             }
         }
     } else {
@@ -323,12 +358,11 @@ __device__ __forceinline__ bool store_row64(const TcParams &P, int which, long l
         for (int gq = 0; gq < 8; ++gq) {
             if constexpr (BITS == 2) {
                 // one half per gq: s < 4 from x0 (dim gq + 8 s), s >= 4 from x1
-                uint32_t acc = EXACT ? 0u : 0u - magic_sum(2, 8);
+                uint32_t acc = 0u - magic_sum(2, 8);
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
-                    acc += code_of<EXACT>(x0[8 * s2 + gq], z[0], sc[0], rc[0], zr[0], qmax, tmax)
-                           << (2 * s2);
-                    acc += code_of<EXACT>(x1[8 * s2 + gq], z[1], sc[1], rc[1], zr[1], qmax, tmax)
+                    acc += code_fix(x0[8 * s2 + gq], z[0], sc[0], rc[0], zr[0], qmax) << (2 * s2);
+                    acc += code_fix(x1[8 * s2 + gq], z[1], sc[1], rc[1], zr[1], qmax)
                            << (2 * (4 + s2));
                 }
                 if (row >= 0)
@@ -336,13 +370,11 @@ __device__ __forceinline__ bool store_row64(const TcParams &P, int which, long l
                         (uint16_t)acc;
             } else {
                 // halves rr = 0 (x0) and rr = 1 (x1), s < 4: dim gq + 8 (4 rr + s)
-                uint32_t a0 = EXACT ? 0u : 0u - magic_sum(4, 4), a1 = a0;
+                uint32_t a0 = 0u - magic_sum(4, 4), a1 = a0;
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
-                    a0 += code_of<EXACT>(x0[8 * s2 + gq], z[0], sc[0], rc[0], zr[0], qmax, tmax)
-                          << (4 * s2);
-                    a1 += code_of<EXACT>(x1[8 * s2 + gq], z[1], sc[1], rc[1], zr[1], qmax, tmax)
-                          << (4 * s2);
+                    a0 += code_fix(x0[8 * s2 + gq], z[0], sc[0], rc[0], zr[0], qmax) << (4 * s2);
+                    a1 += code_fix(x1[8 * s2 + gq], z[1], sc[1], rc[1], zr[1], qmax) << (4 * s2);
                 }
                 if (row >= 0) {
                     *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 4, tok, gq, 0)) =
@@ -353,7 +385,6 @@ __device__ __forceinline__ bool store_row64(const TcParams &P, int which, long l
             }
         }
     }
-    return tmax >= kTieBand;
 }
 
 // Running clip statistics of one group of a row: kappa = 0 (min, max), kappa = 1 (second
@@ -570,13 +601,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const bool quest = P.clip == kQuestClip;
         for (int k = wg; k < my_tiles; k += C::EPI) {
             const int a = k % C::EPI;
-            if (*abort_flag || !mbar_wait_bounded(&accf[a], (k / C::EPI) & 1)) {
-                *abort_flag = 1;
-                break;
-            }
-            tc_fence_after_sync();
-            const uint32_t taddr =
-                tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * D);
+            // the token's cache row first: its position load overlaps the wait below
             const long tile = blockIdx.x + (long)k * gridDim.x;
             const long u = tile * kTcTile + r;
             long long row = -1;
@@ -593,6 +618,13 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         flag(P.dev_err, KVQ_DEVERR_PAGE_RANGE);
                 }
             }
+            if (*abort_flag || !mbar_wait_bounded(&accf[a], (k / C::EPI) & 1)) {
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t taddr =
+                tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * D);
             // ---- pass 1: clip parameters per group (every lane takes part in the loads)
             float zf[NG], sf[NG], rc[NG];
             bool zero[NG];
@@ -656,15 +688,10 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 const float z2[2] = {zf[0], zf[NG - 1]}, s2[2] = {sf[0], sf[NG - 1]};
                 const float r2[2] = {rc[0], rc[NG - 1]};
                 const bool zr2[2] = {zero[0], zero[NG - 1]};
-                bool tie = bits == 2
-                               ? store_row64<2, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax)
-                               : store_row64<4, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
-                if (tie && row >= 0) {
-                    if (bits == 2)
-                        store_row64<2, true>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
-                    else
-                        store_row64<4, true>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
-                }
+                if (bits == 2)
+                    store_row64<2>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                else
+                    store_row64<4>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
             } else {
                 uint32_t cur[32];
 #pragma unroll 1
@@ -700,7 +727,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 }
             }
             tc_fence_before_sync();
-            mbar_arrive(&acce[a]);                          // the MMA warp may reuse it
+            mbar_arrive_relaxed(&acce[a]);                  // the MMA warp may reuse it
         }
     }
 
