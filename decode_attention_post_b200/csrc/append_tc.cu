@@ -83,11 +83,6 @@ struct TcParams {
     PageMap pm;
 };
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
 // An arrive that orders nothing but itself: the epilogue's release of an accumulator
 // buffer. Its TMEM loads are complete (tcgen05.wait::ld) and fenced before the arrive;
 // its global stores need no ordering with the next MMA, and a releasing arrive would
@@ -103,7 +98,7 @@ __device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar)
 // clamp comes first (the same result: rint and the clamp are both monotone and the clamp
 // bounds are integers) and the rounding to nearest even is the float addition of
 // 1.5 * 2^23, whose bit pattern is then 0x4B400000 + c. A value within 2^-16 of a
-// rounding tie sets `tie`; the caller then recomputes the row with IEEE division.
+// rounding tie is redone with the IEEE quotient (code_fix).
 constexpr float kRoundMagic = 12582912.0f;        // 1.5 * 2^23
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 constexpr float kTieBand = 0.5f - 1.52587890625e-05f;   // 0.5 - 2^-16
@@ -128,17 +123,6 @@ __device__ __forceinline__ uint32_t code_exact(float x, float zf, float sf, bool
     return (uint32_t)fminf(fmaxf(k, 0.f), qmax);
 }
 
-// code of one value: magic-rounded bits (EXACT = false) or the IEEE-division code
-template <bool EXACT>
-__device__ __forceinline__ uint32_t code_of(uint32_t xb, float zf, float sf, float rc, bool zero,
-                                            float qmax, float &tmax)
-{
-    if constexpr (EXACT)
-        return code_exact(__uint_as_float(xb), zf, sf, zero, qmax);
-    else
-        return code_bits(__uint_as_float(xb), zf, rc, qmax, tmax);
-}
-
 // magic-rounded bits 0x4B400000 + c of one value; a quotient within the tie band is
 // redone with IEEE division on the spot (rare: the branch is taken by a few lanes)
 __device__ __forceinline__ uint32_t code_fix(uint32_t xb, float zf, float sf, float rc, bool zero,
@@ -151,6 +135,18 @@ __device__ __forceinline__ uint32_t code_fix(uint32_t xb, float zf, float sf, fl
     if (__builtin_expect(fabsf(__fsub_rn(y, __fsub_rn(r, kRoundMagic))) >= kTieBand, 0))
         return kRoundMagicBits + code_exact(x, zf, sf, zero, qmax);
     return __float_as_uint(r);
+}
+
+// magic-rounded bits of one value: by the reciprocal (EXACT = false; tmax keeps the tie
+// residual) or with the IEEE quotient for a value within the tie band (EXACT = true)
+template <bool EXACT>
+__device__ __forceinline__ uint32_t code_of(uint32_t xb, float zf, float sf, float rc, bool zero,
+                                            float qmax, float &tmax)
+{
+    if constexpr (EXACT)
+        return code_fix(xb, zf, sf, rc, zero, qmax);
+    else
+        return code_bits(__uint_as_float(xb), zf, rc, qmax, tmax);
 }
 
 // sum over e < N of 0x4B400000 * 2^(B*e), modulo 2^32: what packing N magic-rounded codes
@@ -223,11 +219,10 @@ template <int BITS, bool EXACT>
 __device__ __forceinline__ void pack32(const uint32_t (&x)[32], float zf, float sf, float rc,
                                        bool zero, float qmax, float &tie, uint32_t (&w)[BITS])
 {
-    constexpr bool exact = EXACT;
     constexpr int PER = 32 / BITS;                  // codes per word
 #pragma unroll
     for (int q = 0; q < BITS; ++q) {
-        uint32_t acc = exact ? 0u : 0u - magic_sum(BITS, PER);
+        uint32_t acc = 0u - magic_sum(BITS, PER);
 #pragma unroll
         for (int e = 0; e < PER; ++e) {
             const float v = __uint_as_float(x[PER * q + e]);
@@ -248,7 +243,6 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
                                             const float (&rc)[NG], const bool (&zero)[NG],
                                             float qmax)
 {
-    constexpr bool exact = EXACT;
     constexpr int NCH = D / 32;
     float tie = 0.f;
     uint32_t cur[32];
@@ -286,7 +280,7 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
             uint32_t hv[8];
 #pragma unroll
             for (int gq = 0; gq < 8; ++gq) {
-                uint32_t acc = exact ? 0u : 0u - (magic_sum(BITS, 4) << (BITS * base));
+                uint32_t acc = 0u - (magic_sum(BITS, 4) << (BITS * base));
 #pragma unroll
                 for (int n8 = 0; n8 < 4; ++n8) {
                     const float v = __uint_as_float(cur[8 * n8 + gq]);
@@ -316,12 +310,22 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
 // a rounding tie redone by IEEE division, stored as the K row (one or two 16-byte stores)
 // or as the token's halves of its V tile (whole 16-bit halves: half (gq, rr) holds dims
 // 8(E rr + s) + gq at BITS*s, E = 16/BITS). row < 0: nothing stored.
-template <int BITS>
-__device__ __forceinline__ void store_row64(const TcParams &P, int which, long long row,
+// FIX = false: reciprocal codes only; returns whether a value lies within the tie band
+// (then the caller stores the row again with FIX = true, where each such value takes the
+// IEEE quotient).
+template <int BITS, bool FIX>
+__device__ __forceinline__ bool store_row64(const TcParams &P, int which, long long row,
                                             const uint32_t (&x0)[32], const uint32_t (&x1)[32],
                                             const float (&z)[2], const float (&sc)[2],
                                             const float (&rc)[2], const bool (&zr)[2], float qmax)
 {
+    float tmax = 0.f;
+    auto code = [&](uint32_t xb, int hf) -> uint32_t {
+        if constexpr (FIX)
+            return code_fix(xb, z[hf], sc[hf], rc[hf], zr[hf], qmax);
+        else
+            return code_bits(__uint_as_float(xb), z[hf], rc[hf], qmax, tmax);
+    };
     if (!which) {
         // word q of a 32-dim half: dims (32/BITS) q + e at BITS*e
         constexpr int PER = 32 / BITS;
@@ -333,9 +337,7 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
                 uint32_t acc = 0u - magic_sum(BITS, PER);
 #pragma unroll
                 for (int e = 0; e < PER; ++e)
-                    acc += code_fix(hf ? x1[PER * q + e] : x0[PER * q + e], z[hf], sc[hf], rc[hf],
-                                    zr[hf], qmax)
-                           << (BITS * e);
+                    acc += code(hf ? x1[PER * q + e] : x0[PER * q + e], hf) << (BITS * e);
                 w[hf][q] = acc;
             }
         if (row >= 0) {
@@ -361,9 +363,8 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
                 uint32_t acc = 0u - magic_sum(2, 8);
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
-                    acc += code_fix(x0[8 * s2 + gq], z[0], sc[0], rc[0], zr[0], qmax) << (2 * s2);
-                    acc += code_fix(x1[8 * s2 + gq], z[1], sc[1], rc[1], zr[1], qmax)
-                           << (2 * (4 + s2));
+                    acc += code(x0[8 * s2 + gq], 0) << (2 * s2);
+                    acc += code(x1[8 * s2 + gq], 1) << (2 * (4 + s2));
                 }
                 if (row >= 0)
                     *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 2, tok, gq, 0)) =
@@ -373,8 +374,8 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
                 uint32_t a0 = 0u - magic_sum(4, 4), a1 = a0;
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
-                    a0 += code_fix(x0[8 * s2 + gq], z[0], sc[0], rc[0], zr[0], qmax) << (4 * s2);
-                    a1 += code_fix(x1[8 * s2 + gq], z[1], sc[1], rc[1], zr[1], qmax) << (4 * s2);
+                    a0 += code(x0[8 * s2 + gq], 0) << (4 * s2);
+                    a1 += code(x1[8 * s2 + gq], 1) << (4 * s2);
                 }
                 if (row >= 0) {
                     *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 4, tok, gq, 0)) =
@@ -385,6 +386,7 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
             }
         }
     }
+    return tmax >= kTieBand;
 }
 
 // Running clip statistics of one group of a row: kappa = 0 (min, max), kappa = 1 (second
@@ -394,15 +396,17 @@ struct ClipStats {
     float lo, hi, m1, m2, M1, M2, sm9[9], lg9[9];
     double ss;
 
-    __device__ __forceinline__ void reset()
+    __device__ __forceinline__ void reset(int clip)
     {
         lo = m1 = m2 = INFINITY;
         hi = M1 = M2 = -INFINITY;
         ss = 0.0;
+        if (clip > 1) {
 #pragma unroll
-        for (int e = 0; e < 9; ++e) {
-            sm9[e] = INFINITY;
-            lg9[e] = -INFINITY;
+            for (int e = 0; e < 9; ++e) {
+                sm9[e] = INFINITY;
+                lg9[e] = -INFINITY;
+            }
         }
     }
 
@@ -634,7 +638,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 zero[gg] = true;
             }
             ClipStats cs;
-            cs.reset();
+            cs.reset(P.clip);
             // group gr is complete: its scale and zero-point, stored with the row
             auto finish = [&](int gr) {
                 __half sh, zh;
@@ -671,7 +675,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     (which ? P.v_sz : P.k_sz)[row * NG + gr] =
                         (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
                 }
-                cs.reset();                                 // the next group starts fresh
+                cs.reset(P.clip);                           // the next group starts fresh
             };
             if constexpr (D == 64) {
                 // the whole row in registers: one TMEM round trip, both passes (and the
@@ -688,10 +692,15 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 const float z2[2] = {zf[0], zf[NG - 1]}, s2[2] = {sf[0], sf[NG - 1]};
                 const float r2[2] = {rc[0], rc[NG - 1]};
                 const bool zr2[2] = {zero[0], zero[NG - 1]};
-                if (bits == 2)
-                    store_row64<2>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
-                else
-                    store_row64<4>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                const bool tie = bits == 2
+                    ? store_row64<2, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax)
+                    : store_row64<4, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                if (__builtin_expect(tie, 0)) {             // this row again, fixed up
+                    if (bits == 2)
+                        store_row64<2, true>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                    else
+                        store_row64<4, true>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                }
             } else {
                 uint32_t cur[32];
 #pragma unroll 1
