@@ -387,18 +387,13 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
 // smallest and largest), kappa <= 8 (the 9 smallest and largest by insertion), or the
 // QuEST INT sum of squares (float64, each square exact).
 struct ClipStats {
-    float lo4[4], hi4[4], m1, m2, M1, M2, sm9[9], lg9[9];
+    float lo, hi, m1, m2, M1, M2, sm9[9], lg9[9];
     double ss;
 
     __device__ __forceinline__ void reset(int clip)
     {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            lo4[e] = INFINITY;
-            hi4[e] = -INFINITY;
-        }
-        m1 = m2 = INFINITY;
-        M1 = M2 = -INFINITY;
+        lo = m1 = m2 = INFINITY;
+        hi = M1 = M2 = -INFINITY;
         ss = 0.0;
         if (clip > 1) {
 #pragma unroll
@@ -418,12 +413,10 @@ struct ClipStats {
                 ss = fma(v, v, ss);
             }
         } else if (clip == 0) {
-            // four independent chains (a short dependency path per row)
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-                const int c = (j >> 1) & 3;
-                lo4[c] = fmin3(lo4[c], __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
-                hi4[c] = fmax3(hi4[c], __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+                lo = fmin3(lo, __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+                hi = fmax3(hi, __uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
             }
         } else if (clip == 1) {
 #pragma unroll
@@ -454,8 +447,8 @@ struct ClipStats {
     // the clip range [x_(kappa), x_(g-1-kappa)] of the values added
     __device__ __forceinline__ void range(int clip, float &glo, float &ghi) const
     {
-        glo = fminf(fminf(lo4[0], lo4[1]), fminf(lo4[2], lo4[3]));
-        ghi = fmaxf(fmaxf(hi4[0], hi4[1]), fmaxf(hi4[2], hi4[3]));
+        glo = lo;
+        ghi = hi;
         if (clip == 1) {
             glo = m2;
             ghi = M2;
