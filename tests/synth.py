@@ -29,6 +29,7 @@ import numpy as np
 
 STREAM_K, STREAM_V, STREAM_Q, STREAM_TK, STREAM_TV, STREAM_SEQ, STREAM_CACHE = 1, 2, 3, 4, 5, 6, 7
 STREAM_CODEBOOK = 8
+STREAM_WINDOW, STREAM_VQ = 9, 10
 
 
 @dataclasses.dataclass(frozen=True)
@@ -258,3 +259,25 @@ def codebooks(cfg: Config):
         c = r.standard_normal((cfg.Hkv, 256, 4)).astype(np.float16)
         out.append(np.ascontiguousarray(c).view(np.uint16))
     return out[0], out[1]
+
+
+def window_tokens(cfg: Config, b: int, n: int) -> tuple:
+    """Full-precision window tokens of sequence b for full-size tests: keys and values
+    float32 N(0, 1) [Hkv][n][d] (callers round them to bfloat16)."""
+    r = _rng(cfg, STREAM_WINDOW, b)
+    return (r.standard_normal((cfg.Hkv, n, cfg.d)).astype(np.float32),
+            r.standard_normal((cfg.Hkv, n, cfg.d)).astype(np.float32))
+
+
+def random_vq_planes(cfg: Config, b: int, tokens: int) -> tuple:
+    """Uniform random vector-quantized cache contents of sequence b (all KV heads), to
+    exercise the VQ decode at full size without running the encoder: indices uint8
+    [Hkv][tokens][d/4], gains float16 bits uint16 [Hkv][tokens] in [0.5, 1.5) (keys, then
+    values)."""
+    r = _rng(cfg, STREAM_VQ, b)
+    g = lambda: r.uniform(0.5, 1.5, size=(cfg.Hkv, tokens)).astype(np.float16).view(np.uint16)
+    ki = r.integers(0, 256, size=(cfg.Hkv, tokens, cfg.d // 4), dtype=np.uint8)
+    kg = g()
+    vi = r.integers(0, 256, size=(cfg.Hkv, tokens, cfg.d // 4), dtype=np.uint8)
+    vg = g()
+    return ki, kg, vi, vg

@@ -468,6 +468,69 @@ def test_decode_full_size_sampled(idx):
     assert np.array_equal(bf16_bits(out16), bf16_bits(out.to(torch.bfloat16)))
 
 
+def test_window_decode_full_size_sampled():
+    """The batch-64 / 12K-16K shape with the bench's window (S_sink 64, S_keep 256, S_flush
+    128) in the bench's launch configuration: random quantized middles from cache position
+    0, random bfloat16 sink and ring rows (the unused ring slots hold NaN bit patterns);
+    the oracle's windowed decode on sampled sequences, each run on its own."""
+    cfg = synth.CONFIGS[2]
+    S_sink, S_keep, S_flush = 64, 256, 128
+    R = S_keep + S_flush
+    B, Hkv, d, T = cfg.B, cfg.Hkv, cfg.d, cfg.T_cap
+    seql = synth.seqlens(cfg)
+    Qs = [oracle.window_quantized(int(L), S_sink, S_keep, S_flush) for L in seql]
+    gpu_c = oracle.Cache.for_config(cfg)
+    ks = np.full((B, Hkv, S_sink, d), 0x7FC1, np.uint16)
+    vs = ks.copy()
+    kr = np.full((B, Hkv, R, d), 0x7FC1, np.uint16)
+    vr = kr.copy()
+    f16 = lambda a: a.astype(np.float16).view(np.uint16)
+    win = {}
+    for b in range(B):
+        L, Q = int(seql[b]), Qs[b]
+        kc, vc, k_s, k_z, v_s, v_z = synth.random_cache_fields(cfg, b, (Q + 15) // 16 * 16)
+        for h in range(Hkv):
+            gpu_c.pack_tokens(b, h, 0, kc[h], vc[h], np.stack([f16(k_s[h]), f16(k_z[h])], -1),
+                              np.stack([f16(v_s[h]), f16(v_z[h])], -1))
+        pos = list(range(min(S_sink, L))) + list(range(S_sink + Q, L))
+        kw, vw = synth.window_tokens(cfg, b, len(pos))
+        kw, vw = synth.as_dtype(kw, "bf16"), synth.as_dtype(vw, "bf16")
+        for j, t in enumerate(pos):
+            if t < S_sink:
+                ks[b, :, t], vs[b, :, t] = kw[:, j], vw[:, j]
+            else:
+                kr[b, :, t % R], vr[b, :, t % R] = kw[:, j], vw[:, j]
+        win[b] = (pos, kw, vw, (kc, vc, k_s, k_z, v_s, v_z))
+    gc = upload_cache(gpu_c, cfg)
+    q = synth.as_dtype(synth.queries(cfg), "bf16")
+    _, Tv, Tit = synth.transforms(cfg)
+    out = torch.empty((B, cfg.Hq, d), dtype=torch.float32, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ws = torch.empty(kvq.decode_workspace_bytes(gc, cfg.Hq, T), dtype=torch.uint8, device=DEV)
+    kvq.decode_attention_window(t_(q), t_(Tit), gc, S_sink, S_keep, S_flush, t_(ks), t_(vs),
+                                t_(kr), t_(vr), t_(Tv), t_(seql.astype(np.int32)), T, out, ws,
+                                dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    for b in (0, int(np.argmax(seql)), B - 1):
+        L, Q = int(seql[b]), Qs[b]
+        pos, kw, vw, (kc, vc, k_s, k_z, v_s, v_z) = win[b]
+        one = oracle.Cache(1, Hkv, T, d, cfg.bits_k, cfg.bits_v, cfg.group)
+        for h in range(Hkv):
+            one.pack_tokens(0, h, S_sink, kc[h][:Q], vc[h][:Q],
+                            np.stack([f16(k_s[h][:Q]), f16(k_z[h][:Q])], -1),
+                            np.stack([f16(v_s[h][:Q]), f16(v_z[h][:Q])], -1))
+        k_all = np.zeros((1, T, Hkv, d), np.uint16)
+        v_all = np.zeros_like(k_all)
+        for j, t in enumerate(pos):
+            k_all[0, t], v_all[0, t] = kw[:, j], vw[:, j]
+        want = oracle.window_decode(q[b:b + 1], Tit, Tv, k_all, v_all, one,
+                                    np.array([L], np.int32), S_sink, S_keep, S_flush)
+        assert_close(got[b:b + 1], want, where=f"window full size b{b}")
+
+
 def test_append_full_size_sampled_config4():
     """32768-token chunk append of the GPT-OSS-like shape; oracle on sampled tokens."""
     cfg = synth.CONFIGS[4]

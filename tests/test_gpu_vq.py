@@ -93,10 +93,10 @@ def test_vq_append_end_to_end(cfg, B, n, pos, dtype):
         assert np.abs(a.view(np.uint16).astype(np.int32) - b.astype(np.int32)).max() <= 1
 
 
-def gpu_vq_decode(cfg, q, M, gc, seql, out_dtype=torch.float32):
+def gpu_vq_decode(cfg, q, M, gc, seql, out_dtype=torch.float32, mx=None):
     cb_k, cb_v = synth.codebooks(cfg)
     B, Hq = q.shape[0], q.shape[1]
-    mx = int(max(seql))
+    mx = int(max(seql)) if mx is None else mx
     ws = torch.empty(kvq.vq_decode_workspace_bytes(gc, Hq, mx), dtype=torch.uint8, device=DEV)
     out = torch.empty((B, Hq, cfg.d), dtype=out_dtype, device=DEV)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
@@ -154,3 +154,36 @@ def test_vq_decode_split_invariance(splits, monkeypatch):
     out, err = gpu_vq_decode(cfg, q, Tit, gc, seql)
     assert err == 0
     assert_close(out.cpu().numpy(), want, where=f"vq splits={splits}")
+
+
+def test_vq_decode_full_size_sampled():
+    """The batch-64 / 12K-16K shape in the bench's launch configuration over random indices
+    and gains; the oracle on sampled (sequence, head) outputs."""
+    cfg = synth.CONFIGS[2]
+    B, Hkv, d, T = cfg.B, cfg.Hkv, cfg.d, cfg.T_cap
+    seql = synth.seqlens(cfg)
+    oc = oracle.VQCache(B, Hkv, T, d)
+    ki_all = oc.k_idx.reshape(B, Hkv, T, d // 4)
+    vi_all = oc.v_idx.reshape(B, Hkv, T, d // 4)
+    kg_all = oc.k_gain.reshape(B, Hkv, T)
+    vg_all = oc.v_gain.reshape(B, Hkv, T)
+    for b in range(B):
+        n = int(seql[b])
+        ki, kg, vi, vg = synth.random_vq_planes(cfg, b, n)
+        ki_all[b, :, :n], kg_all[b, :, :n], vi_all[b, :, :n], vg_all[b, :, :n] = ki, kg, vi, vg
+    gc = upload_vq(oc)
+    q = synth.as_dtype(synth.queries(cfg), "bf16")
+    _, _, Tit = synth.transforms(cfg)
+    cb_k, cb_v = synth.codebooks(cfg)
+    out, err = gpu_vq_decode(cfg, q, Tit, gc, seql, mx=T)
+    assert err == 0
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    rng = np.random.default_rng(2)
+    sel = np.stack([rng.integers(0, B, 10), rng.integers(0, cfg.Hq, 10)], 1).astype(np.int32)
+    sel[0] = [0, 0]
+    sel[1] = [B - 1, cfg.Hq - 1]
+    sel = np.unique(sel, axis=0)
+    want = oracle.vq_decode(q, Tit, cb_k, cb_v, oc, seql, sel=sel)
+    for b, h in sel:
+        assert_close(got[b, h], want[b, h], where=f"vq full size b{b} h{h}")
