@@ -103,17 +103,6 @@ constexpr float kRoundMagic = 12582912.0f;        // 1.5 * 2^23
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 constexpr float kTieBand = 0.5f - 1.52587890625e-05f;   // 0.5 - 2^-16
 
-// bit pattern 0x4B400000 + c of the rounded value; tmax keeps the largest distance of a
-// quotient from its rounded value (a row with tmax >= kTieBand is near a rounding tie)
-__device__ __forceinline__ uint32_t code_bits(float x, float zf, float rc, float qmax, float &tmax)
-{
-    float y = __fmul_rn(__fsub_rn(x, zf), rc);
-    y = fminf(fmaxf(y, 0.f), qmax);
-    const float r = __fadd_rn(y, kRoundMagic);
-    tmax = fmaxf(tmax, fabsf(__fsub_rn(y, __fsub_rn(r, kRoundMagic))));
-    return __float_as_uint(r);
-}
-
 // the same code by IEEE division (ties to even); s_h == 0 or a non-finite range gives 0
 __device__ __forceinline__ uint32_t code_exact(float x, float zf, float sf, bool zero, float qmax)
 {
@@ -121,6 +110,17 @@ __device__ __forceinline__ uint32_t code_exact(float x, float zf, float sf, bool
         return 0u;
     const float k = rintf(__fdiv_rn(__fsub_rn(x, zf), sf));
     return (uint32_t)fminf(fmaxf(k, 0.f), qmax);
+}
+
+// bit pattern 0x4B400000 + c of the rounded value; tie is set when the quotient lies
+// within the tie band (a predicate OR per value: no branch, a one-cycle chain)
+__device__ __forceinline__ uint32_t code_flag(float x, float zf, float rc, float qmax, bool &tie)
+{
+    float y = __fmul_rn(__fsub_rn(x, zf), rc);
+    y = fminf(fmaxf(y, 0.f), qmax);
+    const float r = __fadd_rn(y, kRoundMagic);
+    tie |= fabsf(__fsub_rn(y, __fsub_rn(r, kRoundMagic))) >= kTieBand;
+    return __float_as_uint(r);
 }
 
 // magic-rounded bits 0x4B400000 + c of one value; a quotient within the tie band is
@@ -137,16 +137,16 @@ __device__ __forceinline__ uint32_t code_fix(uint32_t xb, float zf, float sf, fl
     return __float_as_uint(r);
 }
 
-// magic-rounded bits of one value: by the reciprocal (EXACT = false; tmax keeps the tie
-// residual) or with the IEEE quotient for a value within the tie band (EXACT = true)
+// magic-rounded bits of one value: by the reciprocal (EXACT = false; tie is set near a
+// rounding tie) or with the IEEE quotient for a value within the tie band (EXACT = true)
 template <bool EXACT>
 __device__ __forceinline__ uint32_t code_of(uint32_t xb, float zf, float sf, float rc, bool zero,
-                                            float qmax, float &tmax)
+                                            float qmax, bool &tie)
 {
     if constexpr (EXACT)
         return code_fix(xb, zf, sf, rc, zero, qmax);
     else
-        return code_bits(__uint_as_float(xb), zf, rc, qmax, tmax);
+        return code_flag(__uint_as_float(xb), zf, rc, qmax, tie);
 }
 
 // sum over e < N of 0x4B400000 * 2^(B*e), modulo 2^32: what packing N magic-rounded codes
@@ -217,7 +217,7 @@ __device__ __forceinline__ bool pickb(const bool (&a)[NG], int gr)
 // reciprocal codes (sets tie near a rounding tie); exact = true: IEEE division.
 template <int BITS, bool EXACT>
 __device__ __forceinline__ void pack32(const uint32_t (&x)[32], float zf, float sf, float rc,
-                                       bool zero, float qmax, float &tie, uint32_t (&w)[BITS])
+                                       bool zero, float qmax, bool &tie, uint32_t (&w)[BITS])
 {
     constexpr int PER = 32 / BITS;                  // codes per word
 #pragma unroll
@@ -244,7 +244,7 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
                                             float qmax)
 {
     constexpr int NCH = D / 32;
-    float tie = 0.f;
+    bool tie = false;
     uint32_t cur[32];
     tmem_ld32_async(taddr, cur);
     tmem_ld_wait();
@@ -302,7 +302,7 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
             }
         }
     }
-    return tie >= kTieBand;
+    return tie;
 }
 
 // d = 64: the token's whole row x0 (dims 0-31), x1 (dims 32-63) is in registers. Codes
@@ -310,16 +310,22 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
 // a rounding tie redone by IEEE division, stored as the K row (one or two 16-byte stores)
 // or as the token's halves of its V tile (whole 16-bit halves: half (gq, rr) holds dims
 // 8(E rr + s) + gq at BITS*s, E = 16/BITS). row < 0: nothing stored.
-// (Measured on the 32K-token chunk: this per-value branch beats a branch-free pass with
-// a whole-row fix-up pass for rows near a tie, 0.48 against 0.61 ms.)
-template <int BITS>
-__device__ __forceinline__ void store_row64(const TcParams &P, int which, long long row,
+// FIX = false: reciprocal codes, returns whether a value lies within the tie band (the
+// caller then stores the row again with FIX = true, where each such value takes the IEEE
+// quotient). Measured on the 32K-token chunk: the tie test as a predicate OR in this pass
+// is much cheaper than a branch per value or a float max chain.
+template <int BITS, bool FIX>
+__device__ __forceinline__ bool store_row64(const TcParams &P, int which, long long row,
                                             const uint32_t (&x0)[32], const uint32_t (&x1)[32],
                                             const float (&z)[2], const float (&sc)[2],
                                             const float (&rc)[2], const bool (&zr)[2], float qmax)
 {
+    bool tie = false;
     auto code = [&](uint32_t xb, int hf, int) -> uint32_t {
-        return code_fix(xb, z[hf], sc[hf], rc[hf], zr[hf], qmax);
+        if constexpr (FIX)
+            return code_fix(xb, z[hf], sc[hf], rc[hf], zr[hf], qmax);
+        else
+            return code_flag(__uint_as_float(xb), z[hf], rc[hf], qmax, tie);
     };
     if (!which) {
         // word q of a 32-dim half: dims (32/BITS) q + e at BITS*e
@@ -381,6 +387,7 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
             }
         }
     }
+    return tie;
 }
 
 // Running clip statistics of one group of a row: kappa = 0 (min, max), kappa = 1 (second
@@ -686,10 +693,15 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 const float z2[2] = {zf[0], zf[NG - 1]}, s2[2] = {sf[0], sf[NG - 1]};
                 const float r2[2] = {rc[0], rc[NG - 1]};
                 const bool zr2[2] = {zero[0], zero[NG - 1]};
-                if (bits == 2)
-                    store_row64<2>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
-                else
-                    store_row64<4>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                const bool tie = bits == 2
+                    ? store_row64<2, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax)
+                    : store_row64<4, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                if (__builtin_expect(tie, 0)) {             // this row again, fixed up
+                    if (bits == 2)
+                        store_row64<2, true>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                    else
+                        store_row64<4, true>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
+                }
             } else {
                 uint32_t cur[32];
 #pragma unroll 1
