@@ -13,8 +13,8 @@
 //      rounds of a warp-wide min (max) with removal of one instance (exact, ties safe);
 //      for the QuEST INT quantizer, the group RMS from a float64 sum of squares.
 //   4. Scale and zero-point use IEEE float32 division (__fdiv_rn); codes use the
-//      reciprocal with the IEEE quotient near rounding ties, ties to even, so they
-//      match the definition bit for bit.
+//      correctly rounded quotient from a reciprocal and one correction, ties to even, so
+//      they match the definition bit for bit.
 //   5. Codes are packed in registers by OR-reductions over lanes and written as whole
 //      32-bit words (K rows) or whole 16-bit halves (V tiles); every token owns whole
 //      bytes, so no read-modify-write is needed even for single-token appends. The
@@ -138,10 +138,9 @@ __device__ __forceinline__ TokenSlot token_slot(const TokenMap &tm, const void *
 // Quantize one token held by a warp (lane l holds dims l + 32 r in vals[r]) and store it
 // at cache row `row`: per group the clip range (order statistics, or the RMS for the QuEST
 // INT quantizer, kappa == kQuestClip), the float16 scale and zero-point, and the codes
-// c = clamp(rint((x - z) / s), 0, qmax) computed as (x - z) * rcp_rn(s), which is within
-// 2 ulp of the IEEE quotient; a value within 2^-20 of a rounding tie takes the IEEE
-// quotient, so the codes are those of the definition bit for bit (rint as a float32 add
-// and subtract of 1.5 * 2^23 on y clamped to [-1, qmax + 1], ties to even). The K row
+// c = clamp(rint((x - z) / s), 0, qmax) from the correctly rounded quotient (div_rn: a
+// reciprocal and one correction), so the codes are those of the definition bit for bit
+// (rint as the float32 addition of 1.5 * 2^23 to the clamped quotient, ties to even). The K row
 // (whole 32-bit words) or the token's halves of its V tile are packed in registers by
 // OR-reductions over the lanes that share a word or half. bits is 2 or 4.
 constexpr float kRoundMagic = 12582912.0f;      // 1.5 * 2^23
@@ -203,20 +202,14 @@ __device__ __forceinline__ void quantize_store_token(const float (&vals)[D / 32]
             flag(dev_err, KVQ_DEVERR_NONFINITE);
         const bool zero = !finite || sf == 0.f;
         const float rc = zero ? 0.f : __frcp_rn(sf);
-        const float ymax = (float)(qmax + 1);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             if (r < r0 || r >= r0 + nr || zero)
                 continue;
-            const float dlt = __fsub_rn(vals[r], zf);
-            float y = fminf(fmaxf(__fmul_rn(dlt, rc), -1.f), ymax);
-            float k = __fsub_rn(__fadd_rn(y, kRoundMagic), kRoundMagic);
-            if (fabsf(y - k) >= 0.5f - 9.5367431640625e-07f * fmaxf(fabsf(y), 1.f)) {
-                y = fminf(fmaxf(__fdiv_rn(dlt, sf), -1.f), ymax);
-                k = __fsub_rn(__fadd_rn(y, kRoundMagic), kRoundMagic);
-            }
-            k = fminf(fmaxf(k, 0.f), (float)qmax);
-            cq[r] = (uint32_t)(__float_as_int(__fadd_rn(k, kRoundMagic)) - 0x4B400000);
+            // the correctly rounded quotient, clamped, rounded to nearest even
+            const float y = fminf(fmaxf(div_rn(__fsub_rn(vals[r], zf), sf, rc), 0.f),
+                                  (float)qmax);
+            cq[r] = (uint32_t)(__float_as_int(__fadd_rn(y, kRoundMagic)) - 0x4B400000);
         }
         if (lane == 0) {
             uint32_t pair = (uint32_t)__half_as_ushort(sh) |

@@ -3,24 +3,24 @@
 // 5.3; "Spend Bits Where Queries Look", "Three requirements", item 3).
 //
 // CTA = (KV head, one of {K, V}, slice of the 128-token tiles of the flattened
-// (sequence, new token) list), 6 warps with fixed roles:
-//   warp 8, one lane   TMA: each 128-token input tile [128 x d] bf16 lands in a 3-stage
-//                      shared-memory ring in the 128-byte-swizzled K-major layout (3-D
-//                      tensor map over [tokens][Hkv][d], no multicast);
-//   warp 9, one lane   tcgen05.mma: X~[128 x d] = X . T_hi^T + X . T_lo^T into one float32
+// (sequence, new token) list), one CTA per SM, warps with fixed roles:
+//   TMA warp, one lane each 128-token input tile [128 x d] bf16 lands in a 4-stage (d = 64)
+//                      or 3-stage (d = 128) shared-memory ring in the 128-byte-swizzled
+//                      K-major layout (3-D tensor map over [tokens][Hkv][d], no multicast);
+//   MMA warp, one lane tcgen05.mma: X~[128 x d] = X . T_hi^T + X . T_lo^T into one float32
 //                      TMEM accumulator (T split into two bfloat16 pieces, 16 significant
 //                      bits; X is bfloat16, hence exact), M = 128, N = d, K = 16 per
-//                      instruction; two accumulator buffers so that the next tile's MMAs
-//                      overlap this tile's epilogue;
-//   warps 0-7          epilogue, two warpgroups taking alternate tiles (one accumulator
-//                      buffer each): thread r owns token r of the tile; tcgen05.ld brings its
-//                      transformed values into registers 32 columns at a time, in two
-//                      passes: per group the clip range (order statistics, or the RMS for
-//                      the QuEST INT quantizer) and the float16 scale and zero-point, then
-//                      the codes (reciprocal multiply; a row with a value within 2^-16 of a
-//                      rounding tie is redone with IEEE division, so the codes are those of
-//                      the definition bit for bit) and the fixed-width stores (one K row,
-//                      or the token's halves of its 16-token V tile).
+//                      instruction; one accumulator buffer per epilogue warpgroup so that
+//                      the next tiles' MMAs overlap this tile's epilogue;
+//   epilogue warps     three (d = 64) or two (d = 128) warpgroups taking the tiles round
+//                      robin: thread r owns token r of the tile; tcgen05.ld brings its
+//                      transformed values into registers (the whole row at d = 64, 32
+//                      columns at a time at d = 128), in two passes: per group the clip
+//                      range (order statistics, or the RMS for the QuEST INT quantizer) and
+//                      the float16 scale and zero-point, then the codes (the correctly
+//                      rounded quotient by a reciprocal and one correction, so the codes are
+//                      those of the definition bit for bit) and the fixed-width stores (one
+//                      K row, or the token's halves of its 16-token V tile).
 // T (the B operand, N = d output dims x K = d input dims, K-major) is converted and
 // swizzled into shared memory once per CTA. Every wait is bounded; a wait that gives up
 // flags KVQ_DEVERR_WAIT_TIMEOUT, the CTA waits (bounded) for its copies and MMAs in flight,
@@ -94,59 +94,19 @@ __device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar)
 }
 
 // Codes of a group: c = clamp(rint(f32(f32(x - z) / s)), 0, qmax) for float16 (s, z).
-// The quotient is taken as a reciprocal multiply (within 2 ulp of the IEEE quotient), the
-// clamp comes first (the same result: rint and the clamp are both monotone and the clamp
-// bounds are integers) and the rounding to nearest even is the float addition of
-// 1.5 * 2^23, whose bit pattern is then 0x4B400000 + c. A value within 2^-16 of a
-// rounding tie is redone with the IEEE quotient (code_fix).
+// The quotient is the correctly rounded one (div_rn: a reciprocal and one correction), so
+// the codes are those of the definition bit for bit with no tie test; the clamp comes first
+// (the same result: rint and the clamp are both monotone and the clamp bounds are
+// integers) and the rounding to nearest even is the float addition of 1.5 * 2^23, whose
+// bit pattern is then 0x4B400000 + c. A zero or non-finite scale (rc = 0) gives code 0.
 constexpr float kRoundMagic = 12582912.0f;        // 1.5 * 2^23
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
-constexpr float kTieBand = 0.5f - 1.52587890625e-05f;   // 0.5 - 2^-16
 
-// the same code by IEEE division (ties to even); s_h == 0 or a non-finite range gives 0
-__device__ __forceinline__ uint32_t code_exact(float x, float zf, float sf, bool zero, float qmax)
+__device__ __forceinline__ uint32_t code_rn(uint32_t xb, float zf, float sf, float rc, float qmax)
 {
-    if (zero)
-        return 0u;
-    const float k = rintf(__fdiv_rn(__fsub_rn(x, zf), sf));
-    return (uint32_t)fminf(fmaxf(k, 0.f), qmax);
-}
-
-// bit pattern 0x4B400000 + c of the rounded value; tie is set when the quotient lies
-// within the tie band (a predicate OR per value: no branch, a one-cycle chain)
-__device__ __forceinline__ uint32_t code_flag(float x, float zf, float rc, float qmax, bool &tie)
-{
-    float y = __fmul_rn(__fsub_rn(x, zf), rc);
+    float y = div_rn(__fsub_rn(__uint_as_float(xb), zf), sf, rc);
     y = fminf(fmaxf(y, 0.f), qmax);
-    const float r = __fadd_rn(y, kRoundMagic);
-    tie |= fabsf(__fsub_rn(y, __fsub_rn(r, kRoundMagic))) >= kTieBand;
-    return __float_as_uint(r);
-}
-
-// magic-rounded bits 0x4B400000 + c of one value; a quotient within the tie band is
-// redone with IEEE division on the spot (rare: the branch is taken by a few lanes)
-__device__ __forceinline__ uint32_t code_fix(uint32_t xb, float zf, float sf, float rc, bool zero,
-                                             float qmax)
-{
-    const float x = __uint_as_float(xb);
-    float y = __fmul_rn(__fsub_rn(x, zf), rc);
-    y = fminf(fmaxf(y, 0.f), qmax);
-    const float r = __fadd_rn(y, kRoundMagic);
-    if (__builtin_expect(fabsf(__fsub_rn(y, __fsub_rn(r, kRoundMagic))) >= kTieBand, 0))
-        return kRoundMagicBits + code_exact(x, zf, sf, zero, qmax);
-    return __float_as_uint(r);
-}
-
-// magic-rounded bits of one value: by the reciprocal (EXACT = false; tie is set near a
-// rounding tie) or with the IEEE quotient for a value within the tie band (EXACT = true)
-template <bool EXACT>
-__device__ __forceinline__ uint32_t code_of(uint32_t xb, float zf, float sf, float rc, bool zero,
-                                            float qmax, bool &tie)
-{
-    if constexpr (EXACT)
-        return code_fix(xb, zf, sf, rc, zero, qmax);
-    else
-        return code_flag(__uint_as_float(xb), zf, rc, qmax, tie);
+    return __float_as_uint(__fadd_rn(y, kRoundMagic));
 }
 
 // sum over e < N of 0x4B400000 * 2^(B*e), modulo 2^32: what packing N magic-rounded codes
@@ -202,32 +162,20 @@ __device__ __forceinline__ float pick(const float (&a)[NG], int gr)
     return v;
 }
 
-template <int NG>
-__device__ __forceinline__ bool pickb(const bool (&a)[NG], int gr)
-{
-    bool v = a[0];
-#pragma unroll
-    for (int i = 1; i < NG; ++i)
-        v = gr == i ? a[i] : v;
-    return v;
-}
 
 // Codes of 32 consecutive dims (column c0.. of the row) packed as BITS-bit fields of
-// 32-bit words: `words` words, field e of word q = dim c0 + (32/BITS) q + e. exact = false:
-// reciprocal codes (sets tie near a rounding tie); exact = true: IEEE division.
-template <int BITS, bool EXACT>
+// 32-bit words: `words` words, field e of word q = dim c0 + (32/BITS) q + e.
+template <int BITS>
 __device__ __forceinline__ void pack32(const uint32_t (&x)[32], float zf, float sf, float rc,
-                                       bool zero, float qmax, bool &tie, uint32_t (&w)[BITS])
+                                       float qmax, uint32_t (&w)[BITS])
 {
     constexpr int PER = 32 / BITS;                  // codes per word
 #pragma unroll
     for (int q = 0; q < BITS; ++q) {
         uint32_t acc = 0u - magic_sum(BITS, PER);
 #pragma unroll
-        for (int e = 0; e < PER; ++e) {
-            const float v = __uint_as_float(x[PER * q + e]);
-            acc += code_of<EXACT>(__float_as_uint(v), zf, sf, rc, zero, qmax, tie) << (BITS * e);
-        }
+        for (int e = 0; e < PER; ++e)
+            acc += code_rn(x[PER * q + e], zf, sf, rc, qmax) << (BITS * e);
         w[q] = acc;
     }
 }
@@ -236,18 +184,14 @@ __device__ __forceinline__ void pack32(const uint32_t (&x)[32], float zf, float 
 // SM hide the load latency), stored as the K row (little-endian bit stream, dim j at
 // bit BITS*j) or as the token's halves of its 16-token V tile (half (gq, rr) holds dims
 // 8(E rr + s) + gq at BITS*s, E = 16/BITS). row < 0: codes not stored (the warp still
-// takes part in the TMEM loads). Returns whether a value was within the tie band.
-template <int D, int GS, int NG, int BITS, bool V, bool EXACT>
-__device__ __forceinline__ bool store_codes(const TcParams &P, long long row, uint32_t taddr,
+// takes part in the TMEM loads).
+template <int D, int GS, int NG, int BITS, bool V>
+__device__ __forceinline__ void store_codes(const TcParams &P, long long row, uint32_t taddr,
                                             const float (&zf)[NG], const float (&sf)[NG],
-                                            const float (&rc)[NG], const bool (&zero)[NG],
-                                            float qmax)
+                                            const float (&rc)[NG], float qmax)
 {
     constexpr int NCH = D / 32;
-    bool tie = false;
     uint32_t cur[32];
-    tmem_ld32_async(taddr, cur);
-    tmem_ld_wait();
     unsigned char *vbase = nullptr;
     int tok = 0;
     if (V && row >= 0) {
@@ -256,13 +200,13 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
     }
 #pragma unroll 1
     for (int c = 0; c < NCH; ++c) {
-        if (c > 0) { tmem_ld32_async(taddr + 32 * c, cur); tmem_ld_wait(); }
+        tmem_ld32_async(taddr + 32 * c, cur);
+        tmem_ld_wait();
         const int gr = (32 * c) / GS;
         const float z = pick(zf, gr), s = pick(sf, gr), r = pick(rc, gr);
-        const bool zr = pickb(zero, gr);
         if (!V) {
             uint32_t w[BITS];
-            pack32<BITS, EXACT>(cur, z, s, r, zr, qmax, tie, w);
+            pack32<BITS>(cur, z, s, r, qmax, w);
             if (row >= 0) {
                 uint32_t *dst = reinterpret_cast<uint32_t *>(P.k_codes + row * (D * BITS / 8)) + BITS * c;
                 if (BITS == 2)
@@ -282,11 +226,8 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
             for (int gq = 0; gq < 8; ++gq) {
                 uint32_t acc = 0u - (magic_sum(BITS, 4) << (BITS * base));
 #pragma unroll
-                for (int n8 = 0; n8 < 4; ++n8) {
-                    const float v = __uint_as_float(cur[8 * n8 + gq]);
-                    acc += code_of<EXACT>(__float_as_uint(v), z, s, r, zr, qmax, tie)
-                           << (BITS * (base + n8));
-                }
+                for (int n8 = 0; n8 < 4; ++n8)
+                    acc += code_rn(cur[8 * n8 + gq], z, s, r, qmax) << (BITS * (base + n8));
                 hv[gq] = acc;
             }
             if (row >= 0) {
@@ -302,32 +243,21 @@ __device__ __forceinline__ bool store_codes(const TcParams &P, long long row, ui
             }
         }
     }
-    return tie;
 }
 
 // d = 64: the token's whole row x0 (dims 0-31), x1 (dims 32-63) is in registers. Codes
-// with the group parameters of each half (p0: dims 0-31, p1: dims 32-63), each value near
-// a rounding tie redone by IEEE division, stored as the K row (one or two 16-byte stores)
-// or as the token's halves of its V tile (whole 16-bit halves: half (gq, rr) holds dims
-// 8(E rr + s) + gq at BITS*s, E = 16/BITS). row < 0: nothing stored.
-// FIX = false: reciprocal codes, returns whether a value lies within the tie band (the
-// caller then stores the row again with FIX = true, where each such value takes the IEEE
-// quotient). Measured on the 32K-token chunk: keeping this pass free of branches and of
-// anything that holds the row's registers beyond it (the fix-up reloads the row) matters
-// more than anything else in the epilogue -- 0.22 ms without a tie test at all, 0.47 with
-// a branch per value, 0.61 with a fix-up from the same registers.
-template <int BITS, bool FIX>
-__device__ __forceinline__ bool store_row64(const TcParams &P, int which, long long row,
+// with the group parameters of each half (index 0: dims 0-31, 1: dims 32-63), stored as
+// the K row (one or two 16-byte stores) or as the token's halves of its V tile (whole
+// 16-bit halves: half (gq, rr) holds dims 8(E rr + s) + gq at BITS*s, E = 16/BITS).
+// row < 0: nothing stored.
+template <int BITS>
+__device__ __forceinline__ void store_row64(const TcParams &P, int which, long long row,
                                             const uint32_t (&x0)[32], const uint32_t (&x1)[32],
                                             const float (&z)[2], const float (&sc)[2],
-                                            const float (&rc)[2], const bool (&zr)[2], float qmax)
+                                            const float (&rc)[2], float qmax)
 {
-    bool tie = false;
-    auto code = [&](uint32_t xb, int hf, int) -> uint32_t {
-        if constexpr (FIX)
-            return code_fix(xb, z[hf], sc[hf], rc[hf], zr[hf], qmax);
-        else
-            return code_flag(__uint_as_float(xb), z[hf], rc[hf], qmax, tie);
+    auto code = [&](uint32_t xb, int hf) -> uint32_t {
+        return code_rn(xb, z[hf], sc[hf], rc[hf], qmax);
     };
     if (!which) {
         // word q of a 32-dim half: dims (32/BITS) q + e at BITS*e
@@ -340,7 +270,7 @@ __device__ __forceinline__ bool store_row64(const TcParams &P, int which, long l
                 uint32_t acc = 0u - magic_sum(BITS, PER);
 #pragma unroll
                 for (int e = 0; e < PER; ++e)
-                    acc += code(hf ? x1[PER * q + e] : x0[PER * q + e], hf, e) << (BITS * e);
+                    acc += code(hf ? x1[PER * q + e] : x0[PER * q + e], hf) << (BITS * e);
                 w[hf][q] = acc;
             }
         if (row >= 0) {
@@ -366,8 +296,8 @@ __device__ __forceinline__ bool store_row64(const TcParams &P, int which, long l
                 uint32_t acc = 0u - magic_sum(2, 8);
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
-                    acc += code(x0[8 * s2 + gq], 0, s2) << (2 * s2);
-                    acc += code(x1[8 * s2 + gq], 1, s2 + 2) << (2 * (4 + s2));
+                    acc += code(x0[8 * s2 + gq], 0) << (2 * s2);
+                    acc += code(x1[8 * s2 + gq], 1) << (2 * (4 + s2));
                 }
                 if (row >= 0)
                     *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 2, tok, gq, 0)) =
@@ -377,8 +307,8 @@ __device__ __forceinline__ bool store_row64(const TcParams &P, int which, long l
                 uint32_t a0 = 0u - magic_sum(4, 4), a1 = a0;
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
-                    a0 += code(x0[8 * s2 + gq], 0, s2) << (4 * s2);
-                    a1 += code(x1[8 * s2 + gq], 1, s2 + 2) << (4 * s2);
+                    a0 += code(x0[8 * s2 + gq], 0) << (4 * s2);
+                    a1 += code(x1[8 * s2 + gq], 1) << (4 * s2);
                 }
                 if (row >= 0) {
                     *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 4, tok, gq, 0)) =
@@ -389,7 +319,6 @@ __device__ __forceinline__ bool store_row64(const TcParams &P, int which, long l
             }
         }
     }
-    return tie;
 }
 
 // Running clip statistics of one group of a row: kappa = 0 (min, max), kappa = 1 (second
@@ -601,7 +530,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         // r of warp quarter q owns TMEM lane (token row) 32 q + r. Two passes over the row:
         // the clip parameters of every group, then the codes (d = 64: the whole row held in
         // registers; d = 128: 32 columns at a time from TMEM). The buffer is released after
-        // the row is done, so a row near a rounding tie can be recoded with IEEE division.
+        // the row is done.
         const int wg = warp / 4, quarter = warp % 4;
         const int r = quarter * 32 + lane;
         const float qmax = (float)((1u << bits) - 1u);
@@ -634,12 +563,9 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * D);
             // ---- pass 1: clip parameters per group (every lane takes part in the loads)
             float zf[NG], sf[NG], rc[NG];
-            bool zero[NG];
 #pragma unroll
-            for (int gg = 0; gg < NG; ++gg) {
+            for (int gg = 0; gg < NG; ++gg)
                 zf[gg] = sf[gg] = rc[gg] = 0.f;
-                zero[gg] = true;
-            }
             ClipStats cs;
             cs.reset(P.clip);
             // group gr is complete: its scale and zero-point, stored with the row
@@ -669,7 +595,6 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     if (gg == gr) {
                         sf[gg] = sfv;
                         zf[gg] = zfv;
-                        zero[gg] = zr;
                         rc[gg] = rcv;
                     }
                 if (row >= 0) {
@@ -681,8 +606,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 cs.reset(P.clip);                           // the next group starts fresh
             };
             if constexpr (D == 64) {
-                // the whole row in registers: one TMEM round trip, both passes (and the
-                // exact redo of a row near a tie) from registers
+                // the whole row in registers: one TMEM round trip for both passes
                 uint32_t x0[32], x1[32];
                 tmem_ld32_async(taddr, x0);
                 tmem_ld32_async(taddr + 32, x1);
@@ -694,25 +618,10 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 finish(NG - 1);
                 const float z2[2] = {zf[0], zf[NG - 1]}, s2[2] = {sf[0], sf[NG - 1]};
                 const float r2[2] = {rc[0], rc[NG - 1]};
-                const bool zr2[2] = {zero[0], zero[NG - 1]};
-                const bool tie = bits == 2
-                    ? store_row64<2, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax)
-                    : store_row64<4, false>(P, which, row, x0, x1, z2, s2, r2, zr2, qmax);
-                // Rare: a row near a rounding tie. The whole warp reloads its rows from TMEM
-                // (the accumulator is still held; the load is warp-collective) and the rows
-                // with a tie are stored again with the IEEE quotient for those values. The
-                // reload lets the registers of the first pass die as its codes are formed.
-                if (__any_sync(0xffffffffu, tie)) {
-                    uint32_t y0[32], y1[32];
-                    tmem_ld32_async(taddr, y0);
-                    tmem_ld32_async(taddr + 32, y1);
-                    tmem_ld_wait();
-                    const long long rw = tie ? row : -1;
-                    if (bits == 2)
-                        store_row64<2, true>(P, which, rw, y0, y1, z2, s2, r2, zr2, qmax);
-                    else
-                        store_row64<4, true>(P, which, rw, y0, y1, z2, s2, r2, zr2, qmax);
-                }
+                if (bits == 2)
+                    store_row64<2>(P, which, row, x0, x1, z2, s2, r2, qmax);
+                else
+                    store_row64<4>(P, which, row, x0, x1, z2, s2, r2, qmax);
             } else {
                 uint32_t cur[32];
 #pragma unroll 1
@@ -723,28 +632,17 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     if ((32 * c + 32) % GS == 0)          // the group ends with this chunk
                         finish((32 * c) / GS);
                 }
-                // ---- pass 2: codes; pass 3 (rows near a rounding tie only): the same by
-                //      division
-                bool tie;
-                if (!which)
-                    tie = bits == 2 ? store_codes<D, GS, NG, 2, false, false>(P, row, taddr, zf, sf, rc, zero, qmax)
-                                    : store_codes<D, GS, NG, 4, false, false>(P, row, taddr, zf, sf, rc, zero, qmax);
-                else
-                    tie = bits == 2 ? store_codes<D, GS, NG, 2, true, false>(P, row, taddr, zf, sf, rc, zero, qmax)
-                                    : store_codes<D, GS, NG, 4, true, false>(P, row, taddr, zf, sf, rc, zero, qmax);
-                if (__any_sync(0xffffffffu, tie)) {
-                    const long long rw = tie ? row : -1;
-                    if (!which) {
-                        if (bits == 2)
-                            store_codes<D, GS, NG, 2, false, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
-                        else
-                            store_codes<D, GS, NG, 4, false, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
-                    } else {
-                        if (bits == 2)
-                            store_codes<D, GS, NG, 2, true, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
-                        else
-                            store_codes<D, GS, NG, 4, true, true>(P, rw, taddr, zf, sf, rc, zero, qmax);
-                    }
+                // ---- pass 2: codes
+                if (!which) {
+                    if (bits == 2)
+                        store_codes<D, GS, NG, 2, false>(P, row, taddr, zf, sf, rc, qmax);
+                    else
+                        store_codes<D, GS, NG, 4, false>(P, row, taddr, zf, sf, rc, qmax);
+                } else {
+                    if (bits == 2)
+                        store_codes<D, GS, NG, 2, true>(P, row, taddr, zf, sf, rc, qmax);
+                    else
+                        store_codes<D, GS, NG, 4, true>(P, row, taddr, zf, sf, rc, qmax);
                 }
             }
             tc_fence_before_sync();
