@@ -109,6 +109,40 @@ __device__ __forceinline__ uint32_t code_rn(uint32_t xb, float zf, float sf, flo
     return __float_as_uint(__fadd_rn(y, kRoundMagic));
 }
 
+// Two values at a time on the paired float32 instructions of sm_100 (add/mul/fma .f32x2;
+// each lane of a pair is an ordinary IEEE float32 operation, so the codes equal code_rn's):
+// (ca, cb) = code_rn of xa with the parameters (za, sa, ra) and of xb with (zb, sb, rb),
+// given as pairs nz = (-za, -zb), sb2 = (sa, sb), nsb2 = (-sa, -sb), rc2 = (ra, rb).
+__device__ __forceinline__ uint64_t f2pack(uint32_t a, uint32_t b)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ void f2unpack(uint64_t v, uint32_t &a, uint32_t &b)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v));
+}
+
+__device__ __forceinline__ void code_rn2(uint32_t xa, uint32_t xb, uint64_t nz, uint64_t nsb2,
+                                         uint64_t rc2, float qmax, uint32_t &ca, uint32_t &cb)
+{
+    uint64_t a, q0, r, q, m;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(a) : "l"(f2pack(xa, xb)), "l"(nz));      // x - z
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q0) : "l"(a), "l"(rc2));                 // RN(a y)
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(q0), "l"(nsb2), "l"(a));    // a - q0 s
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(r), "l"(rc2), "l"(q0));     // q0 + r y
+    uint32_t qa, qb;
+    f2unpack(q, qa, qb);
+    const float ya = fminf(fmaxf(__uint_as_float(qa), 0.f), qmax);
+    const float yb = fminf(fmaxf(__uint_as_float(qb), 0.f), qmax);
+    const uint64_t magic2 = ((uint64_t)__float_as_uint(kRoundMagic) << 32) | __float_as_uint(kRoundMagic);
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(m) : "l"(f2pack(__float_as_uint(ya), __float_as_uint(yb))),
+        "l"(magic2));
+    f2unpack(m, ca, cb);
+}
+
 // sum over e < N of 0x4B400000 * 2^(B*e), modulo 2^32: what packing N magic-rounded codes
 // with multiply-adds leaves above the codes themselves
 __host__ __device__ constexpr uint32_t magic_sum(int B, int N)
@@ -256,11 +290,16 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
                                             const float (&z)[2], const float (&sc)[2],
                                             const float (&rc)[2], float qmax)
 {
-    auto code = [&](uint32_t xb, int hf) -> uint32_t {
-        return code_rn(xb, z[hf], sc[hf], rc[hf], qmax);
+    auto pair = [](float a, float b) {
+        return ((uint64_t)__float_as_uint(b) << 32) | __float_as_uint(a);
     };
+    // parameter pairs: (half 0, half 0), (half 1, half 1) and (half 0, half 1)
+    const uint64_t nz00 = pair(-z[0], -z[0]), nz11 = pair(-z[1], -z[1]), nz01 = pair(-z[0], -z[1]);
+    const uint64_t ns00 = pair(-sc[0], -sc[0]), ns11 = pair(-sc[1], -sc[1]),
+                   ns01 = pair(-sc[0], -sc[1]);
+    const uint64_t rc00 = pair(rc[0], rc[0]), rc11 = pair(rc[1], rc[1]), rc01 = pair(rc[0], rc[1]);
     if (!which) {
-        // word q of a 32-dim half: dims (32/BITS) q + e at BITS*e
+        // word q of a 32-dim half: dims (32/BITS) q + e at BITS*e; codes two at a time
         constexpr int PER = 32 / BITS;
         uint32_t w[2][BITS];
 #pragma unroll
@@ -269,8 +308,14 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
             for (int q = 0; q < BITS; ++q) {
                 uint32_t acc = 0u - magic_sum(BITS, PER);
 #pragma unroll
-                for (int e = 0; e < PER; ++e)
-                    acc += code(hf ? x1[PER * q + e] : x0[PER * q + e], hf) << (BITS * e);
+                for (int e = 0; e < PER; e += 2) {
+                    const uint32_t xa = hf ? x1[PER * q + e] : x0[PER * q + e];
+                    const uint32_t xb = hf ? x1[PER * q + e + 1] : x0[PER * q + e + 1];
+                    uint32_t ca, cb;
+                    code_rn2(xa, xb, hf ? nz11 : nz00, hf ? ns11 : ns00, hf ? rc11 : rc00, qmax,
+                             ca, cb);
+                    acc += (ca << (BITS * e)) + (cb << (BITS * (e + 1)));
+                }
                 w[hf][q] = acc;
             }
         if (row >= 0) {
@@ -296,8 +341,9 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
                 uint32_t acc = 0u - magic_sum(2, 8);
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
-                    acc += code(x0[8 * s2 + gq], 0) << (2 * s2);
-                    acc += code(x1[8 * s2 + gq], 1) << (2 * (4 + s2));
+                    uint32_t ca, cb;
+                    code_rn2(x0[8 * s2 + gq], x1[8 * s2 + gq], nz01, ns01, rc01, qmax, ca, cb);
+                    acc += (ca << (2 * s2)) + (cb << (2 * (4 + s2)));
                 }
                 if (row >= 0)
                     *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 2, tok, gq, 0)) =
@@ -307,8 +353,10 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
                 uint32_t a0 = 0u - magic_sum(4, 4), a1 = a0;
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
-                    a0 += code(x0[8 * s2 + gq], 0) << (4 * s2);
-                    a1 += code(x1[8 * s2 + gq], 1) << (4 * s2);
+                    uint32_t ca, cb;
+                    code_rn2(x0[8 * s2 + gq], x1[8 * s2 + gq], nz01, ns01, rc01, qmax, ca, cb);
+                    a0 += ca << (4 * s2);
+                    a1 += cb << (4 * s2);
                 }
                 if (row >= 0) {
                     *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 4, tok, gq, 0)) =
