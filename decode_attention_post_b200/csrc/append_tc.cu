@@ -102,17 +102,12 @@ __device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar)
 constexpr float kRoundMagic = 12582912.0f;        // 1.5 * 2^23
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 
-__device__ __forceinline__ uint32_t code_rn(uint32_t xb, float zf, float sf, float rc, float qmax)
-{
-    float y = div_rn(__fsub_rn(__uint_as_float(xb), zf), sf, rc);
-    y = fminf(fmaxf(y, 0.f), qmax);
-    return __float_as_uint(__fadd_rn(y, kRoundMagic));
-}
-
-// Two values at a time on the paired float32 instructions of sm_100 (add/mul/fma .f32x2;
-// each lane of a pair is an ordinary IEEE float32 operation, so the codes equal code_rn's):
-// (ca, cb) = code_rn of xa with the parameters (za, sa, ra) and of xb with (zb, sb, rb),
-// given as pairs nz = (-za, -zb), sb2 = (sa, sb), nsb2 = (-sa, -sb), rc2 = (ra, rb).
+// Two codes at a time on the paired float32 instructions of sm_100 (add/mul/fma .f32x2;
+// each lane of a pair is an ordinary IEEE float32 operation): the bits 0x4B400000 + c of
+// the code of xa with the parameters (za, sa, ra = RN(1/sa)) and of xb with (zb, sb, rb),
+// given as pairs nz = (-za, -zb), nsb2 = (-sa, -sb), rc2 = (ra, rb): x - z, the quotient
+// by div_rn's steps (RN(a y), the exact residual, one correction), the clamp, the magic
+// addition. The first element of a pair is its low 32 bits.
 __device__ __forceinline__ uint64_t f2pack(uint32_t a, uint32_t b)
 {
     uint64_t r;
@@ -200,18 +195,27 @@ __device__ __forceinline__ float pick(const float (&a)[NG], int gr)
 // Codes of 32 consecutive dims (column c0.. of the row) packed as BITS-bit fields of
 // 32-bit words: `words` words, field e of word q = dim c0 + (32/BITS) q + e.
 template <int BITS>
-__device__ __forceinline__ void pack32(const uint32_t (&x)[32], float zf, float sf, float rc,
-                                       float qmax, uint32_t (&w)[BITS])
+__device__ __forceinline__ void pack32(const uint32_t (&x)[32], uint64_t nz2, uint64_t ns2,
+                                       uint64_t rc2, float qmax, uint32_t (&w)[BITS])
 {
     constexpr int PER = 32 / BITS;                  // codes per word
 #pragma unroll
     for (int q = 0; q < BITS; ++q) {
         uint32_t acc = 0u - magic_sum(BITS, PER);
 #pragma unroll
-        for (int e = 0; e < PER; ++e)
-            acc += code_rn(x[PER * q + e], zf, sf, rc, qmax) << (BITS * e);
+        for (int e = 0; e < PER; e += 2) {
+            uint32_t ca, cb;
+            code_rn2(x[PER * q + e], x[PER * q + e + 1], nz2, ns2, rc2, qmax, ca, cb);
+            acc += (ca << (BITS * e)) + (cb << (BITS * (e + 1)));
+        }
         w[q] = acc;
     }
+}
+
+// (a, a) as a float32 pair
+__device__ __forceinline__ uint64_t f2dup(float a)
+{
+    return ((uint64_t)__float_as_uint(a) << 32) | __float_as_uint(a);
 }
 
 // One token's codes from its TMEM row, 32 columns per iteration (the other warps of the
@@ -237,10 +241,11 @@ __device__ __forceinline__ void store_codes(const TcParams &P, long long row, ui
         tmem_ld32_async(taddr + 32 * c, cur);
         tmem_ld_wait();
         const int gr = (32 * c) / GS;
-        const float z = pick(zf, gr), s = pick(sf, gr), r = pick(rc, gr);
+        const uint64_t nz2 = f2dup(-pick(zf, gr)), ns2 = f2dup(-pick(sf, gr)),
+                       rc2 = f2dup(pick(rc, gr));
         if (!V) {
             uint32_t w[BITS];
-            pack32<BITS>(cur, z, s, r, qmax, w);
+            pack32<BITS>(cur, nz2, ns2, rc2, qmax, w);
             if (row >= 0) {
                 uint32_t *dst = reinterpret_cast<uint32_t *>(P.k_codes + row * (D * BITS / 8)) + BITS * c;
                 if (BITS == 2)
@@ -260,8 +265,11 @@ __device__ __forceinline__ void store_codes(const TcParams &P, long long row, ui
             for (int gq = 0; gq < 8; ++gq) {
                 uint32_t acc = 0u - (magic_sum(BITS, 4) << (BITS * base));
 #pragma unroll
-                for (int n8 = 0; n8 < 4; ++n8)
-                    acc += code_rn(cur[8 * n8 + gq], z, s, r, qmax) << (BITS * (base + n8));
+                for (int n8 = 0; n8 < 4; n8 += 2) {
+                    uint32_t ca, cb;
+                    code_rn2(cur[8 * n8 + gq], cur[8 * (n8 + 1) + gq], nz2, ns2, rc2, qmax, ca, cb);
+                    acc += (ca << (BITS * (base + n8))) + (cb << (BITS * (base + n8 + 1)));
+                }
                 hv[gq] = acc;
             }
             if (row >= 0) {
