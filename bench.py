@@ -434,6 +434,7 @@ def run_gpu(args):
         del w
         torch.cuda.empty_cache()
         line["chunk_append"] = chunk_append(device, stream)
+        line["chunk_append_d128"] = chunk_append(device, stream, d128=True)
         line["append_config0"] = append_config0(device, stream)
         line["decode_configs"] = [decode_config_line(i, device, stream, peak)
                                   for i in DECODE_CONFIGS]
@@ -694,12 +695,17 @@ def vq_decode(w, cfg, stream, dec_ms, peak):
     return res
 
 
-def chunk_append(device, stream):
-    """32768-token chunk append of the GPT-OSS-20B-like shape (batch 8, 8 KV heads, d 64)."""
+def chunk_append(device, stream, d128=False):
+    """32768-token chunk append of the GPT-OSS-20B-like shape (batch 8, 8 KV heads, d 64);
+    d128: a 16384-token chunk of the Qwen3-8B-like heads (batch 8, 8 KV heads, d 128)."""
     import torch
     import decode_attention_post_b200 as kvq
-    cfg = synth.CONFIGS[APPEND_CONFIG_IDX]
-    n = cfg.append_n
+    if d128:
+        cfg = synth.CONFIGS[CONFIG_IDX].with_(B=8)
+        n = 16384
+    else:
+        cfg = synth.CONFIGS[APPEND_CONFIG_IDX]
+        n = cfg.append_n
     qp = kvq.QParams(cfg.bits_k, cfg.bits_v, cfg.group, cfg.clip_alpha)
     cache = kvq.KVCache.allocate(cfg.B, cfg.Hkv, cfg.T_cap, cfg.d, qp, device=device)
     Tk, Tv, _ = synth.transforms(cfg)
@@ -716,7 +722,8 @@ def chunk_append(device, stream):
     nbytes = tokheads * (2 * cfg.d * 2 + cfg.d * (cfg.bits_k + cfg.bits_v) // 8 + 8 * ng) + \
         2 * cfg.Hkv * cfg.d * cfg.d * 4
     flops = tokheads * 4 * cfg.d * cfg.d
-    return {"workload": cfg.name, "ms": round(ms, 4),
+    return {"workload": cfg.name if not d128 else "qwen3-8b-like-b8-d128-append16k",
+            "ms": round(ms, 4),
             "tok_per_s": round(cfg.B * n / (ms * 1e-3), 1),
             "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
             "TFLOP_s": round(flops / (ms * 1e-3) / 1e12, 2), "bytes": nbytes}
@@ -843,6 +850,8 @@ def profile_case(name):
     peak, _ = peaks()
     if name == "chunk_append":
         res = chunk_append(device, stream)
+    elif name == "chunk_append_d128":
+        res = chunk_append(device, stream, d128=True)
     elif name == "append_config0":
         res = append_config0(device, stream)
     elif name.startswith("decode_config"):
@@ -894,7 +903,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--profile-case", default=None,
-                    help="run one kernel's workload alone (chunk_append, append_config0, "
+                    help="run one kernel's workload alone (chunk_append, chunk_append_d128, "
+                         "append_config0, "
                          "decode_config1/2/3/4, bf16_config1, vq_config1, window_config1) "
                          "for an ncu capture")
     args = ap.parse_args()
