@@ -192,7 +192,11 @@ __device__ __forceinline__ void quantize_store_token(const float (&vals)[D / 32]
             const float lo = order_stat<R, false>(vmin, kappa, lane);
             const float hi = order_stat<R, true>(vmax, kappa, lane);
             const float range = __fsub_rn(hi, lo);
-            const float s = __fdiv_rn(range, (float)qmax);
+            // range / qmax correctly rounded (div_rn; tiny or non-finite ranges, outside
+            // its conditions, by IEEE division)
+            const float s = (range >= 0x1p-100f && range <= 0x1p+100f)
+                                ? div_rn(range, (float)qmax, __frcp_rn((float)qmax))
+                                : __fdiv_rn(range, (float)qmax);
             sh = __float2half_rn(s);
             zh = __float2half_rn(lo);
             finite = isfinite(range) && isfinite(s);

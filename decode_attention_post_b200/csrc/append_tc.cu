@@ -590,6 +590,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const int wg = warp / 4, quarter = warp % 4;
         const int r = quarter * 32 + lane;
         const float qmax = (float)((1u << bits) - 1u);
+        const float rqmax = __frcp_rn(qmax);
         const bool quest = P.clip == kQuestClip;
         for (int k = wg; k < my_tiles; k += C::EPI) {
             const int a = k % C::EPI;
@@ -638,7 +639,11 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     float glo, ghi;
                     cs.range(P.clip, glo, ghi);
                     const float range = __fsub_rn(ghi, glo);
-                    const float sv = __fdiv_rn(range, qmax);
+                    // range / qmax correctly rounded (div_rn; tiny or non-finite ranges,
+                    // outside its conditions, by IEEE division)
+                    const float sv = (range >= 0x1p-100f && range <= 0x1p+100f)
+                                         ? div_rn(range, qmax, rqmax)
+                                         : __fdiv_rn(range, qmax);
                     sh = __float2half_rn(sv);
                     zh = __float2half_rn(glo);
                     finite = isfinite(range) && isfinite(sv);
