@@ -365,7 +365,7 @@ __device__ __forceinline__ void merge_if_last(const DecodeParams &P, size_t pair
     }
 }
 
-// WIN: the grid has one more split per pair, the full-precision window's (split nsplit);
+// WIN: the grid has one more split per pair, the full-precision window's (slice z = 0);
 // a separate instantiation, so that the plain decode carries none of its code.
 template <int D, int G, int BK, int BV, bool WIN>
 __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) decode_kernel(DecodeParams P)
@@ -377,7 +377,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
     uint64_t *stall_bars = bars_all + kDecodeWarps * kDecodeStages;
     int *flag_smem = reinterpret_cast<int *>(stall_bars + kDecodeWarps);
 
-    const int h = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
+    // with a window, grid slice z = 0 is the window split (often the pair's longest CTA: it
+    // starts first) and z = 1 + sigma the quantized split sigma
+    const int h = blockIdx.x, b = blockIdx.y, sigma = (int)blockIdx.z - (WIN ? 1 : 0);
     const int lane = threadIdx.x & 31;
     // the warp index through a broadcast shuffle: the compiler then knows it is the same
     // in every lane, keeps the ring and copy addresses in uniform registers and issues the
@@ -393,7 +395,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
 
     int seqlen = P.seqlens[b];
     if (seqlen < 0 || seqlen > P.max_seqlen) {
-        if (sigma == 0 && h == 0 && threadIdx.x == 0)
+        if (blockIdx.z == 0 && h == 0 && threadIdx.x == 0)
             flag(P.dev_err, KVQ_DEVERR_SEQLEN_CLAMPED);
         seqlen = seqlen < 0 ? 0 : P.max_seqlen;
     }
@@ -403,7 +405,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (Cfg<D, G, BK, BV>::MINB)) 
         seqlen = window_quantized(seqlen, P.win_sink, P.win_keep, P.win_flush);
     const int nsplit_b = (seqlen + P.split_tokens - 1) / P.split_tokens;
     const int nmerge = nsplit_b + (windowed ? 1 : 0);   // partials merged for the pair
-    if (WIN && sigma == P.nsplit) {
+    if (WIN && sigma < 0) {
         // ---- the window split: its partial in the last slot, or the output when nothing
         //      of the sequence is quantized
         if (L_all == 0)
@@ -815,8 +817,8 @@ cudaError_t launch_decode_t(const DecodeLaunch &L, cudaStream_t st)
             return e;
     }
     // decode: CTA (KV head, sequence, split), splits slowest so that the short last
-    // splits of the sequences run last, then the window splits (split nsplit) when there is
-    // a full-precision window; a programmatic dependent of qprep
+    // splits of the sequences run last; with a full-precision window its split comes first
+    // (slice z = 0); a programmatic dependent of qprep
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(L.p.Hkv, L.p.B, L.p.nsplit + (win ? 1 : 0));
     cfg.blockDim = dim3(kDecodeWarps * 32);

@@ -35,8 +35,8 @@ struct DecodeParams {
     int part_slots;             // partial slots per (sequence, KV head): split slots
                                 // (>= nsplit) + 1, the last one for the window's partial
     // full-precision window (win_flush = 0: none): the cache holds the quantized middle,
-    // seqlens are whole lengths; split nsplit of every pair attends over the window and
-    // its partial goes to the last slot
+    // seqlens are whole lengths; one more CTA per pair (grid slice z = 0) attends over the
+    // window and its partial goes to the last slot
     int win_sink, win_keep, win_flush;
     const void *win_q;                                  // bfloat16 [B][Hq][d], as given
     const void *k_sink, *v_sink, *k_recent, *v_recent;  // bfloat16 window rows
