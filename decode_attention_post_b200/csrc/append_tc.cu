@@ -105,9 +105,10 @@ constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 // Two codes at a time on the paired float32 instructions of sm_100 (add/mul/fma .f32x2;
 // each lane of a pair is an ordinary IEEE float32 operation): the bits 0x4B400000 + c of
 // the code of xa with the parameters (za, sa, ra = RN(1/sa)) and of xb with (zb, sb, rb),
-// given as pairs nz = (-za, -zb), nsb2 = (-sa, -sb), rc2 = (ra, rb): x - z, the quotient
-// by div_rn's steps (RN(a y), the exact residual, one correction), the clamp, the magic
-// addition. The first element of a pair is its low 32 bits.
+// given as pairs nz = (-za, -zb), nsb2 = (-sa, -sb), rc2 = (ra, rb): x - z and the
+// quotient by div_rn's steps (RN(a y), the exact residual, one correction) on pairs, then
+// per value the clamp and the magic addition. The first element of a pair is its low 32
+// bits; callers pair adjacent registers (no moves to build the pairs).
 __device__ __forceinline__ uint64_t f2pack(uint32_t a, uint32_t b)
 {
     uint64_t r;
@@ -123,7 +124,7 @@ __device__ __forceinline__ void f2unpack(uint64_t v, uint32_t &a, uint32_t &b)
 __device__ __forceinline__ void code_rn2(uint32_t xa, uint32_t xb, uint64_t nz, uint64_t nsb2,
                                          uint64_t rc2, float qmax, uint32_t &ca, uint32_t &cb)
 {
-    uint64_t a, q0, r, q, m;
+    uint64_t a, q0, r, q;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(a) : "l"(f2pack(xa, xb)), "l"(nz));      // x - z
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q0) : "l"(a), "l"(rc2));                 // RN(a y)
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(q0), "l"(nsb2), "l"(a));    // a - q0 s
@@ -132,10 +133,8 @@ __device__ __forceinline__ void code_rn2(uint32_t xa, uint32_t xb, uint64_t nz, 
     f2unpack(q, qa, qb);
     const float ya = fminf(fmaxf(__uint_as_float(qa), 0.f), qmax);
     const float yb = fminf(fmaxf(__uint_as_float(qb), 0.f), qmax);
-    const uint64_t magic2 = ((uint64_t)__float_as_uint(kRoundMagic) << 32) | __float_as_uint(kRoundMagic);
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(m) : "l"(f2pack(__float_as_uint(ya), __float_as_uint(yb))),
-        "l"(magic2));
-    f2unpack(m, ca, cb);
+    ca = __float_as_uint(__fadd_rn(ya, kRoundMagic));
+    cb = __float_as_uint(__fadd_rn(yb, kRoundMagic));
 }
 
 // sum over e < N of 0x4B400000 * 2^(B*e), modulo 2^32: what packing N magic-rounded codes
@@ -192,26 +191,6 @@ __device__ __forceinline__ float pick(const float (&a)[NG], int gr)
 }
 
 
-// Codes of 32 consecutive dims (column c0.. of the row) packed as BITS-bit fields of
-// 32-bit words: `words` words, field e of word q = dim c0 + (32/BITS) q + e.
-template <int BITS>
-__device__ __forceinline__ void pack32(const uint32_t (&x)[32], uint64_t nz2, uint64_t ns2,
-                                       uint64_t rc2, float qmax, uint32_t (&w)[BITS])
-{
-    constexpr int PER = 32 / BITS;                  // codes per word
-#pragma unroll
-    for (int q = 0; q < BITS; ++q) {
-        uint32_t acc = 0u - magic_sum(BITS, PER);
-#pragma unroll
-        for (int e = 0; e < PER; e += 2) {
-            uint32_t ca, cb;
-            code_rn2(x[PER * q + e], x[PER * q + e + 1], nz2, ns2, rc2, qmax, ca, cb);
-            acc += (ca << (BITS * e)) + (cb << (BITS * (e + 1)));
-        }
-        w[q] = acc;
-    }
-}
-
 // (a, a) as a float32 pair
 __device__ __forceinline__ uint64_t f2dup(float a)
 {
@@ -243,9 +222,22 @@ __device__ __forceinline__ void store_codes(const TcParams &P, long long row, ui
         const int gr = (32 * c) / GS;
         const uint64_t nz2 = f2dup(-pick(zf, gr)), ns2 = f2dup(-pick(sf, gr)),
                        rc2 = f2dup(pick(rc, gr));
+        // the chunk's 32 codes (magic bit patterns), two adjacent values at a time
+        uint32_t cc[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+            code_rn2(cur[e], cur[e + 1], nz2, ns2, rc2, qmax, cc[e], cc[e + 1]);
         if (!V) {
             uint32_t w[BITS];
-            pack32<BITS>(cur, nz2, ns2, rc2, qmax, w);
+            constexpr int PER = 32 / BITS;
+#pragma unroll
+            for (int q = 0; q < BITS; ++q) {
+                uint32_t acc = 0u - magic_sum(BITS, PER);
+#pragma unroll
+                for (int e = 0; e < PER; ++e)
+                    acc += cc[PER * q + e] << (BITS * e);
+                w[q] = acc;
+            }
             if (row >= 0) {
                 uint32_t *dst = reinterpret_cast<uint32_t *>(P.k_codes + row * (D * BITS / 8)) + BITS * c;
                 if (BITS == 2)
@@ -265,11 +257,8 @@ __device__ __forceinline__ void store_codes(const TcParams &P, long long row, ui
             for (int gq = 0; gq < 8; ++gq) {
                 uint32_t acc = 0u - (magic_sum(BITS, 4) << (BITS * base));
 #pragma unroll
-                for (int n8 = 0; n8 < 4; n8 += 2) {
-                    uint32_t ca, cb;
-                    code_rn2(cur[8 * n8 + gq], cur[8 * (n8 + 1) + gq], nz2, ns2, rc2, qmax, ca, cb);
-                    acc += (ca << (BITS * (base + n8))) + (cb << (BITS * (base + n8 + 1)));
-                }
+                for (int n8 = 0; n8 < 4; ++n8)
+                    acc += cc[8 * n8 + gq] << (BITS * (base + n8));
                 hv[gq] = acc;
             }
             if (row >= 0) {
@@ -301,13 +290,21 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
     auto pair = [](float a, float b) {
         return ((uint64_t)__float_as_uint(b) << 32) | __float_as_uint(a);
     };
-    // parameter pairs: (half 0, half 0), (half 1, half 1) and (half 0, half 1)
-    const uint64_t nz00 = pair(-z[0], -z[0]), nz11 = pair(-z[1], -z[1]), nz01 = pair(-z[0], -z[1]);
-    const uint64_t ns00 = pair(-sc[0], -sc[0]), ns11 = pair(-sc[1], -sc[1]),
-                   ns01 = pair(-sc[0], -sc[1]);
-    const uint64_t rc00 = pair(rc[0], rc[0]), rc11 = pair(rc[1], rc[1]), rc01 = pair(rc[0], rc[1]);
+    // the 64 codes (magic bit patterns), two adjacent values at a time, half 0 then half 1
+    uint32_t c0[32], c1[32];
+    {
+        const uint64_t nz0 = pair(-z[0], -z[0]), ns0 = pair(-sc[0], -sc[0]),
+                       r0 = pair(rc[0], rc[0]);
+        const uint64_t nz1 = pair(-z[1], -z[1]), ns1 = pair(-sc[1], -sc[1]),
+                       r1 = pair(rc[1], rc[1]);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            code_rn2(x0[e], x0[e + 1], nz0, ns0, r0, qmax, c0[e], c0[e + 1]);
+            code_rn2(x1[e], x1[e + 1], nz1, ns1, r1, qmax, c1[e], c1[e + 1]);
+        }
+    }
     if (!which) {
-        // word q of a 32-dim half: dims (32/BITS) q + e at BITS*e; codes two at a time
+        // word q of a 32-dim half: dims (32/BITS) q + e at BITS*e
         constexpr int PER = 32 / BITS;
         uint32_t w[2][BITS];
 #pragma unroll
@@ -316,14 +313,8 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
             for (int q = 0; q < BITS; ++q) {
                 uint32_t acc = 0u - magic_sum(BITS, PER);
 #pragma unroll
-                for (int e = 0; e < PER; e += 2) {
-                    const uint32_t xa = hf ? x1[PER * q + e] : x0[PER * q + e];
-                    const uint32_t xb = hf ? x1[PER * q + e + 1] : x0[PER * q + e + 1];
-                    uint32_t ca, cb;
-                    code_rn2(xa, xb, hf ? nz11 : nz00, hf ? ns11 : ns00, hf ? rc11 : rc00, qmax,
-                             ca, cb);
-                    acc += (ca << (BITS * e)) + (cb << (BITS * (e + 1)));
-                }
+                for (int e = 0; e < PER; ++e)
+                    acc += (hf ? c1[PER * q + e] : c0[PER * q + e]) << (BITS * e);
                 w[hf][q] = acc;
             }
         if (row >= 0) {
@@ -345,26 +336,21 @@ __device__ __forceinline__ void store_row64(const TcParams &P, int which, long l
 #pragma unroll
         for (int gq = 0; gq < 8; ++gq) {
             if constexpr (BITS == 2) {
-                // one half per gq: s < 4 from x0 (dim gq + 8 s), s >= 4 from x1
+                // one half per gq: s < 4 from half 0 (dim gq + 8 s), s >= 4 from half 1
                 uint32_t acc = 0u - magic_sum(2, 8);
 #pragma unroll
-                for (int s2 = 0; s2 < 4; ++s2) {
-                    uint32_t ca, cb;
-                    code_rn2(x0[8 * s2 + gq], x1[8 * s2 + gq], nz01, ns01, rc01, qmax, ca, cb);
-                    acc += (ca << (2 * s2)) + (cb << (2 * (4 + s2)));
-                }
+                for (int s2 = 0; s2 < 4; ++s2)
+                    acc += (c0[8 * s2 + gq] << (2 * s2)) + (c1[8 * s2 + gq] << (2 * (4 + s2)));
                 if (row >= 0)
                     *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 2, tok, gq, 0)) =
                         (uint16_t)acc;
             } else {
-                // halves rr = 0 (x0) and rr = 1 (x1), s < 4: dim gq + 8 (4 rr + s)
+                // halves rr = 0 (half 0) and rr = 1 (half 1), s < 4: dim gq + 8 (4 rr + s)
                 uint32_t a0 = 0u - magic_sum(4, 4), a1 = a0;
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
-                    uint32_t ca, cb;
-                    code_rn2(x0[8 * s2 + gq], x1[8 * s2 + gq], nz01, ns01, rc01, qmax, ca, cb);
-                    a0 += ca << (4 * s2);
-                    a1 += cb << (4 * s2);
+                    a0 += c0[8 * s2 + gq] << (4 * s2);
+                    a1 += c1[8 * s2 + gq] << (4 * s2);
                 }
                 if (row >= 0) {
                     *reinterpret_cast<uint16_t *>(vbase + v_half_offset(64, 4, tok, gq, 0)) =
