@@ -26,10 +26,11 @@ constexpr int kCapAlign = 64;        // T_cap granularity (whole decode blocks)
 // Dev. 34(1), 1990): q0 = RN(a y) is within an ulp of a/b, the residual r = a - q0 b is
 // exact in one fused multiply-add, and RN(q0 + r y) is RN(a / b) when nothing overflows or
 // underflows -- here b is a positive float16 scale (a normal float32 number) and |a / b|
-// stays far inside the float32 range. No branch and no call, so it can run for every value of a row; the
-// quantizers then need no tie test (checked against IEEE division on the B200 over 1.2e9
-// operand pairs, half of them within a few ulps of a rounding tie, and by the bit-exact
-// parity tests).
+// stays far inside the float32 range. No branch and no call, so it can run for every
+// value of a row; the quantizers then need no tie test (tests/test_division_method.py
+// carries out these steps in exact arithmetic against the correctly rounded quotient, on
+// random and near-tie operands; the append parity tests compare every code with the
+// oracle's).
 __device__ __forceinline__ float div_rn(float a, float b, float y)
 {
     const float q0 = __fmul_rn(a, y);
