@@ -197,18 +197,48 @@ __device__ __forceinline__ uint64_t f2dup(float a)
     return ((uint64_t)__float_as_uint(a) << 32) | __float_as_uint(a);
 }
 
-// One token's codes from its TMEM row, 32 columns per iteration (the other warps of the
-// SM hide the load latency), stored as the K row (little-endian bit stream, dim j at
-// bit BITS*j) or as the token's halves of its 16-token V tile (half (gq, rr) holds dims
-// 8(E rr + s) + gq at BITS*s, E = 16/BITS). row < 0: codes not stored (the warp still
-// takes part in the TMEM loads).
+// The 32 codes (magic bit patterns) of chunk c (dims 32c .. 32c + 31) of a row, two
+// adjacent values at a time, with the parameters of the chunk's group.
+template <int GS, int NG>
+__device__ __forceinline__ void chunk_codes(const uint32_t (&cur)[32], int c,
+                                            const float (&zf)[NG], const float (&sf)[NG],
+                                            const float (&rc)[NG], float qmax, uint32_t (&cc)[32])
+{
+    const int gr = (32 * c) / GS;
+    const uint64_t nz2 = f2dup(-pick(zf, gr)), ns2 = f2dup(-pick(sf, gr)), rc2 = f2dup(pick(rc, gr));
+#pragma unroll
+    for (int e = 0; e < 32; e += 2)
+        code_rn2(cur[e], cur[e + 1], nz2, ns2, rc2, qmax, cc[e], cc[e + 1]);
+}
+
+// Value-tile halves from one chunk's codes: the chunk's dims are 32c + 8 n8 + gq (n8 < 4,
+// gq < 8), and half (gq, rr) holds dims 8(E rr + s) + gq at bits BITS*s, E = 16/BITS, so
+// the chunk gives fields base .. base + 3 of half gq (base = 4 (c & 1) for 2-bit codes,
+// 0 for 4-bit codes).
+template <int BITS>
+__device__ __forceinline__ void v_fields(const uint32_t (&cc)[32], int base, uint32_t (&hv)[8])
+{
+#pragma unroll
+    for (int gq = 0; gq < 8; ++gq) {
+        uint32_t acc = 0u - (magic_sum(BITS, 4) << (BITS * base));
+#pragma unroll
+        for (int n8 = 0; n8 < 4; ++n8)
+            acc += cc[8 * n8 + gq] << (BITS * (base + n8));
+        hv[gq] = acc;
+    }
+}
+
+// One token's codes from its TMEM row, two 32-column chunks per TMEM round trip, stored as
+// the K row (little-endian bit stream, dim j at bit BITS*j) or as the token's halves of
+// its 16-token V tile (with 2-bit codes the chunk pair fills whole halves). row < 0: codes
+// not stored (the warp still takes part in the TMEM loads).
 template <int D, int GS, int NG, int BITS, bool V>
 __device__ __forceinline__ void store_codes(const TcParams &P, long long row, uint32_t taddr,
                                             const float (&zf)[NG], const float (&sf)[NG],
                                             const float (&rc)[NG], float qmax)
 {
     constexpr int NCH = D / 32;
-    uint32_t cur[32];
+    static_assert(NCH % 2 == 0, "chunk pairs");
     unsigned char *vbase = nullptr;
     int tok = 0;
     if (V && row >= 0) {
@@ -216,60 +246,54 @@ __device__ __forceinline__ void store_codes(const TcParams &P, long long row, ui
         tok = (int)(row % kTileTokens);
     }
 #pragma unroll 1
-    for (int c = 0; c < NCH; ++c) {
-        tmem_ld32_async(taddr + 32 * c, cur);
+    for (int c = 0; c < NCH; c += 2) {
+        uint32_t xa[32], xb[32];
+        tmem_ld32_async(taddr + 32 * c, xa);
+        tmem_ld32_async(taddr + 32 * (c + 1), xb);
         tmem_ld_wait();
-        const int gr = (32 * c) / GS;
-        const uint64_t nz2 = f2dup(-pick(zf, gr)), ns2 = f2dup(-pick(sf, gr)),
-                       rc2 = f2dup(pick(rc, gr));
-        // the chunk's 32 codes (magic bit patterns), two adjacent values at a time
-        uint32_t cc[32];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2)
-            code_rn2(cur[e], cur[e + 1], nz2, ns2, rc2, qmax, cc[e], cc[e + 1]);
+        uint32_t ca[32], cb[32];
+        chunk_codes<GS, NG>(xa, c, zf, sf, rc, qmax, ca);
+        chunk_codes<GS, NG>(xb, c + 1, zf, sf, rc, qmax, cb);
         if (!V) {
-            uint32_t w[BITS];
+            // word q of chunk c: dims 32c + (32/BITS) q + e at BITS*e
             constexpr int PER = 32 / BITS;
+            uint32_t w[2 * BITS];
 #pragma unroll
-            for (int q = 0; q < BITS; ++q) {
+            for (int q = 0; q < 2 * BITS; ++q) {
                 uint32_t acc = 0u - magic_sum(BITS, PER);
 #pragma unroll
                 for (int e = 0; e < PER; ++e)
-                    acc += cc[PER * q + e] << (BITS * e);
+                    acc += (q < BITS ? ca[PER * q + e] : cb[PER * (q - BITS) + e]) << (BITS * e);
                 w[q] = acc;
             }
             if (row >= 0) {
-                uint32_t *dst = reinterpret_cast<uint32_t *>(P.k_codes + row * (D * BITS / 8)) + BITS * c;
-                if (BITS == 2)
-                    *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1 % BITS]);
-                else
-                    *reinterpret_cast<uint4 *>(dst) =
-                        make_uint4(w[0], w[1 % BITS], w[2 % BITS], w[3 % BITS]);
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    reinterpret_cast<uint32_t *>(P.k_codes + row * (D * BITS / 8)) + BITS * c);
+                if constexpr (BITS == 2) {
+                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                } else {
+                    dst[0] = make_uint4(w[0], w[1 % (2 * BITS)], w[2 % (2 * BITS)], w[3 % (2 * BITS)]);
+                    dst[1] = make_uint4(w[4 % (2 * BITS)], w[5 % (2 * BITS)], w[6 % (2 * BITS)],
+                                        w[7 % (2 * BITS)]);
+                }
             }
         } else {
-            // The chunk's dims are 32c + 8 n8 + gq (n8 < 4, gq < 8). The half (gq, rr) holds
-            // dims 8(E rr + s) + gq at bits BITS*s, E = 16/BITS: with 4-bit codes chunk c is
-            // all of the halves rr = c; with 2-bit codes chunk c is fields 4(c&1) .. +3 of
-            // the halves rr = c/2, i.e. their byte c&1 (each token owns whole bytes).
-            const int base = BITS == 2 ? 4 * (c & 1) : 0;
-            uint32_t hv[8];
-#pragma unroll
-            for (int gq = 0; gq < 8; ++gq) {
-                uint32_t acc = 0u - (magic_sum(BITS, 4) << (BITS * base));
-#pragma unroll
-                for (int n8 = 0; n8 < 4; ++n8)
-                    acc += cc[8 * n8 + gq] << (BITS * (base + n8));
-                hv[gq] = acc;
-            }
+            uint32_t ha[8], hb[8];
+            v_fields<BITS>(ca, BITS == 2 ? 0 : 0, ha);
+            v_fields<BITS>(cb, BITS == 2 ? 4 : 0, hb);
             if (row >= 0) {
 #pragma unroll
                 for (int gq = 0; gq < 8; ++gq) {
-                    if (BITS == 4)
+                    if constexpr (BITS == 4) {
                         *reinterpret_cast<uint16_t *>(vbase + v_half_offset(D, 4, tok, gq, c)) =
-                            (uint16_t)hv[gq];
-                    else
-                        vbase[v_half_offset(D, 2, tok, gq, c >> 1) + (c & 1)] =
-                            (unsigned char)(hv[gq] >> (8 * (c & 1)));
+                            (uint16_t)ha[gq];
+                        *reinterpret_cast<uint16_t *>(vbase + v_half_offset(D, 4, tok, gq, c + 1)) =
+                            (uint16_t)hb[gq];
+                    } else {
+                        // chunks c (fields 0-3) and c + 1 (fields 4-7) of half rr = c / 2
+                        *reinterpret_cast<uint16_t *>(vbase + v_half_offset(D, 2, tok, gq, c >> 1)) =
+                            (uint16_t)(ha[gq] + hb[gq]);
+                    }
                 }
             }
         }
@@ -670,14 +694,19 @@ append_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 else
                     store_row64<4>(P, which, row, x0, x1, z2, s2, r2, qmax);
             } else {
-                uint32_t cur[32];
+                // pass 1 over chunk pairs: two 32-column loads per TMEM round trip
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    tmem_ld32_async(taddr + 32 * c, cur);
+                for (int c = 0; c < D / 32; c += 2) {
+                    uint32_t xa[32], xb[32];
+                    tmem_ld32_async(taddr + 32 * c, xa);
+                    tmem_ld32_async(taddr + 32 * (c + 1), xb);
                     tmem_ld_wait();
-                    cs.add32(cur, P.clip, quest);
-                    if ((32 * c + 32) % GS == 0)          // the group ends with this chunk
+                    cs.add32(xa, P.clip, quest);
+                    if ((32 * c + 32) % GS == 0)          // the group ends with chunk c
                         finish((32 * c) / GS);
+                    cs.add32(xb, P.clip, quest);
+                    if ((32 * c + 64) % GS == 0)          // ... or with chunk c + 1
+                        finish((32 * c + 32) / GS);
                 }
                 // ---- pass 2: codes
                 if (!which) {
