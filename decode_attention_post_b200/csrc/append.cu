@@ -660,14 +660,11 @@ cudaError_t launch_append_fp32(const void *k, const void *v, int in_bf16, const 
 
 }  // namespace
 
-cudaError_t append_mma(const void *k, const void *v, const float *Tk, const float *Tv, int B,
-                       int n, const kvq_cache *c, int kappa, const int32_t *pos, int32_t *dev_err,
-                       cudaStream_t st);
-
 // Window flush of kvq_window_append: the positions leaving the full-precision window
-// (from the recent ring or the n_new new tokens) through the float32 CUDA-core path; the
-// flattened list holds S_flush * ceil(n_new / S_flush) entries per sequence, the most any
-// sequence can flush in one call.
+// (from the recent ring or the n_new new tokens) through the short tensor-core kernel
+// (both transforms given) or the float32 CUDA-core kernel; the flattened list holds
+// S_flush * ceil(n_new / S_flush) entries per sequence, the most any sequence can flush
+// in one call.
 cudaError_t window_flush_launch(const void *k_new, const void *v_new, const float *Tk,
                                 const float *Tv, int B, int n_new, const kvq_cache *c, int kappa,
                                 const void *ring_k, const void *ring_v, const int32_t *len,
@@ -705,10 +702,9 @@ cudaError_t append_tc(const void *k, const void *v, const float *Tk, const float
                       cudaStream_t st);
 
 // bfloat16 inputs with both transforms: chunks of 256 tokens or more go to the tcgen05
-// tensor-core kernel, shorter (decode-time) appends to the short mma.sync kernel
-// (KVQ_APPEND_PATH=mma / fp32 select the older warp-level chunk kernel or the CUDA-core
-// kernel instead, for comparison); float32 inputs, identity transforms and unaligned
-// inputs use the float32 CUDA-core kernel.
+// tensor-core kernel (which counts tokens in 32 bits), shorter (decode-time) appends to
+// the short mma.sync kernel; float32 inputs, identity transforms, unaligned inputs and
+// chunks beyond 2^31 tokens use the float32 CUDA-core kernel.
 cudaError_t append_launch(const void *k, const void *v, int in_bf16, const float *Tk,
                           const float *Tv, int B, int n, const kvq_cache *c, int kappa,
                           const int32_t *pos, int32_t *dev_err, cudaStream_t st)
@@ -716,14 +712,9 @@ cudaError_t append_launch(const void *k, const void *v, int in_bf16, const float
     const long tokens = (long)B * n;
     const bool a16 = ((uintptr_t)k % 16 == 0) && ((uintptr_t)v % 16 == 0) &&
                      ((uintptr_t)Tk % 16 == 0) && ((uintptr_t)Tv % 16 == 0);
-    const char *path = getenv("KVQ_APPEND_PATH");
-    const bool force_fp32 = path && path[0] == 'f';
-    if (in_bf16 && Tk && Tv && a16 && tokens >= 256 && !force_fp32) {
-        if ((path && path[0] == 'm') || tokens > 0x7fffff00L)
-            return append_mma(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
+    if (in_bf16 && Tk && Tv && a16 && tokens >= 256 && tokens <= 0x7fffff00L)
         return append_tc(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
-    }
-    if (in_bf16 && Tk && Tv && a16 && !force_fp32) {
+    if (in_bf16 && Tk && Tv && a16 && tokens < 256) {
         if (c->d == 64)
             return launch_append_small<64>(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
         return launch_append_small<128>(k, v, Tk, Tv, B, n, c, kappa, pos, dev_err, st);
